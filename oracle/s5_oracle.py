@@ -1,0 +1,263 @@
+"""CPU oracle for the Step 5 Preview sparse and sliding-window attention layers.
+
+TEST INFRASTRUCTURE ONLY.  This module exists to check the CUDA library.  Only
+the test suite, the package smoke check and the benchmark's CPU-baseline leg
+may import it; the library itself never calls it and has no CPU fallback.  It
+shares no code with the CUDA path: it does not import the package, and the
+package does not import it.  Its inputs are plain numpy arrays (or any object
+that supports numpy-style fancy indexing on the first axis, for lazily drawn
+key/value rows).
+
+Everything here is the plain definition, evaluated in float64:
+
+* block scoring and top-512 selection: a full stable sort on the composite key
+  (score descending, block index ascending);
+* attention: the softmax over an explicit token set, one head at a time, with
+  head h reading KV group h // 16.
+
+Sources (the pages give prose and a configuration table, no formulas or code):
+
+[HA]  SGLang day-0 blog "Step 5 Preview: Day-0 Inference and RL Support with
+      SGLang and Miles", section "Hybrid Attention": three of every four layers
+      read the most recent 512 tokens; the fourth scores summaries of 8-token
+      blocks, selects up to 512 historical blocks, and reads the individual
+      tokens of those blocks and of the current block.
+[KS]  same page, section "Kernels from StepFun": indexer scoring of each query
+      against the compressed history in the paged cache; sparse decode splits
+      long histories into partitions and merges partial results.
+[CFG] StepFun open-weights blog, section "What the config says": 64 query
+      heads, 4 KV groups, head dim 192; one 256-dim key per 8-token block; top
+      512 blocks (k = 4,096 tokens); 512-token sliding windows.
+[SAV] same blog, section "What sparse attention does and doesn't save": the
+      indexer scores every block; up to 512 historical blocks plus the current
+      one are read.
+
+Readings taken where the pages are silent (each the plainest one):
+
+* history of a query at absolute position t: the complete blocks 0 .. c-1 with
+  c = t // 8; the current block c is always read, causally (tokens 8c .. t);
+* block score = plain dot product of the 256-dim indexer query with the block
+  key (no normalisation; any monotone map leaves the selection unchanged);
+* selection shared by all four KV groups; ties go to the lower block index;
+  selected indices are reported in ascending order, -1 padded;
+* softmax scale ``sm_scale`` (1/sqrt(192) by default), natural exponent;
+* the sliding window covers positions max(0, t - W + 1) .. t (the query
+  included);
+* outputs rounded to bf16 with round-to-nearest-even directly from float64.
+
+Parity status: block selection is pinned by brute force, tie cases and the
+subset characterisation of top-k; the attention functions are pinned by closed
+forms (one token, identical keys, two tokens), the reduction of sparse and
+sliding-window attention to full causal attention, weight normalisation and
+invariance to the order of the selected blocks.  The pages print no worked
+numerical example, so attention values beyond these properties are pinned only
+by them.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+N_HEADS = 64
+N_KV = 4
+HEADS_PER_GROUP = N_HEADS // N_KV
+HEAD_DIM = 192
+BLOCK = 8
+INDEX_DIM = 256
+TOPK = 512
+WINDOW = 512
+DEFAULT_SM_SCALE = 1.0 / math.sqrt(HEAD_DIM)
+
+
+# ----------------------------------------------------------------------------
+# rounding
+# ----------------------------------------------------------------------------
+
+def round_bf16(x) -> np.ndarray:
+    """Round float64 values to the nearest bf16 value (ties to even), returned
+    as float64.  bf16 keeps 8 significant bits; rounding is done once, from
+    float64, never through float32.  Finite values in the normal range only
+    (attention outputs are bounded by the values they average)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                # x = m * 2**e, 0.5 <= |m| < 1
+    r = np.rint(m * 256.0)            # 8 significant bits; rint rounds halves to even
+    return np.ldexp(r / 256.0, e)
+
+
+# ----------------------------------------------------------------------------
+# indexer: block scores and top-k selection   [HA], [KS], [CFG], [SAV]
+# ----------------------------------------------------------------------------
+
+def current_block(t: int) -> int:
+    """Index of the block that holds position t; blocks before it are history."""
+    return t // BLOCK
+
+
+def block_scores(qx, kx) -> np.ndarray:
+    """score[b] = sum_d qx[d] * kx[b, d] in float64.
+
+    Exact for the integer-valued inputs used in the parity tests (|score| is
+    far below 2**53)."""
+    qx = np.asarray(qx, dtype=np.float64)
+    kx = np.asarray(kx, dtype=np.float64)
+    return kx @ qx
+
+
+def select_topk(scores, topk: int = TOPK) -> np.ndarray:
+    """The ``topk`` largest scores, ties to the lower index, as ascending indices.
+
+    With fewer than ``topk`` candidates every index is returned.  The result is
+    padded with -1 to length ``topk``."""
+    scores = np.asarray(scores, dtype=np.float64)
+    c = scores.shape[0]
+    out = np.full(topk, -1, dtype=np.int64)
+    if c <= topk:
+        out[:c] = np.arange(c)
+        return out
+    idx = np.arange(c)
+    order = np.lexsort((idx, -scores))  # primary: -score ascending; secondary: index ascending
+    out[:] = np.sort(order[:topk])
+    return out
+
+
+def index_topk_query(qx, kx_seq, t: int, topk: int = TOPK) -> np.ndarray:
+    """Selection for one query at absolute position t.
+
+    ``kx_seq[b]`` is the 256-dim key of block b of the query's sequence; only
+    blocks 0 .. t//8 - 1 are scored."""
+    c = current_block(t)
+    if c <= topk:
+        return select_topk(np.zeros(c), topk)
+    return select_topk(block_scores(qx, kx_seq[np.arange(c)]), topk)
+
+
+def selection_count(sel) -> int:
+    sel = np.asarray(sel)
+    return int((sel >= 0).sum())
+
+
+# ----------------------------------------------------------------------------
+# token sets   [HA], [SAV]
+# ----------------------------------------------------------------------------
+
+def sparse_token_set(sel, t: int) -> np.ndarray:
+    """Positions read by a sparse-layer query at t: the 8 tokens of every
+    selected block plus tokens 8c .. t of the current block c = t // 8."""
+    sel = np.asarray(sel, dtype=np.int64)
+    sel = sel[sel >= 0]
+    c = current_block(t)
+    hist = (sel[:, None] * BLOCK + np.arange(BLOCK)[None, :]).reshape(-1)
+    cur = np.arange(c * BLOCK, t + 1)
+    return np.concatenate([hist, cur])
+
+
+def swa_token_set(t: int, window: int = WINDOW) -> np.ndarray:
+    """Positions read by a sliding-window query at t: max(0, t - W + 1) .. t."""
+    return np.arange(max(0, t - window + 1), t + 1)
+
+
+# ----------------------------------------------------------------------------
+# attention over an explicit token set   [HA], [CFG]
+# ----------------------------------------------------------------------------
+
+def gqa_attention(q, k_rows, v_rows, sm_scale: float = DEFAULT_SM_SCALE, return_weights: bool = False):
+    """Grouped-query attention of one query token over an explicit token set.
+
+    q        [64][192]      (head h reads KV group h // 16)
+    k_rows   [n][4][192]    keys of the n tokens of the set
+    v_rows   [n][4][192]    values of the same tokens
+    returns  out float64 [64][192] (not rounded), lse float64 [64]
+             (natural log of the softmax denominator, scores included), and,
+             with ``return_weights``, the softmax weights [64][n].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k_rows = np.asarray(k_rows, dtype=np.float64)
+    v_rows = np.asarray(v_rows, dtype=np.float64)
+    n = k_rows.shape[0]
+    out = np.zeros((N_HEADS, HEAD_DIM))
+    lse = np.full(N_HEADS, -np.inf)
+    weights = np.zeros((N_HEADS, n))
+    if n == 0:
+        return (out, lse, weights) if return_weights else (out, lse)
+    for h in range(N_HEADS):
+        g = h // HEADS_PER_GROUP
+        s = sm_scale * (k_rows[:, g, :] @ q[h])   # s_j = scale * q . k_j
+        m = s.max()
+        w = np.exp(s - m)
+        l = w.sum()
+        p = w / l
+        out[h] = p @ v_rows[:, g, :]
+        lse[h] = m + math.log(l)
+        weights[h] = p
+    return (out, lse, weights) if return_weights else (out, lse)
+
+
+def sparse_attention_query(q, sel, t: int, k_seq, v_seq, sm_scale: float = DEFAULT_SM_SCALE):
+    """Sparse-layer attention of one query at t over its selected blocks and
+    current block.  ``k_seq[pos]`` / ``v_seq[pos]`` give [4][192] rows of the
+    query's sequence (fancy indexing on positions)."""
+    T = sparse_token_set(sel, t)
+    return gqa_attention(q, k_seq[T], v_seq[T], sm_scale)
+
+
+def swa_attention_query(q, t: int, k_seq, v_seq, window: int = WINDOW, sm_scale: float = DEFAULT_SM_SCALE):
+    """Sliding-window attention of one query at t."""
+    T = swa_token_set(t, window)
+    return gqa_attention(q, k_seq[T], v_seq[T], sm_scale)
+
+
+# ----------------------------------------------------------------------------
+# batched drivers (varlen batches: per sequence, ctx cached tokens, then nq queries)
+# ----------------------------------------------------------------------------
+
+def query_positions(ctx, nq):
+    """(sequence, position) of every query row, rows ordered by sequence."""
+    rows = []
+    for s, (c, n) in enumerate(zip(ctx, nq)):
+        for j in range(n):
+            rows.append((s, c + j))
+    return rows
+
+
+def index_topk_batch(qx, kx_of_seq, ctx, nq, topk: int = TOPK, rows=None):
+    """Selections [n_rows][topk] (-1 padded) and counts for the given rows.
+
+    ``kx_of_seq(s)`` returns an array indexable by block ids of sequence s."""
+    pos = query_positions(ctx, nq)
+    rows = range(len(pos)) if rows is None else rows
+    sel, cnt = [], []
+    for r in rows:
+        s, t = pos[r]
+        x = index_topk_query(qx[r], kx_of_seq(s), t, topk)
+        sel.append(x)
+        cnt.append(selection_count(x))
+    return np.array(sel, dtype=np.int64).reshape(-1, topk), np.array(cnt, dtype=np.int64)
+
+
+def sparse_attention_batch(q, sel, ctx, nq, kv_of_seq, sm_scale: float = DEFAULT_SM_SCALE, rows=None):
+    """Sparse attention for the given rows: (out [n][64][192], lse [n][64])."""
+    pos = query_positions(ctx, nq)
+    rows = list(range(len(pos))) if rows is None else list(rows)
+    outs, lses = [], []
+    for i, r in enumerate(rows):
+        s, t = pos[r]
+        k_seq, v_seq = kv_of_seq(s)
+        o, l = sparse_attention_query(q[i], sel[i], t, k_seq, v_seq, sm_scale)
+        outs.append(o)
+        lses.append(l)
+    return np.array(outs), np.array(lses)
+
+
+def swa_attention_batch(q, ctx, nq, kv_of_seq, window: int = WINDOW, sm_scale: float = DEFAULT_SM_SCALE, rows=None):
+    """Sliding-window attention for the given rows: (out [n][64][192], lse [n][64])."""
+    pos = query_positions(ctx, nq)
+    rows = list(range(len(pos))) if rows is None else list(rows)
+    outs, lses = [], []
+    for i, r in enumerate(rows):
+        s, t = pos[r]
+        k_seq, v_seq = kv_of_seq(s)
+        o, l = swa_attention_query(q[i], t, k_seq, v_seq, window, sm_scale)
+        outs.append(o)
+        lses.append(l)
+    return np.array(outs), np.array(lses)

@@ -1,0 +1,403 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: brute force,
+an independent characterisation, a closed form, an invariant, or a value the
+pages print.  A plausible mistake in the oracle (a dropped term, a wrong sign,
+a wrong head-to-group map, an off-by-one in the window or the current block,
+a wrong tie-break) fails at least one of them.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import s5_oracle as O
+
+RNG = np.random.default_rng(12345)
+
+
+# ---------------------------------------------------------------- rounding
+
+def test_round_bf16_ties_and_double_rounding():
+    one = 1.0
+    assert O.round_bf16(one) == 1.0
+    # halfway between 1 and 1 + 2**-7 -> even (1.0)
+    assert O.round_bf16(1 + 2 ** -8) == 1.0
+    # halfway between 1 + 2**-7 and 1 + 2**-6 -> even (1 + 2**-6)
+    assert O.round_bf16(1 + 3 * 2 ** -8) == 1 + 2 ** -6
+    # just above the halfway point: rounding through float32 would drop the
+    # 2**-30 and tie to 1.0; rounding once from float64 goes up
+    assert O.round_bf16(1 + 2 ** -8 + 2 ** -30) == 1 + 2 ** -7
+    assert O.round_bf16(-(1 + 2 ** -8 + 2 ** -30)) == -(1 + 2 ** -7)
+    assert O.round_bf16(0.0) == 0.0
+
+
+def test_round_bf16_matches_library_on_float32_values():
+    # for values already in float32, one rounding to bf16 is what torch does
+    x = (RNG.standard_normal(20000) * 10.0 ** RNG.uniform(-3, 3, 20000)).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.round_bf16(x.astype(np.float64)), ref)
+
+
+# ---------------------------------------------------------------- selection
+
+def _naive_topk(scores, k):
+    """Repeated max extraction, scanning in index order with a strict '>'
+    so the lower index wins a tie."""
+    scores = list(scores)
+    taken = [False] * len(scores)
+    out = []
+    for _ in range(min(k, len(scores))):
+        best = -1
+        for i, s in enumerate(scores):
+            if taken[i]:
+                continue
+            if best < 0 or s > scores[best]:
+                best = i
+        taken[best] = True
+        out.append(best)
+    return sorted(out)
+
+
+def _subset_characterisation(scores, k):
+    """The unique k-subset S with: every member beats every non-member
+    (higher score, or equal score and lower index)."""
+    c = len(scores)
+    found = []
+    for S in itertools.combinations(range(c), k):
+        inside = set(S)
+        ok = all((scores[x] > scores[y]) or (scores[x] == scores[y] and x < y)
+                 for x in inside for y in range(c) if y not in inside)
+        if ok:
+            found.append(list(S))
+    assert len(found) == 1
+    return found[0]
+
+
+@pytest.mark.parametrize("trial", range(40))
+def test_select_topk_brute_force(trial):
+    c = int(RNG.integers(1, 40))
+    k = int(RNG.choice([1, 3, 8]))
+    scores = RNG.integers(-3, 4, c).astype(np.float64)  # many ties
+    got = O.select_topk(scores, k)
+    want = _naive_topk(scores, k)
+    assert list(got[:len(want)]) == want
+    assert np.all(got[len(want):] == -1)
+
+
+@pytest.mark.parametrize("trial", range(25))
+def test_select_topk_subset_definition(trial):
+    c = int(RNG.integers(5, 12))
+    k = int(RNG.integers(1, 5))
+    scores = RNG.integers(-2, 3, c).astype(np.float64)
+    got = O.select_topk(scores, k)
+    assert list(got) == _subset_characterisation(list(scores), k)
+
+
+def test_select_topk_tie_cases():
+    # all equal -> the first 512 blocks
+    assert list(O.select_topk(np.zeros(2000), 512)) == list(range(512))
+    # strictly decreasing -> the first 512
+    assert list(O.select_topk(-np.arange(2000.0), 512)) == list(range(512))
+    # strictly increasing -> the last 512
+    assert list(O.select_topk(np.arange(2000.0), 512)) == list(range(1488, 2000))
+    # a tie straddling the cut: 500 clear winners, then ties broken by index
+    s = np.zeros(3000)
+    winners = RNG.choice(3000, 500, replace=False)
+    s[winners] = 10
+    got = O.select_topk(s, 512)
+    rest = [i for i in range(3000) if i not in set(winners.tolist())][:12]
+    assert list(got) == sorted(winners.tolist() + rest)
+
+
+def test_select_topk_short_history_takes_all():
+    for c in [0, 1, 7, 511, 512]:
+        got = O.select_topk(RNG.standard_normal(c), 512)
+        assert list(got[:c]) == list(range(c))
+        assert np.all(got[c:] == -1)
+
+
+def test_index_topk_scores_only_history_blocks():
+    # blocks at or after the current block must never be scored
+    c_t = 600  # t in block 600
+    t = c_t * 8 + 5
+    kx = RNG.integers(-4, 5, (c_t + 10, 256)).astype(np.float64)
+    qx = RNG.integers(-4, 5, 256).astype(np.float64)
+    kx[c_t:] = 4 * np.sign(qx)  # make the future/current blocks score highest
+    sel = O.index_topk_query(qx, kx, t, 512)
+    assert sel.max() < c_t and len(set(sel.tolist())) == 512
+    scores = kx[:c_t] @ qx
+    assert list(sel) == _naive_topk(scores, 512)
+
+
+def test_block_scores_exact_integers():
+    kx = RNG.integers(-4, 5, (1000, 256))
+    qx = RNG.integers(-4, 5, 256)
+    want = kx.astype(np.int64) @ qx.astype(np.int64)
+    got = O.block_scores(qx.astype(np.float64), kx.astype(np.float64))
+    assert np.array_equal(got, want.astype(np.float64))
+
+
+# ---------------------------------------------------------------- token sets
+
+@pytest.mark.parametrize("trial", range(20))
+def test_sparse_token_set_membership(trial):
+    t = int(RNG.integers(0, 6000))
+    c = t // 8
+    n = min(512, c)
+    sel = np.sort(RNG.choice(c, n, replace=False)) if c else np.zeros(0, np.int64)
+    T = set(O.sparse_token_set(sel, t).tolist())
+    sset = set(sel.tolist())
+    for p in range(0, t + 20):
+        inside = (p // 8 in sset) or (p // 8 == c and p <= t)
+        assert (p in T) == inside, (p, t)
+    assert len(T) == len(O.sparse_token_set(sel, t))  # no duplicates
+
+
+def test_swa_token_set_edges():
+    assert list(O.swa_token_set(0, 512)) == [0]
+    assert list(O.swa_token_set(511, 512)) == list(range(0, 512))
+    assert list(O.swa_token_set(512, 512)) == list(range(1, 513))
+    assert len(O.swa_token_set(100000, 512)) == 512
+
+
+# ---------------------------------------------------------------- attention closed forms
+
+def _rand(*shape):
+    return RNG.standard_normal(shape)
+
+
+def test_single_token_returns_its_value():
+    q = _rand(64, 192)
+    k = _rand(1, 4, 192)
+    v = _rand(1, 4, 192)
+    out, lse = O.gqa_attention(q, k, v, 0.1)
+    for h in range(64):
+        assert np.allclose(out[h], v[0, h // 16], atol=0, rtol=0)
+        assert math.isclose(lse[h], 0.1 * float(q[h] @ k[0, h // 16]), rel_tol=1e-14, abs_tol=1e-14)
+
+
+def test_identical_keys_average_values():
+    q = _rand(64, 192)
+    k1 = _rand(1, 4, 192)
+    k = np.repeat(k1, 37, axis=0)
+    v = _rand(37, 4, 192)
+    out, lse = O.gqa_attention(q, k, v, 0.07)
+    for h in range(64):
+        g = h // 16
+        assert np.allclose(out[h], v[:, g].mean(axis=0), rtol=1e-13, atol=1e-13)
+        assert math.isclose(lse[h], 0.07 * float(q[h] @ k1[0, g]) + math.log(37), rel_tol=1e-13)
+
+
+def test_two_tokens_sigmoid_weights():
+    # k0 = e_0, k1 = 0; q_h = x_h * e_0 -> weight of token 0 is sigmoid(scale * x_h)
+    q = np.zeros((64, 192))
+    x = RNG.uniform(-5, 5, 64)
+    q[:, 0] = x
+    k = np.zeros((2, 4, 192))
+    k[0, :, 0] = 1.0
+    v = np.zeros((2, 4, 192))
+    v[0] = 1.0
+    scale = 0.3
+    out, lse = O.gqa_attention(q, k, v, scale)
+    sig = 1.0 / (1.0 + np.exp(-scale * x))
+    assert np.allclose(out, np.repeat(sig[:, None], 192, axis=1), rtol=1e-13, atol=1e-15)
+    assert np.allclose(lse, np.log(np.exp(scale * x) + 1.0), rtol=1e-13)
+
+
+def test_head_reads_group_h_div_16():
+    # each group's values are the constant g + 1; head h must return g(h) + 1
+    q = _rand(64, 192)
+    k = _rand(9, 4, 192)
+    v = np.zeros((9, 4, 192))
+    for g in range(4):
+        v[:, g] = g + 1
+    out, _ = O.gqa_attention(q, k, v, 0.1)
+    for h in range(64):
+        assert np.allclose(out[h], h // 16 + 1, rtol=1e-14)
+
+
+def test_weights_sum_to_one_and_positive():
+    q = _rand(64, 192)
+    k = _rand(300, 4, 192)
+    v = _rand(300, 4, 192)
+    _, _, w = O.gqa_attention(q, k, v, O.DEFAULT_SM_SCALE, return_weights=True)
+    assert np.all(w > 0)
+    assert np.allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+
+
+def test_zero_scale_is_uniform_average():
+    q = _rand(64, 192)
+    k = _rand(50, 4, 192)
+    v = _rand(50, 4, 192)
+    out, lse = O.gqa_attention(q, k, v, 0.0)
+    for h in range(64):
+        assert np.allclose(out[h], v[:, h // 16].mean(axis=0), rtol=1e-13, atol=1e-14)
+    assert np.allclose(lse, math.log(50), rtol=1e-14)
+
+
+def test_lse_is_log_sum_exp_of_scores():
+    q = _rand(64, 192) * 0.1
+    k = _rand(20, 4, 192)
+    v = _rand(20, 4, 192)
+    _, lse = O.gqa_attention(q, k, v, 0.5)
+    for h in range(64):
+        s = 0.5 * (k[:, h // 16] @ q[h])
+        assert math.isclose(lse[h], math.log(sum(math.exp(x) for x in s)), rel_tol=1e-12)
+
+
+def test_scale_shift_invariance():
+    # adding the same amount to every score leaves the output unchanged
+    q = _rand(64, 192)
+    k = _rand(40, 4, 192)
+    v = _rand(40, 4, 192)
+    out1, lse1 = O.gqa_attention(q, k, v, 0.1)
+    kb = k + 0.0
+    # shift every key by a vector orthogonal to nothing in particular: use q-dependent shift
+    # per group, k_j + u_g changes s_j by scale * q_h . u_g, the same for all j
+    u = _rand(4, 192)
+    kb = k + u[None]
+    out2, lse2 = O.gqa_attention(q, kb, v, 0.1)
+    assert np.allclose(out1, out2, rtol=1e-11, atol=1e-12)
+    for h in range(64):
+        assert math.isclose(lse2[h] - lse1[h], 0.1 * float(q[h] @ u[h // 16]), rel_tol=1e-9, abs_tol=1e-11)
+
+
+# ---------------------------------------------------------------- invariants of the layers
+
+def _full_causal(q, k_seq, v_seq, t, scale):
+    """Full causal attention over positions 0..t, written with the group map
+    applied by repeating KV groups to heads (a different formulation)."""
+    K = np.repeat(k_seq[: t + 1], 16, axis=1)   # [n][64][192]
+    V = np.repeat(v_seq[: t + 1], 16, axis=1)
+    s = scale * np.einsum("hd,nhd->hn", q, K)
+    w = np.exp(s)
+    w /= w.sum(axis=1, keepdims=True)
+    return np.einsum("hn,nhd->hd", w, V)
+
+
+@pytest.mark.parametrize("t", [0, 5, 7, 8, 63, 64, 200, 4095])
+def test_sparse_equals_full_when_history_fits(t):
+    # c = t // 8 <= 512: every history block is selected
+    L = t + 1
+    k_seq = _rand(L, 4, 192)
+    v_seq = _rand(L, 4, 192)
+    q = _rand(64, 192)
+    kx = RNG.integers(-4, 5, (L // 8 + 1, 256)).astype(np.float64)
+    qx = RNG.integers(-4, 5, 256).astype(np.float64)
+    sel = O.index_topk_query(qx, kx, t, 512)
+    out, _ = O.sparse_attention_query(q, sel, t, k_seq, v_seq, 0.08)
+    assert np.allclose(out, _full_causal(q, k_seq, v_seq, t, 0.08), rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("t,window", [(0, 512), (100, 512), (511, 512), (700, 701), (50, 4096)])
+def test_swa_equals_full_when_window_covers(t, window):
+    k_seq = _rand(t + 1, 4, 192)
+    v_seq = _rand(t + 1, 4, 192)
+    q = _rand(64, 192)
+    out, _ = O.swa_attention_query(q, t, k_seq, v_seq, window, 0.08)
+    assert np.allclose(out, _full_causal(q, k_seq, v_seq, t, 0.08), rtol=1e-11, atol=1e-12)
+
+
+def test_swa_excludes_tokens_outside_window():
+    t, W = 900, 512
+    k_seq = _rand(t + 1, 4, 192)
+    v_seq = _rand(t + 1, 4, 192)
+    q = _rand(64, 192)
+    out1, _ = O.swa_attention_query(q, t, k_seq, v_seq, W, 0.1)
+    k2, v2 = k_seq.copy(), v_seq.copy()
+    k2[: t - W + 1] = 50.0  # would dominate if read
+    v2[: t - W + 1] = 1e6
+    out2, _ = O.swa_attention_query(q, t, k2, v2, W, 0.1)
+    assert np.array_equal(out1, out2)
+    # and the oldest in-window token is read
+    k3 = k_seq.copy()
+    k3[t - W + 1] = 3.0 * q.mean(axis=0) / 16
+    out3, _ = O.swa_attention_query(q, t, k3, v_seq, W, 0.1)
+    assert not np.allclose(out1, out3)
+
+
+def test_sparse_order_invariance():
+    t = 8 * 3000 + 3
+    L = t + 1
+    k_seq = _rand(L, 4, 192)
+    v_seq = _rand(L, 4, 192)
+    q = _rand(64, 192)
+    sel = np.sort(RNG.choice(3000, 512, replace=False))
+    out1, lse1 = O.sparse_attention_query(q, sel, t, k_seq, v_seq, 0.07)
+    perm = RNG.permutation(sel)
+    out2, lse2 = O.sparse_attention_query(q, perm, t, k_seq, v_seq, 0.07)
+    assert np.allclose(out1, out2, rtol=1e-12, atol=1e-12)
+    assert np.allclose(lse1, lse2, rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_causal_within_current_block():
+    t = 8 * 700 + 2  # three tokens of the current block are visible
+    L = t + 6
+    k_seq = _rand(L, 4, 192)
+    v_seq = _rand(L, 4, 192)
+    q = _rand(64, 192)
+    sel = np.sort(RNG.choice(700, 512, replace=False))
+    out1, _ = O.sparse_attention_query(q, sel, t, k_seq, v_seq, 0.1)
+    k2, v2 = k_seq.copy(), v_seq.copy()
+    k2[t + 1:] = 40.0
+    v2[t + 1:] = 1e6
+    out2, _ = O.sparse_attention_query(q, sel, t, k2, v2, 0.1)
+    assert np.array_equal(out1, out2)
+    # an unselected history block is never read
+    unsel = sorted(set(range(700)) - set(sel.tolist()))[0]
+    k2[unsel * 8: unsel * 8 + 8] = 40.0
+    v2[unsel * 8: unsel * 8 + 8] = 1e6
+    out3, _ = O.sparse_attention_query(q, sel, t, k2, v2, 0.1)
+    assert np.array_equal(out1, out3)
+
+
+def test_batch_driver_rows():
+    ctx, nq = [20, 5000], [2, 3]
+    rows = O.query_positions(ctx, nq)
+    assert rows == [(0, 20), (0, 21), (1, 5000), (1, 5001), (1, 5002)]
+
+
+# ---------------------------------------------------------------- the pages' arithmetic
+
+def _golden(name):
+    path = os.path.join(os.path.dirname(__file__), "golden", name)
+    out = {}
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        parts = [p.strip() for p in line.split("|")]
+        out[parts[0]] = (float(parts[1]), float(parts[3]))
+    return out
+
+
+def test_bytes_model_reproduces_pages():
+    from block_sparse_gqa_indexer_b200 import roofline as R
+    g = _golden("pages_byte_arithmetic.txt")
+    got = {
+        "kv_bytes_per_token_layer": R.kv_bytes_per_token(),
+        "kv_bytes_per_token_23": R.model_kv_bytes_per_token(),
+        "session_128k": R.session_kv_bytes(128 * 1024),
+        "session_1m": R.session_kv_bytes(1 << 20),
+        "swa_69_layers": R.swa_resident_bytes(),
+        "index_key_overhead": R.index_key_overhead(),
+        "selected_1m_23_layers": R.selected_bytes_per_step(),
+        "blocks_per_layer_1m": (1 << 20) // 8,
+        "indexer_1m_1byte": R.indexer_bytes_per_step(1 << 20, 1),
+        "indexer_1m_2byte": R.indexer_bytes_per_step(1 << 20, 2),
+        "dense_1m": R.session_kv_bytes(1 << 20),
+    }
+    assert set(got) == set(g)
+    for k, (val, tol) in g.items():
+        assert abs(got[k] - val) <= tol * val + 1e-9, (k, got[k], val)
+
+
+def test_sparse_tokens_bounds():
+    from block_sparse_gqa_indexer_b200 import roofline as R
+    # a query reads 4,097 .. 4,104 tokens once 512 history blocks exist
+    assert {R.sparse_tokens(8 * 5000 + j) for j in range(8)} == set(range(4097, 4105))
+    assert R.sparse_tokens(0) == 1
+    assert R.scored_blocks(8 * 512 + 7) == 0 and R.scored_blocks(8 * 513) == 513

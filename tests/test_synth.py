@@ -1,0 +1,84 @@
+"""Host checks of the seeded input generator and the paged layout it builds."""
+import numpy as np
+import torch
+
+from block_sparse_gqa_indexer_b200 import synth as S
+
+
+def test_counter_hash_reference_values():
+    # mul32 against Python's exact integers
+    a = torch.tensor([0, 1, 0xFFFFFFFF, 0x12345678, 0xDEADBEEF], dtype=torch.int64)
+    for b in [0x85EBCA6B, 0xC2B2AE35, 1, 0xFFFFFFFF]:
+        got = S._mul32(a, b).tolist()
+        assert got == [(int(x) * b) & 0xFFFFFFFF for x in a.tolist()]
+
+
+def _fmix32_py(h):
+    h ^= h >> 16
+    h = (h * 0x85EBCA6B) & 0xFFFFFFFF
+    h ^= h >> 13
+    h = (h * 0xC2B2AE35) & 0xFFFFFFFF
+    h ^= h >> 16
+    return h
+
+
+def test_fmix32_matches_definition():
+    xs = [0, 1, 2, 0x7FFFFFFF, 0x80000000, 0xFFFFFFFF, 123456789]
+    got = S._fmix32(torch.tensor(xs, dtype=torch.int64)).tolist()
+    assert got == [_fmix32_py(x) for x in xs]
+    assert _fmix32_py(0) == 0 and _fmix32_py(1) == 0x514E28B7  # MurmurHash3 fmix32(1)
+
+
+def test_uniform_and_normal_moments():
+    idx = torch.arange(1 << 20, dtype=torch.int64)
+    u = S.uniform_int(9, 2, idx, -4, 4)
+    assert int(u.min()) == -4 and int(u.max()) == 4
+    counts = torch.bincount(u + 4).double()
+    assert float((counts / counts.mean() - 1).abs().max()) < 0.02
+    x = S.normal_bf16(9, 3, idx).double()
+    assert abs(float(x.mean())) < 0.01 and abs(float(x.std()) - 1) < 0.01
+    assert float(x.abs().max()) < 3.5  # Irwin-Hall(4) support is +-sqrt(12)
+
+
+def test_generator_is_deterministic_and_seed_dependent():
+    idx = torch.arange(5000, dtype=torch.int64)
+    a = S.normal_bf16(1, 3, idx)
+    assert torch.equal(a, S.normal_bf16(1, 3, idx))
+    assert not torch.equal(a, S.normal_bf16(2, 3, idx))
+    assert not torch.equal(a, S.normal_bf16(1, 4, idx))
+
+
+def test_paged_pools_hold_logical_values():
+    w = S.Workload(ctx=[130, 0, 77], nq=[3, 2, 1], seed=5)
+    pt = w.page_table()
+    assert sorted(pt[pt >= 0].tolist()) == list(range(w.num_pages))
+    k, v = w.kv_pools("cpu", pt)
+    ip = w.index_pool("cpu", pt)
+    for s in range(w.batch):
+        L = w.lens[s]
+        pos = torch.arange(L)
+        kk, vv = w.k_tokens(s, pos), w.v_tokens(s, pos)
+        for p in range(L):
+            page = int(pt[s, p // 64])
+            assert torch.equal(k[page, :, p % 64], kk[p])
+            assert torch.equal(v[page, :, p % 64], vv[p])
+        blocks = torch.arange(L // 8)
+        kb = w.kx_blocks(s, blocks)
+        for b in range(L // 8):
+            assert torch.equal(ip[int(pt[s, b // 8]), b % 8], kb[b])
+    # index values are small integers
+    assert set(torch.unique(ip.float()).tolist()) <= set(range(-4, 5))
+
+
+def test_config_shapes():
+    assert S.config_workloads(1)[0].ctx == [16384]
+    w2 = S.config_workloads(2)[0]
+    assert w2.batch == 64 and all(1024 <= c <= 131072 for c in w2.ctx)
+    w3 = S.config_workloads(3)[0]
+    assert w3.total_q == 256 and all(32768 <= c <= 131072 for c in w3.ctx)
+    w4 = S.config_workloads(4)[0]
+    assert w4.ctx == [114688] and w4.nq == [16384]
+    w5 = S.config_workloads(5)
+    assert len(w5) == 4 and w5[0].ctx == [1 << 20] * 4
+    # different layers draw different values
+    assert not torch.equal(w5[0].k_tokens(0, torch.arange(4)), w5[1].k_tokens(0, torch.arange(4)))
