@@ -1,0 +1,328 @@
+// C ABI of the s5attn library: argument checks, workspace layout, TMA
+// descriptors and launch selection.  Every entry point here is declared in
+// include/s5attn.h, which states the semantics, layouts and error rules.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "s5_common.cuh"
+#include "s5_kernels.h"
+
+using namespace s5;
+
+namespace {
+
+constexpr int kAbiVersion = 100;
+constexpr int kSelCap = 16384;      // one-stage select keeps a row's keys in shared memory
+constexpr int kSeg = 8192;          // two-stage select: blocks per segment
+constexpr int kMaxSeg = 32;         // ... and segments per row (kSeg * kMaxSeg >= S5_MAX_LEN / 8)
+constexpr int kTargetCtas = 2048;   // attention CTAs to aim for (~7 waves of 2 CTAs x 148 SMs)
+constexpr int kMaxSplit = 32;
+constexpr int kScorePagesPerCta = 64;  // indexer CTA: 64 pages = 512 block keys = 256 KB
+
+static_assert((long long)kSeg * kMaxSeg >= S5_MAX_LEN / S5_BLOCK_SIZE, "segments must cover the longest row");
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Longest history of any row: a query at t < max_len has c = t / 8 <= (max_len - 1) / 8 blocks.
+int max_blocks(const s5_batch_desc *b) {
+  const int h = b->max_len >= 1 ? (b->max_len - 1) / kBlk : 0;
+  return h > 1 ? h : 1;
+}
+
+// ---------------------------------------------------------------- argument checks
+
+s5_status check_batch(const s5_batch_desc *b) {
+  if (b == nullptr) return S5_ERR_INVALID_ARG;
+  if (b->batch < 1 || b->max_pages < 1 || b->total_q < 0 || b->max_q < 0 || b->max_len < 0)
+    return S5_ERR_INVALID_ARG;
+  if (b->max_len > S5_MAX_LEN) return S5_ERR_UNSUPPORTED;
+  if ((long long)b->max_pages * kPage < (long long)b->max_len) return S5_ERR_INVALID_ARG;
+  if (b->total_q > 0 && (b->max_q < 1 || b->max_len < 1)) return S5_ERR_INVALID_ARG;
+  if (b->page_table == nullptr || b->ctx_lens == nullptr || b->cu_q == nullptr) return S5_ERR_INVALID_ARG;
+  if ((long long)b->total_q * kHeads > 0x7fffffffLL) return S5_ERR_UNSUPPORTED;
+  return S5_OK;
+}
+
+s5_status check_kv(const s5_kv_desc *kv) {
+  if (kv == nullptr || kv->k_pool == nullptr || kv->v_pool == nullptr) return S5_ERR_INVALID_ARG;
+  if (kv->page_size != kPage || kv->n_kv_heads != kKv || kv->head_dim != kD) return S5_ERR_UNSUPPORTED;
+  if (kv->num_pages < 1) return S5_ERR_INVALID_ARG;
+  if ((long long)kv->num_pages * kKv * kPage >= (1LL << 31)) return S5_ERR_UNSUPPORTED;
+  if (!aligned16(kv->k_pool) || !aligned16(kv->v_pool)) return S5_ERR_INVALID_ARG;
+  return S5_OK;
+}
+
+// ---------------------------------------------------------------- workspace layout
+
+struct IndexWs {
+  size_t scores, cand_key, cand_idx, end;
+  int stride, n_seg;
+  bool two_stage;
+};
+
+IndexWs index_ws(const s5_batch_desc *b) {
+  IndexWs w{};
+  w.stride = max_blocks(b);
+  w.two_stage = w.stride > kSelCap;
+  w.n_seg = w.two_stage ? (w.stride + kSeg - 1) / kSeg : 0;
+  size_t off = kWsHeader;
+  w.scores = off;
+  off = align_up(off + (size_t)b->total_q * w.stride * sizeof(float), 256);
+  w.cand_key = off;
+  off = align_up(off + (size_t)b->total_q * w.n_seg * kMaxTopk * sizeof(uint32_t), 256);
+  w.cand_idx = off;
+  off = align_up(off + (size_t)b->total_q * w.n_seg * kMaxTopk * sizeof(int32_t), 256);
+  w.end = off;
+  return w;
+}
+
+// Partitions per (row, group): enough CTAs to fill the GPU, each warp at least
+// two block pairs, and no CTA owning more than kMaxList blocks.
+int choose_split(int total_q, int blocks_per_row) {
+  const int units = total_q * kKv;
+  int n = (kTargetCtas + units / 2) / (units > 0 ? units : 1);
+  const int by_work = blocks_per_row / (4 * 4);  // 4 warps x 2 pairs x 2 blocks
+  n = n < by_work ? n : by_work;
+  n = n > kMaxSplit ? kMaxSplit : n;
+  const int by_list = (blocks_per_row + kMaxList - 1) / kMaxList;
+  if (n < by_list) n = by_list;
+  return n < 1 ? 1 : n;
+}
+
+struct AttnWs {
+  size_t part_o, part_lse, end;
+  int n_split;
+};
+
+AttnWs attn_ws(const s5_batch_desc *b, int blocks_per_row) {
+  AttnWs w{};
+  w.n_split = choose_split(b->total_q, blocks_per_row);
+  size_t off = kWsHeader;
+  w.part_o = off;
+  if (w.n_split > 1) {
+    off = align_up(off + (size_t)b->total_q * kHeads * w.n_split * kD * sizeof(float), 256);
+    w.part_lse = off;
+    off = align_up(off + (size_t)b->total_q * kHeads * w.n_split * sizeof(float), 256);
+  } else {
+    w.part_lse = off;
+  }
+  w.end = off;
+  return w;
+}
+
+int sparse_blocks_per_row(int topk) { return topk + 1; }
+int swa_blocks_per_row(const s5_batch_desc *b, int window) {
+  long long w = window < b->max_len ? window : b->max_len;
+  return (int)((w + kBlk - 1) / kBlk + 1);
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// A pool bf16 [num_pages][4][64][192] viewed as rows of 192 = 3 x 64 elements;
+// one box is one 8-token block of one group: {64, 3, 8}, 128-byte swizzle.
+bool make_kv_map(CUtensorMap *m, const void *pool, int num_pages) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {64, 3, (cuuint64_t)num_pages * kKv * kPage};
+  cuuint64_t strides[2] = {128, (cuuint64_t)kD * 2};
+  cuuint32_t box[3] = {64, 3, (cuuint32_t)kBlk};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(pool), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+s5_status cuda_status(cudaError_t e) { return e == cudaSuccess ? S5_OK : S5_ERR_CUDA; }
+
+s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, const void *q, const int32_t *sel,
+                      const int32_t *sel_count, int32_t topk, int32_t window, float sm_scale, void *out,
+                      float *lse, void *ws, size_t ws_bytes, cudaStream_t stream) {
+  s5_status st = check_batch(b);
+  if (st != S5_OK) return st;
+  if ((st = check_kv(kv)) != S5_OK) return st;
+  if (!std::isfinite(sm_scale)) return S5_ERR_INVALID_ARG;
+  if (mode == kModeSparse && (topk < 1 || topk > kMaxTopk)) return S5_ERR_INVALID_ARG;
+  if (mode == kModeSwa && window < 1) return S5_ERR_INVALID_ARG;
+  if (ws == nullptr) return S5_ERR_WORKSPACE;
+  if (b->total_q == 0) return S5_OK;
+  if (q == nullptr || out == nullptr || !aligned16(q) || !aligned16(out)) return S5_ERR_INVALID_ARG;
+  if (mode == kModeSparse && (sel == nullptr || sel_count == nullptr)) return S5_ERR_INVALID_ARG;
+  const int bpr = (mode == kModeSparse) ? sparse_blocks_per_row(topk) : swa_blocks_per_row(b, window);
+  const AttnWs w = attn_ws(b, bpr);
+  if (ws_bytes < w.end) return S5_ERR_WORKSPACE;
+  CUtensorMap tk, tv;
+  if (!make_kv_map(&tk, kv->k_pool, kv->num_pages) || !make_kv_map(&tv, kv->v_pool, kv->num_pages))
+    return S5_ERR_CUDA;
+  AttnArgs a{};
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  a.q = q;
+  a.sel = sel;
+  a.sel_count = sel_count;
+  a.topk = topk;
+  a.window = window;
+  a.page_table = b->page_table;
+  a.max_pages = b->max_pages;
+  a.ctx_lens = b->ctx_lens;
+  a.cu_q = b->cu_q;
+  a.batch = b->batch;
+  a.max_len = b->max_len;
+  a.num_pages = kv->num_pages;
+  a.scale_log2 = sm_scale * 1.4426950408889634f;
+  a.n_split = w.n_split;
+  a.out = out;
+  a.lse = lse;
+  a.part_o = reinterpret_cast<float *>(wsb + w.part_o);
+  a.part_lse = reinterpret_cast<float *>(wsb + w.part_lse);
+  a.err = reinterpret_cast<int32_t *>(ws);
+  return cuda_status(launch_gqa_decode(mode, a, tk, tv, b->total_q, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+s5_status s5_workspace_size(const s5_batch_desc *batch, int32_t window, size_t *bytes) {
+  if (bytes == nullptr) return S5_ERR_INVALID_ARG;
+  s5_status st = check_batch(batch);
+  if (st != S5_OK) return st;
+  if (window < 0) return S5_ERR_INVALID_ARG;
+  size_t need = index_ws(batch).end;
+  const size_t sp = attn_ws(batch, sparse_blocks_per_row(kMaxTopk)).end;
+  if (sp > need) need = sp;
+  if (window > 0) {
+    const size_t sw = attn_ws(batch, swa_blocks_per_row(batch, window)).end;
+    if (sw > need) need = sw;
+  }
+  *bytes = need;
+  return S5_OK;
+}
+
+s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *batch, const void *q_index,
+                              int32_t topk, int32_t *sel, int32_t *sel_count, void *workspace,
+                              size_t workspace_bytes, s5_stream_t stream) {
+  s5_status st = check_batch(batch);
+  if (st != S5_OK) return st;
+  if (index == nullptr || index->key_pool == nullptr || index->num_pages < 1) return S5_ERR_INVALID_ARG;
+  if (index->index_dim != kDx) return S5_ERR_UNSUPPORTED;
+  if (!aligned16(index->key_pool)) return S5_ERR_INVALID_ARG;
+  if (topk < 1 || topk > kMaxTopk) return S5_ERR_INVALID_ARG;
+  if (workspace == nullptr) return S5_ERR_WORKSPACE;
+  if (batch->total_q == 0) return S5_OK;
+  if (q_index == nullptr || sel == nullptr || sel_count == nullptr || !aligned16(q_index))
+    return S5_ERR_INVALID_ARG;
+  const IndexWs w = index_ws(batch);
+  if (workspace_bytes < w.end) return S5_ERR_WORKSPACE;
+  uint8_t *wsb = static_cast<uint8_t *>(workspace);
+  int32_t *err = reinterpret_cast<int32_t *>(workspace);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  IndexScoreArgs ia{};
+  ia.key_pool = index->key_pool;
+  ia.num_pages = index->num_pages;
+  ia.page_table = batch->page_table;
+  ia.max_pages = batch->max_pages;
+  ia.ctx_lens = batch->ctx_lens;
+  ia.cu_q = batch->cu_q;
+  ia.batch = batch->batch;
+  ia.total_q = batch->total_q;
+  ia.q_index = q_index;
+  ia.scores = reinterpret_cast<float *>(wsb + w.scores);
+  ia.score_stride = w.stride;
+  ia.pages_per_cta = kScorePagesPerCta;
+  ia.topk = topk;
+  ia.err = err;
+  const int pages = (w.stride + kBpp - 1) / kBpp;
+  const int grid_pages = (pages + kScorePagesPerCta - 1) / kScorePagesPerCta;
+  cudaError_t e = launch_index_score(ia, batch->max_q, grid_pages, batch->batch, cs);
+  if (e != cudaSuccess) return S5_ERR_CUDA;
+
+  SelectArgs sa{};
+  sa.scores = ia.scores;
+  sa.score_stride = w.stride;
+  sa.ctx_lens = batch->ctx_lens;
+  sa.cu_q = batch->cu_q;
+  sa.batch = batch->batch;
+  sa.topk = topk;
+  sa.sel = sel;
+  sa.sel_count = sel_count;
+  sa.seg = kSeg;
+  sa.n_seg = w.n_seg;
+  sa.cand_key = reinterpret_cast<uint32_t *>(wsb + w.cand_key);
+  sa.cand_idx = reinterpret_cast<int32_t *>(wsb + w.cand_idx);
+  sa.err = err;
+  return cuda_status(launch_topk_select(sa, batch->total_q, w.two_stage, cs));
+}
+
+s5_status s5_sparse_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, const void *q, const int32_t *sel,
+                             const int32_t *sel_count, int32_t topk, float sm_scale, void *out, float *lse,
+                             void *workspace, size_t workspace_bytes, s5_stream_t stream) {
+  return attn_common(kModeSparse, kv, batch, q, sel, sel_count, topk, 0, sm_scale, out, lse, workspace,
+                     workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+s5_status s5_swa_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, const void *q, int32_t window,
+                          float sm_scale, void *out, float *lse, void *workspace, size_t workspace_bytes,
+                          s5_stream_t stream) {
+  return attn_common(kModeSwa, kv, batch, q, nullptr, nullptr, 0, window, sm_scale, out, lse, workspace,
+                     workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+s5_status s5_reset_device_error(void *workspace, s5_stream_t stream) {
+  if (workspace == nullptr) return S5_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(workspace, 0, sizeof(ErrRec), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+s5_status s5_get_device_error(void *workspace, s5_stream_t stream, int32_t *code, int32_t *info) {
+  if (workspace == nullptr || code == nullptr || info == nullptr) return S5_ERR_INVALID_ARG;
+  ErrRec rec{};
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&rec, workspace, sizeof(rec), cudaMemcpyDeviceToHost, cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return S5_ERR_CUDA;
+  *code = rec.code;
+  *info = rec.code ? rec.info : -1;
+  return S5_OK;
+}
+
+const char *s5_status_string(s5_status status) {
+  switch (status) {
+    case S5_OK: return "S5_OK";
+    case S5_ERR_INVALID_ARG: return "S5_ERR_INVALID_ARG: bad pointer, size or descriptor field";
+    case S5_ERR_UNSUPPORTED: return "S5_ERR_UNSUPPORTED: outside what this build implements";
+    case S5_ERR_CUDA: return "S5_ERR_CUDA: a CUDA launch or runtime call failed";
+    case S5_ERR_DEVICE_BOUNDS: return "S5_ERR_DEVICE_BOUNDS: device data out of range";
+    case S5_ERR_TIMEOUT: return "S5_ERR_TIMEOUT: a bounded in-kernel wait expired";
+    case S5_ERR_WORKSPACE: return "S5_ERR_WORKSPACE: workspace missing or too small";
+  }
+  return "S5_ERR_UNKNOWN";
+}
+
+int32_t s5_abi_version(void) { return kAbiVersion; }
+
+}  // extern "C"

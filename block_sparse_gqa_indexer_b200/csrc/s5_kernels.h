@@ -1,0 +1,75 @@
+// Internal interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace s5 {
+
+constexpr int kModeSparse = 0;
+constexpr int kModeSwa = 1;
+constexpr int kMaxList = 544;  // blocks one attention CTA may own (>= 512 + 1)
+
+struct IndexScoreArgs {
+  const void *key_pool;
+  int num_pages;
+  const int32_t *page_table;
+  int max_pages;
+  const int32_t *ctx_lens;
+  const int32_t *cu_q;
+  int batch;
+  int total_q;
+  const void *q_index;
+  float *scores;     // [total_q][score_stride]
+  int score_stride;  // >= history blocks of any row
+  int pages_per_cta;
+  int topk;
+  int32_t *err;
+};
+
+struct SelectArgs {
+  const float *scores;
+  int score_stride;
+  const int32_t *ctx_lens;
+  const int32_t *cu_q;
+  int batch;
+  int topk;
+  int32_t *sel;
+  int32_t *sel_count;
+  // two-stage select
+  int seg;    // blocks per segment
+  int n_seg;  // segments per row (stride of the candidate arrays)
+  uint32_t *cand_key;
+  int32_t *cand_idx;
+  int32_t *err;
+};
+
+struct AttnArgs {
+  const void *q;
+  const int32_t *sel;
+  const int32_t *sel_count;
+  int topk;
+  int window;
+  const int32_t *page_table;
+  int max_pages;
+  const int32_t *ctx_lens;
+  const int32_t *cu_q;
+  int batch;
+  int max_len;
+  int num_pages;
+  float scale_log2;  // sm_scale * log2(e)
+  int n_split;
+  void *out;
+  float *lse;
+  float *part_o;    // [total_q * 64][n_split][192]
+  float *part_lse;  // [total_q * 64][n_split]   (base-2)
+  int32_t *err;
+};
+
+cudaError_t launch_index_score(const IndexScoreArgs &a, int max_q, int grid_pages, int n_seq, cudaStream_t st);
+cudaError_t launch_topk_select(const SelectArgs &a, int total_q, bool two_stage, cudaStream_t st);
+cudaError_t launch_gqa_decode(int mode, const AttnArgs &a, const CUtensorMap &tk, const CUtensorMap &tv,
+                              int total_q, cudaStream_t st);
+
+}  // namespace s5

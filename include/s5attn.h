@@ -1,0 +1,181 @@
+/*
+ * s5attn.h - C ABI of the B200 (sm_100a) sparse / sliding-window GQA library.
+ *
+ * The library computes the attention hot path of the Step 5 Preview hybrid
+ * attention layers:
+ *
+ *   sparse full-attention layer  (SGLang day-0 blog "Step 5 Preview: Day-0
+ *     Inference and RL Support with SGLang and Miles", section "Hybrid
+ *     Attention"; StepFun open-weights blog, section "What the config says"):
+ *     an indexer scores one 256-dim key per 8-token block of history, each
+ *     query token keeps its 512 best blocks plus its current block, and
+ *     grouped-query attention (64 query heads, 4 KV groups, head dim 192)
+ *     runs over the tokens of those blocks only;
+ *   sliding-window layer (same sections): causal GQA over the most recent
+ *     512 tokens.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers.  Every tensor pointer is DEVICE memory owned by the caller; the
+ *   library never allocates, frees or takes ownership, and never keeps a
+ *   pointer after the call returns.  Descriptors are HOST structs read during
+ *   the call only.
+ * Streams.  Work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream) and the call returns without synchronising, except
+ *   s5_get_device_error.  No entry point allocates or synchronises, so the
+ *   compute calls can be captured into a CUDA graph.
+ * Layouts.  All layouts are dense, row-major, little-endian; bf16 is IEEE
+ *   bfloat16.
+ *     K / V pool      bf16 [num_pages][4 kv groups][64 tokens][192]
+ *                     (one 8-token block of one group = 3,072 contiguous bytes)
+ *     index-key pool  bf16 [num_pages][8 blocks][256]: slot j of the page that
+ *                     holds logical page P of a sequence is the key of block
+ *                     8P + j (shares the sparse layer's page table)
+ *     page table      int32 [batch][max_pages]; logical page P of sequence s
+ *                     lives in physical page page_table[s][P]
+ *     q               bf16 [total_q][64][192]; head h reads KV group h / 16
+ *     q_index         bf16 [total_q][256]
+ *     sel             int32 [total_q][topk]
+ *     out             bf16 [total_q][64][192];  lse fp32 [total_q][64]
+ * Batches.  Sequence s has ctx_lens[s] cached tokens followed by
+ *   cu_q[s+1] - cu_q[s] new query tokens whose K/V are ALREADY in the pools;
+ *   query row r of sequence s sits at absolute position
+ *   t = ctx_lens[s] + (r - cu_q[s]).  Its current block is c = t / 8 and its
+ *   history blocks are 0 .. c-1.
+ * Errors.  Argument checks run on the host before anything is enqueued and
+ *   return S5_ERR_INVALID_ARG / S5_ERR_UNSUPPORTED / S5_ERR_WORKSPACE with
+ *   nothing enqueued.  Launch failures return S5_ERR_CUDA.  Faults in device
+ *   data (a page id, block id, length or count out of range) never trap: the
+ *   kernel records the first one in the workspace error record, skips the
+ *   offending access and continues; read it with s5_get_device_error.  Every
+ *   wait inside a kernel is bounded; a wait that runs out records
+ *   S5_ERR_TIMEOUT.
+ * Determinism.  Results are bit-identical run to run for identical inputs
+ *   and launch configuration (fixed reduction orders, no atomics on data).
+ */
+#ifndef S5ATTN_H
+#define S5ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *s5_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  S5_OK = 0,
+  S5_ERR_INVALID_ARG = 1,   /* bad pointer, size or descriptor field            */
+  S5_ERR_UNSUPPORTED = 2,   /* valid request outside what this build implements */
+  S5_ERR_CUDA = 3,          /* a CUDA launch or runtime call failed             */
+  S5_ERR_DEVICE_BOUNDS = 4, /* device data out of range (recorded by a kernel)  */
+  S5_ERR_TIMEOUT = 5,       /* a bounded in-kernel wait expired                 */
+  S5_ERR_WORKSPACE = 6      /* workspace missing or smaller than required       */
+} s5_status;
+
+/* Geometry compiled into this build (StepFun open-weights blog, "What the
+ * config says"; SGLang day-0 blog, "Get Started": --page-size 64). */
+#define S5_N_HEADS 64
+#define S5_N_KV_HEADS 4
+#define S5_HEAD_DIM 192
+#define S5_PAGE_SIZE 64
+#define S5_BLOCK_SIZE 8
+#define S5_INDEX_DIM 256
+#define S5_MAX_TOPK 512
+#define S5_MAX_LEN (1 << 21) /* longest sequence (cached + new tokens) */
+
+/* One attention layer's paged KV cache. */
+typedef struct {
+  const void *k_pool;  /* device bf16 [num_pages][4][64][192], 16-byte aligned */
+  const void *v_pool;  /* device bf16, same shape                               */
+  int32_t num_pages;   /* >= 1                                                  */
+  int32_t page_size;   /* must be S5_PAGE_SIZE                                  */
+  int32_t n_kv_heads;  /* must be S5_N_KV_HEADS                                 */
+  int32_t head_dim;    /* must be S5_HEAD_DIM                                   */
+} s5_kv_desc;
+
+/* The sparse layer's block-key pool (same pages as its KV pool). */
+typedef struct {
+  const void *key_pool; /* device bf16 [num_pages][8][256], 16-byte aligned */
+  int32_t num_pages;
+  int32_t index_dim;    /* must be S5_INDEX_DIM */
+} s5_index_desc;
+
+/* A varlen batch and its page table. */
+typedef struct {
+  const int32_t *page_table; /* device int32 [batch][max_pages]                      */
+  const int32_t *ctx_lens;   /* device int32 [batch]: cached tokens before new queries */
+  const int32_t *cu_q;       /* device int32 [batch+1]: query-row offsets, cu_q[0]=0   */
+  int32_t batch;             /* >= 1                                                  */
+  int32_t max_pages;         /* row stride of page_table                              */
+  int32_t total_q;           /* cu_q[batch]; 0 is allowed (nothing is enqueued)       */
+  int32_t max_q;             /* upper bound on new tokens of any sequence             */
+  int32_t max_len;           /* upper bound on ctx_lens[s] + new tokens, <= S5_MAX_LEN */
+} s5_batch_desc;
+
+/* Bytes of device workspace any of the calls below may use for this batch
+ * (window: the largest sliding window that will be requested, or 0).  The
+ * first 256 bytes hold the device error record: zero them once (or call
+ * s5_reset_device_error) before first use; later calls keep them. */
+s5_status s5_workspace_size(const s5_batch_desc *batch, int32_t window, size_t *bytes);
+
+/* Indexer: score every history block of every query row and keep the best
+ * `topk` (SGLang day-0 blog, "Kernels from StepFun": indexer scoring against
+ * the compressed history in the paged cache; "Hybrid Attention": up to 512
+ * historical blocks).
+ *   score(r, b) = sum_d q_index[r][d] * key(s, b)[d]  for b < c(r), in fp32
+ *   (exact for integer-valued inputs; otherwise a fixed summation order).
+ * The indexer query is a per-token 256-dim input shared by all heads: the
+ * pages fix only the key side, so this is an assumption of the API.
+ * Selection: the `topk` best blocks by (score descending, block index
+ * ascending); all c blocks when c <= topk.  Written to sel[r][0..n-1] in
+ * ascending block order, sel[r][n..topk-1] = -1, sel_count[r] = n.
+ * topk in [1, 512].  sel / sel_count are device int32. */
+s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *batch,
+                              const void *q_index, int32_t topk, int32_t *sel,
+                              int32_t *sel_count, void *workspace, size_t workspace_bytes,
+                              s5_stream_t stream);
+
+/* Sparse gathered GQA (SGLang day-0 blog, "Hybrid Attention" and "Kernels
+ * from StepFun": attention over the selected blocks plus the current block;
+ * long selections are split into partitions whose partial results are
+ * merged).  For row r at position t and head h (group g = h / 16):
+ *   T   = union of tokens 8b..8b+7 over b in sel[r][0..sel_count[r]-1],
+ *         plus tokens 8c..t of the current block c = t / 8
+ *   out = sum_{j in T} softmax_j(sm_scale * q[r][h] . K[j][g]) V[j][g]
+ *   lse = log sum_{j in T} exp(sm_scale * q[r][h] . K[j][g])   (may be NULL)
+ * sel entries may come in any order; -1 entries past sel_count are ignored.
+ * sel_count[r] <= min(topk, c); entries must be distinct blocks < c. */
+s5_status s5_sparse_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch,
+                             const void *q, const int32_t *sel, const int32_t *sel_count,
+                             int32_t topk, float sm_scale, void *out, float *lse,
+                             void *workspace, size_t workspace_bytes, s5_stream_t stream);
+
+/* Sliding-window GQA (SGLang day-0 blog, "Hybrid Attention": three of four
+ * layers read the most recent 512 tokens).  T = positions
+ * max(0, t - window + 1) .. t; otherwise as s5_sparse_gqa_attn.  Pages that
+ * hold no position of any window are never read, so a sliding-window pool
+ * may leave them unmapped (-1). */
+s5_status s5_swa_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, const void *q,
+                          int32_t window, float sm_scale, void *out, float *lse,
+                          void *workspace, size_t workspace_bytes, s5_stream_t stream);
+
+/* Zero the device error record (asynchronous, on `stream`). */
+s5_status s5_reset_device_error(void *workspace, s5_stream_t stream);
+
+/* Synchronise `stream` and read the device error record: *code is S5_OK or
+ * the first recorded s5_status, *info the offending query row (or -1). */
+s5_status s5_get_device_error(void *workspace, s5_stream_t stream, int32_t *code, int32_t *info);
+
+/* Static English name of a status code. */
+const char *s5_status_string(s5_status status);
+
+/* ABI version of this header (major * 100 + minor). */
+int32_t s5_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* S5ATTN_H */

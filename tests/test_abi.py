@@ -1,0 +1,93 @@
+"""The C-ABI library loads and exports every entry point its header declares,
+and its host-side checks reject bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "s5attn.h")
+
+
+@pytest.fixture(scope="module")
+def s5():
+    from block_sparse_gqa_indexer_b200 import build
+    build.build()
+    from block_sparse_gqa_indexer_b200 import s5 as mod
+    return mod
+
+
+def _declared():
+    text = open(HEADER).read()
+    return set(re.findall(r"^\s*(?:s5_status|const char \*|int32_t)\s*(s5_\w+)\s*\(", text, re.M))
+
+
+def test_header_declarations_match_binding(s5):
+    assert _declared() == set(s5.SYMBOLS)
+
+
+def test_every_declared_symbol_is_exported(s5):
+    lib = ctypes.CDLL(s5.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(s5):
+    assert s5.s5_abi_version() == 100
+    for code in range(7):
+        assert s5.s5_status_string(code).startswith("S5_")
+    assert s5.s5_status_string(99) == "S5_ERR_UNKNOWN"
+
+
+def _batch(**kw):
+    fake = 0x1000
+    d = dict(page_table=fake, ctx_lens=fake, cu_q=fake, batch=2, max_pages=4, total_q=2, max_q=1, max_len=200)
+    d.update(kw)
+    from block_sparse_gqa_indexer_b200 import s5
+    return s5.BatchDesc(**d)
+
+
+def test_workspace_size_is_host_only(s5):
+    n = ctypes.c_size_t(0)
+    b = _batch()
+    assert s5._lib.s5_workspace_size(ctypes.byref(b), 512, ctypes.byref(n)) == 0
+    assert n.value >= 256
+    # the headline batch: 64 rows, 131,073 tokens each
+    b = _batch(batch=64, total_q=64, max_pages=2049, max_len=131073)
+    assert s5._lib.s5_workspace_size(ctypes.byref(b), 512, ctypes.byref(n)) == 0
+    parts = 64 * 64 * 8 * (192 + 1) * 4  # 8 partitions per row and group
+    assert parts <= n.value < parts + 64 * 16384 * 4 + 4096
+
+
+@pytest.mark.parametrize("field,val,code", [
+    ("batch", 0, 1), ("max_pages", 0, 1), ("total_q", -1, 1), ("max_len", (1 << 21) + 1, 2),
+    ("max_len", 4 * 64 + 1, 1), ("page_table", 0, 1),
+])
+def test_bad_batch_rejected(s5, field, val, code):
+    n = ctypes.c_size_t(0)
+    b = _batch(**{field: val})
+    assert s5._lib.s5_workspace_size(ctypes.byref(b), 512, ctypes.byref(n)) == code
+
+
+def test_bad_descriptors_rejected_before_launch(s5):
+    fake = ctypes.c_void_p(0x1000)
+    b = _batch()
+    kv = s5.KvDesc(0x1000, 0x1000, 8, 64, 4, 128)  # head_dim 128: not this build
+    assert s5._lib.s5_sparse_gqa_attn(ctypes.byref(kv), ctypes.byref(b), fake, fake, fake, 512, 0.1, fake, None,
+                                      fake, 1 << 30, None) == s5.S5_ERR_UNSUPPORTED
+    kv = s5.KvDesc(0x1000, 0x1000, 8, 64, 4, 192)
+    assert s5._lib.s5_sparse_gqa_attn(ctypes.byref(kv), ctypes.byref(b), fake, fake, fake, 513, 0.1, fake, None,
+                                      fake, 1 << 30, None) == s5.S5_ERR_INVALID_ARG
+    assert s5._lib.s5_swa_gqa_attn(ctypes.byref(kv), ctypes.byref(b), fake, 0, 0.1, fake, None, fake, 1 << 30,
+                                   None) == s5.S5_ERR_INVALID_ARG
+    assert s5._lib.s5_sparse_gqa_attn(ctypes.byref(kv), ctypes.byref(b), fake, fake, fake, 512, 0.1, fake, None,
+                                      fake, 16, None) == s5.S5_ERR_WORKSPACE
+    ix = s5.IndexDesc(0x1000, 8, 128)
+    assert s5._lib.s5_index_score_topk(ctypes.byref(ix), ctypes.byref(b), fake, 512, fake, fake, fake, 1 << 30,
+                                       None) == s5.S5_ERR_UNSUPPORTED
+    ix = s5.IndexDesc(0x1000, 8, 256)
+    assert s5._lib.s5_index_score_topk(ctypes.byref(ix), ctypes.byref(b), fake, 0, fake, fake, fake, 1 << 30,
+                                       None) == s5.S5_ERR_INVALID_ARG
+    assert s5._lib.s5_index_score_topk(ctypes.byref(ix), ctypes.byref(b), fake, 512, fake, fake, None, 1 << 30,
+                                       None) == s5.S5_ERR_WORKSPACE

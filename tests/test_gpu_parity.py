@@ -1,0 +1,253 @@
+"""CUDA path against the CPU oracle, through the C ABI.
+
+Selections must match bit-exactly (integer-valued indexer inputs make the fp32
+scores exact); attention outputs must be within max-abs 2e-2 and rel-RMS 5e-3
+of the float64 oracle (rounded to bf16), lse within 1e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_gqa_indexer_b200 import synth as S
+from oracle import s5_oracle as O
+from tests.harness import (DeviceInputs, LSE_ABS, assert_attn_close, oracle_selection, oracle_sparse,
+                           oracle_swa, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_index(lib, d: DeviceInputs):
+    lib.s5_index_score_topk(d.key_pool, d.batch, d.qx, S.TOPK, d.sel, d.sel_count, d.ws)
+
+
+def _run_sparse(lib, d: DeviceInputs, sel=None, sm_scale=O.DEFAULT_SM_SCALE):
+    lib.s5_sparse_gqa_attn(d.k_pool, d.v_pool, d.batch, d.q, d.sel if sel is None else sel, d.sel_count, S.TOPK,
+                           sm_scale, d.out, d.lse, d.ws)
+
+
+def _check_no_device_error(lib, d):
+    code, info = lib.s5_get_device_error(d.ws)
+    assert code == 0, (lib.s5_status_string(code), info)
+
+
+def _check_selection(lib, d, rows):
+    torch.cuda.synchronize()
+    want = oracle_selection(d.w, rows)
+    got = d.sel.cpu().numpy()[rows]
+    cnt = d.sel_count.cpu().numpy()[rows]
+    for i, r in enumerate(rows):
+        assert np.array_equal(got[i], want[i]), f"row {r}: selection differs"
+        assert cnt[i] == O.selection_count(want[i])
+    return want
+
+
+def _check_sparse_out(d, rows, sel_rows, what):
+    want, want_lse = oracle_sparse(d.w, rows, sel_rows)
+    got = d.out.float().cpu().numpy()[rows]
+    assert_attn_close(got, want, what)
+    lse = d.lse.cpu().numpy()[rows]
+    assert np.abs(lse - want_lse).max() <= LSE_ABS
+
+
+# ------------------------------------------------------------------ small cases (every row checked)
+
+SMALL_SPARSE = [
+    # ctx per sequence, nq per sequence: history below / at / above 512 blocks, ragged tails
+    ([0, 5, 7, 8, 100], [1, 1, 1, 1, 1]),
+    ([4095, 4096, 4103, 4104, 4111], [1, 1, 1, 1, 1]),
+    ([6000, 9999, 20001], [1, 1, 1]),
+    ([5000, 4090, 12345], [4, 4, 4]),            # verify: 4 tokens each, crossing block edges
+    ([3, 4200, 777, 16383, 9000], [2, 3, 1, 4, 0]),  # varlen, an empty sequence
+]
+
+
+@pytest.mark.parametrize("ctx,nq", SMALL_SPARSE)
+def test_sparse_small_all_rows(lib, ctx, nq):
+    w = S.Workload(ctx=ctx, nq=nq, seed=11)
+    d = DeviceInputs(w, lib)
+    _run_index(lib, d)
+    _run_sparse(lib, d)
+    rows = list(range(w.total_q))
+    want_sel = _check_selection(lib, d, rows)
+    _check_sparse_out(d, rows, want_sel, f"sparse ctx={ctx} nq={nq}")
+    _check_no_device_error(lib, d)
+
+
+@pytest.mark.parametrize("ctx,nq,window", [
+    ([0, 1, 300, 511, 512, 513, 1000], [1] * 7, 512),
+    ([7000, 65, 2047], [4, 2, 1], 512),
+    ([2500, 100], [1, 3], 64),
+    ([900, 33], [1, 1], 4096),  # window covers everything: full causal attention
+])
+def test_swa_small_all_rows(lib, ctx, nq, window):
+    w = S.Workload(ctx=ctx, nq=nq, seed=12)
+    d = DeviceInputs(w, lib, with_index=False)
+    lib.s5_swa_gqa_attn(d.k_pool, d.v_pool, d.batch, d.q, window, O.DEFAULT_SM_SCALE, d.out, d.lse, d.ws)
+    rows = list(range(w.total_q))
+    want, want_lse = oracle_swa(w, rows, window)
+    assert_attn_close(d.out.float().cpu().numpy(), want, f"swa ctx={ctx} W={window}")
+    assert np.abs(d.lse.cpu().numpy() - want_lse).max() <= LSE_ABS
+    _check_no_device_error(lib, d)
+
+
+def test_sparse_equals_swa_when_history_fits(lib):
+    # c <= 512 selects every history block: sparse == sliding window with W >= length
+    w = S.Workload(ctx=[1000, 4000, 4095], nq=[1, 2, 1], seed=13)
+    d = DeviceInputs(w, lib)
+    _run_index(lib, d)
+    _run_sparse(lib, d)
+    torch.cuda.synchronize()
+    sparse_out = d.out.clone()
+    lib.s5_swa_gqa_attn(d.k_pool, d.v_pool, d.batch, d.q, 1 << 20, O.DEFAULT_SM_SCALE, d.out, d.lse, d.ws)
+    assert_attn_close(sparse_out.float().cpu().numpy(), d.out.float().cpu().numpy(), "sparse vs full")
+
+
+def test_sparse_block_order_invariance(lib):
+    w = S.Workload(ctx=[30000, 7777], nq=[1, 2], seed=14)
+    d = DeviceInputs(w, lib)
+    _run_index(lib, d)
+    _run_sparse(lib, d)
+    torch.cuda.synchronize()
+    ref = d.out.float().cpu().numpy()
+    g = torch.Generator().manual_seed(3)
+    sel = d.sel.cpu()
+    perm = sel.clone()
+    for r in range(sel.shape[0]):
+        n = int(d.sel_count[r])
+        perm[r, :n] = sel[r, :n][torch.randperm(n, generator=g)]
+    _run_sparse(lib, d, sel=perm.cuda())
+    assert_attn_close(d.out.float().cpu().numpy(), ref, "permuted selection")
+
+
+def test_deterministic_across_runs(lib):
+    w = S.Workload(ctx=[20000] * 6, nq=[1] * 6, seed=15)
+    d = DeviceInputs(w, lib)
+    outs = []
+    for _ in range(3):
+        _run_index(lib, d)
+        _run_sparse(lib, d)
+        torch.cuda.synchronize()
+        outs.append((d.sel.clone(), d.out.clone(), d.lse.clone()))
+    for o in outs[1:]:
+        assert torch.equal(o[0], outs[0][0]) and torch.equal(o[1], outs[0][1]) and torch.equal(o[2], outs[0][2])
+
+
+def test_softmax_weights_sum_to_one(lib):
+    # with every V row equal to 1, each output is the sum of the softmax weights
+    w = S.Workload(ctx=[9000, 300], nq=[1, 1], seed=16)
+    d = DeviceInputs(w, lib)
+    d.v_pool.fill_(1.0)
+    _run_index(lib, d)
+    _run_sparse(lib, d)
+    torch.cuda.synchronize()
+    # P is rounded to bf16 for the PV product while the denominator sums it in fp32
+    assert float((d.out.float() - 1.0).abs().max()) <= 2 ** -8
+
+
+def test_tie_heavy_selection(lib):
+    # all block keys equal: every score ties, the first 512 blocks win
+    w = S.Workload(ctx=[50000, 8 * 600 + 3], nq=[1, 2], seed=17)
+    d = DeviceInputs(w, lib)
+    d.key_pool.fill_(1.0)
+    _run_index(lib, d)
+    torch.cuda.synchronize()
+    for r in range(w.total_q):
+        assert d.sel[r].tolist() == list(range(512))
+
+
+def test_bad_page_is_reported_not_read(lib):
+    w = S.Workload(ctx=[20000], nq=[1], seed=18)
+    d = DeviceInputs(w, lib)
+    d.batch.page_table[0, 5] = -1  # an unmapped page in the history
+    lib.s5_reset_device_error(d.ws)
+    _run_index(lib, d)
+    _run_sparse(lib, d)
+    code, info = lib.s5_get_device_error(d.ws)
+    assert code == lib.S5_ERR_DEVICE_BOUNDS and info == 0
+    assert torch.isfinite(d.out.float()).all()
+
+
+def test_host_validation(lib):
+    w = S.Workload(ctx=[100], nq=[1], seed=19)
+    d = DeviceInputs(w, lib)
+    with pytest.raises(lib.S5Error) as e:
+        lib.s5_sparse_gqa_attn(d.k_pool, d.v_pool, d.batch, d.q, d.sel, d.sel_count, S.TOPK, float("nan"), d.out,
+                               d.lse, d.ws)
+    assert e.value.code == lib.S5_ERR_INVALID_ARG
+    with pytest.raises(lib.S5Error) as e:
+        lib.s5_swa_gqa_attn(d.k_pool, d.v_pool, d.batch, d.q, 0, 0.1, d.out, d.lse, d.ws)
+    assert e.value.code == lib.S5_ERR_INVALID_ARG
+    with pytest.raises(lib.S5Error) as e:
+        lib.s5_sparse_gqa_attn(d.k_pool, d.v_pool, d.batch, d.q, d.sel, d.sel_count, S.TOPK, 0.1, d.out, d.lse,
+                               d.ws[:64])
+    assert e.value.code == lib.S5_ERR_WORKSPACE
+
+
+# ------------------------------------------------------------------ the configurations (sampled rows)
+
+def _config_sparse(lib, which, n_rows, seed=0):
+    (w,) = S.config_workloads(which)
+    d = DeviceInputs(w, lib)
+    lib.s5_reset_device_error(d.ws)
+    _run_index(lib, d)
+    _run_sparse(lib, d)
+    rows = sample_rows(w.total_q, n_rows, seed)
+    want_sel = _check_selection(lib, d, rows)
+    _check_sparse_out(d, rows, want_sel, f"config {which}")
+    _check_no_device_error(lib, d)
+    return d
+
+
+@pytest.mark.slow
+def test_config1_sparse_decode_b1_16k(lib):
+    _config_sparse(lib, 1, 1)
+
+
+@pytest.mark.slow
+def test_config3_sparse_verify_b64x4(lib):
+    _config_sparse(lib, 3, 8)
+
+
+@pytest.mark.slow
+def test_headline_sparse_decode_b64_128k(lib):
+    _config_sparse(lib, 0, 4)
+
+
+@pytest.mark.slow
+def test_config2_swa_decode_b64(lib):
+    (w,) = S.config_workloads(2)
+    d = DeviceInputs(w, lib, window_only=S.WINDOW, with_index=False)
+    lib.s5_swa_gqa_attn(d.k_pool, d.v_pool, d.batch, d.q, S.WINDOW, O.DEFAULT_SM_SCALE, d.out, d.lse, d.ws)
+    rows = sample_rows(w.total_q, 8)
+    want, want_lse = oracle_swa(w, rows)
+    assert_attn_close(d.out.float().cpu().numpy()[rows], want, "config 2")
+    assert np.abs(d.lse.cpu().numpy()[rows] - want_lse).max() <= LSE_ABS
+    _check_no_device_error(lib, d)
+
+
+@pytest.mark.slow
+def test_config4_sparse_prefill_16k(lib):
+    _config_sparse(lib, 4, 6)
+
+
+@pytest.mark.slow
+def test_config5_hybrid_1m(lib):
+    layers = S.config_workloads(5)
+    for li, w in enumerate(layers):
+        if li < 3:
+            d = DeviceInputs(w, lib, window_only=S.WINDOW, with_index=False)
+            lib.s5_swa_gqa_attn(d.k_pool, d.v_pool, d.batch, d.q, S.WINDOW, O.DEFAULT_SM_SCALE, d.out, d.lse, d.ws)
+            rows = sample_rows(w.total_q, 2, li)
+            want, _ = oracle_swa(w, rows)
+            assert_attn_close(d.out.float().cpu().numpy()[rows], want, f"config 5 swa layer {li}")
+            _check_no_device_error(lib, d)
+        else:
+            d = DeviceInputs(w, lib)
+            _run_index(lib, d)
+            _run_sparse(lib, d)
+            rows = sample_rows(w.total_q, 2, li)
+            want_sel = _check_selection(lib, d, rows)
+            _check_sparse_out(d, rows, want_sel, "config 5 sparse layer")
+            _check_no_device_error(lib, d)
+        del d
+        torch.cuda.empty_cache()
