@@ -1,0 +1,395 @@
+"""Benchmark of one sparse-layer decode step (indexer + top-512 + gathered GQA).
+
+Workload: batch 64, 131,072 cached tokens per sequence, one query token each
+(64 query heads, 4 KV groups, head dim 192, bf16 KV in 64-token pages, one
+256-dim integer-valued bf16 block key per 8 tokens), seeded synthetic data.
+A step is s5_index_score_topk followed by s5_sparse_gqa_attn on resident
+inputs.  Metric: algorithmic bytes of the step (selected KV + scored block
+keys + queries / outputs) per second, with queries/s beside it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own replica (weak scaling; no collective
+on the data path); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_sparse_gqa_indexer_b200 import roofline as R  # noqa: E402
+from block_sparse_gqa_indexer_b200 import synth as S  # noqa: E402
+
+METRIC = "sparse-layer decode selected-KV GB/s (% HBM peak) & queries/s, B=64, 128K ctx"
+UNIT = "GB/s"
+N_ROT = 4  # rotating query sets: each step selects different blocks
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def _workload(rank: int = 0, batch: int = 64, world: int = 1) -> S.Workload:
+    """This rank's shard of a global batch of batch * world sequences (every
+    sequence has 131,072 cached tokens and one query token)."""
+    (w,) = S.config_workloads(0)
+    w.ctx, w.nq = [w.ctx[0]] * (batch * world), [1] * (batch * world)
+    return S.shard(w, rank, world)
+
+
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """The largest value of x over all ranks (x itself without a process group)."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _step_bytes(w: S.Workload) -> dict:
+    sp = R.sparse_decode_bytes(w.ctx, w.nq)
+    # split into the two calls of the step
+    keys = sp["keys"] + w.total_q * (R.index_key_bytes() + 4 * (R.TOPK + 1))  # keys + q_index + sel
+    attn = sp["kv"] + w.total_q * (R.q_bytes() + R.out_bytes() + 4 * (R.TOPK + 1))
+    return {"total": sp["total"], "index": keys, "attn": attn, "kv": sp["kv"], "keys": sp["keys"]}
+
+
+# ---------------------------------------------------------------- clocks
+
+CLOCK_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={CLOCK_FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+
+def _oracle_sample(w: S.Workload, rows):
+    """Inputs of the oracle for `rows` of the workload, drawn on the host."""
+    from oracle import s5_oracle as O
+    seqs, pos = w.query_seq_pos()
+    rt = torch.as_tensor(rows, dtype=torch.int64)
+    qx = w.qx_rows(rt).double().numpy()
+    q = w.q_rows(rt).double().numpy()
+    items = []
+    for i, r in enumerate(rows):
+        s, t = seqs[r], pos[r]
+        c = t // S.BLOCK
+        kx = w.kx_blocks(s, torch.arange(c)).double().numpy()
+        sel = O.index_topk_query(qx[i], kx, t)  # only to know which K/V rows to draw
+        T = O.sparse_token_set(sel, t)
+        kv_pos = torch.as_tensor(T)
+        K = w.k_tokens(s, kv_pos).double().numpy()
+        V = w.v_tokens(s, kv_pos).double().numpy()
+        items.append((qx[i], kx, t, q[i], {int(p): j for j, p in enumerate(T)}, K, V))
+    return items
+
+
+class _RowsByPos:
+    def __init__(self, table, rows):
+        self.table, self.rows = table, rows
+
+    def __getitem__(self, pos):
+        return self.rows[[self.table[int(p)] for p in pos]]
+
+
+def _oracle_time(items) -> float:
+    """Wall time of the oracle (selection + sparse attention) over the sample."""
+    from oracle import s5_oracle as O
+    t0 = time.perf_counter()
+    for qx, kx, t, q, table, K, V in items:
+        sel = O.index_topk_query(qx, kx, t)
+        O.sparse_attention_query(q, sel, t, _RowsByPos(table, K), _RowsByPos(table, V))
+    return time.perf_counter() - t0
+
+
+def _threads() -> int:
+    try:
+        import threadpoolctl
+        return max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info())
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w: S.Workload, n_rows: int = 16) -> dict:
+    rows = list(range(0, w.total_q, max(1, w.total_q // n_rows)))[:n_rows]
+    items = _oracle_sample(w, rows)
+    dt = _oracle_time(items)
+    b = R.sparse_decode_bytes([w.ctx[0]] * len(rows), [1] * len(rows))["total"]
+    return {"value": b / dt / 1e9, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": f"{len(rows)} of the 64 query rows (float64 numpy oracle: full-sort top-512 over 16,384 "
+                      f"block scores + sparse attention); {dt:.2f} s; inputs drawn before timing",
+            "queries_per_s": len(rows) / dt}
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = _workload(0)
+    per_step = 4
+    n = (args.warmup + args.steps) * per_step
+    rows = [(i * 7) % w.total_q for i in range(n)]
+    items = _oracle_sample(w, rows)
+    for i in range(args.warmup):
+        _oracle_time(items[i * per_step:(i + 1) * per_step])
+    times = []
+    for i in range(args.warmup, args.warmup + args.steps):
+        times.append(_oracle_time(items[i * per_step:(i + 1) * per_step]))
+    total = sum(times)
+    b = R.sparse_decode_bytes([w.ctx[0]] * per_step, [1] * per_step)["total"]
+    value = b * args.steps / total / 1e9
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "sparse decode B=64 ctx=131072 (oracle: 4 query rows per step)",
+                       "batch": 64, "ctx": 131072, "topk": 512},
+            "queries_per_s": per_step * args.steps / total,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+                             "sample": f"{per_step} query rows per step, {args.steps} steps"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def _src_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_gqa_indexer_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernels have
+    not changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(kernel)
+    if not e or e.get("src_hash") != _src_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+def run_ours(args) -> None:
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+
+    from block_sparse_gqa_indexer_b200 import s5
+    w = _workload(rank, args.batch, world)
+    pt = w.page_table()
+    k_pool, v_pool = w.kv_pools(dev, pt)
+    key_pool = w.index_pool(dev, pt)
+    batch = s5.Batch.from_host(pt, w.ctx, w.nq, dev)
+    ws = s5.new_workspace(batch, device=dev)
+    tq = w.total_q
+    qs, qxs = [], []
+    for i in range(N_ROT):
+        rows = torch.arange(tq, dtype=torch.int64) + i * tq * world  # a fresh query set per rotation
+        qs.append(w.q_rows(rows, dev))
+        qxs.append(w.qx_rows(rows, dev))
+    sel = torch.empty((tq, S.TOPK), dtype=torch.int32, device=dev)
+    cnt = torch.empty((tq,), dtype=torch.int32, device=dev)
+    out = torch.empty((tq, 64, 192), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((tq, 64), dtype=torch.float32, device=dev)
+    scale = 1.0 / (192 ** 0.5)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        s5.s5_index_score_topk(key_pool, batch, qxs[i % N_ROT], S.TOPK, sel, cnt, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        s5.s5_sparse_gqa_attn(k_pool, v_pool, batch, qs[i % N_ROT], sel, cnt, S.TOPK, scale, out, lse, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    code, info = s5.s5_get_device_error(ws)
+    if code != 0:
+        raise RuntimeError(f"device error after warm-up: {s5.s5_status_string(code)} row {info}")
+
+    # ---- device-timed region ----
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if dist is not None:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    idx_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    ms = max_over_ranks(ms, dist, dev)
+
+    # ---- end to end through the public API: per-step inputs from pinned host memory ----
+    q_host = [x.cpu().pin_memory() for x in qs]
+    qx_host = [x.cpu().pin_memory() for x in qxs]
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    q_dev, qx_dev = torch.empty_like(qs[0]), torch.empty_like(qxs[0])
+    e2e_steps = max(10, args.steps // 4)
+    for i in range(3):
+        s5.sparse_layer_step_host(key_pool, k_pool, v_pool, batch, q_host[i % N_ROT], qx_host[i % N_ROT], out_host,
+                                  lse_host, sel, cnt, q_dev, qx_dev, out, lse, ws, stream=stream)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        s5.sparse_layer_step_host(key_pool, k_pool, v_pool, batch, q_host[i % N_ROT], qx_host[i % N_ROT], out_host,
+                                  lse_host, sel, cnt, q_dev, qx_dev, out, lse, ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    code, info = s5.s5_get_device_error(ws)
+    if code != 0:
+        raise RuntimeError(f"device error: {s5.s5_status_string(code)} row {info}")
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    by = _step_bytes(w)
+    n = world
+    step_ms = ms / args.steps
+    value = n * by["total"] * args.steps / (ms * 1e-3) / 1e9
+    peak, peak_kind = _peaks()
+    # dominant call of the step: the longer of the two, per launch of its main kernel
+    if attn_ms >= idx_ms:
+        dom, dom_ms, dom_bytes = "gqa_decode_kernel", attn_ms, by["attn"]
+    else:
+        dom, dom_ms, dom_bytes = "index_score_kernel", idx_ms, by["index"]
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    cpu = cpu_baseline(w) if (n == 1 and not args.no_cpu) else None
+    launches_per_step = 2 + 2  # score + select, attention + partition merge
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"sparse-layer decode: B={w.batch} per GPU, 131,072 cached tokens each, 1 query "
+                               "token; 64 q heads / 4 KV groups / head dim 192; top-512 of 16,384 blocks + current "
+                               "block",
+                   "batch": w.batch, "ctx": 131072, "topk": 512, "page": 64, "parallelism": f"replicas x{n}",
+                   "l2": "inputs larger than L2: each step reads 1.35 GB (806 MB selected KV + 537 MB block "
+                         "keys) and rotates 4 query sets so consecutive steps select different blocks"},
+        "queries_per_s": n * w.total_q * args.steps / (ms * 1e-3),
+        "pct_hbm_peak": 100.0 * (by["total"] / (step_ms * 1e-3) / 1e9) / peak,
+        "kernels_ms": {"s5_index_score_topk": idx_ms, "s5_sparse_gqa_attn": attn_ms},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
+                     "traffic": _ncu_traffic(dom), "algorithmic_bytes_per_launch": dom_bytes},
+        "cpu_baseline": cpu,
+        "e2e": {"value": n * by["total"] * e2e_steps / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+                "h2d_bytes_per_step": int(qs[0].numel() * 2 + qxs[0].numel() * 2),
+                "d2h_bytes_per_step": int(out.numel() * 2 + lse.numel() * 4), "ms_per_step": e2e_ms / e2e_steps},
+        "clocks": clk,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--batch", type=int, default=64, help="sequences per GPU (64 = the stated workload)")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        args.steps = min(args.steps, 20)
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

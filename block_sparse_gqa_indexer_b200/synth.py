@@ -152,6 +152,8 @@ class Workload:
     layer: int = 0
     index_int: bool = True  # integer-valued indexer inputs (exact fp32 scores)
     perm_pages: bool = True  # shuffle physical pages
+    seq_base: int = 0  # global id of sequence 0 (a shard of a larger batch)
+    row_base: int = 0  # global id of query row 0
 
     def __post_init__(self):
         assert len(self.ctx) == len(self.nq)
@@ -228,14 +230,14 @@ class Workload:
     # ---------------- logical values (any device) ----------------
     def q_rows(self, rows: torch.Tensor, device="cpu") -> torch.Tensor:
         """Attention queries, bf16 [len(rows)][64][192]."""
-        rows = rows.to(device=device, dtype=torch.int64)
+        rows = rows.to(device=device, dtype=torch.int64) + self.row_base
         idx = (rows.view(-1, 1, 1) * N_HEADS + torch.arange(N_HEADS, device=device).view(1, -1, 1)) * HEAD_DIM \
             + torch.arange(HEAD_DIM, device=device).view(1, 1, -1)
         return normal_bf16(self.seed, self.tid(TID_Q), idx)
 
     def qx_rows(self, rows: torch.Tensor, device="cpu") -> torch.Tensor:
         """Indexer queries, bf16 [len(rows)][256] (one per query token, shared by all heads)."""
-        rows = rows.to(device=device, dtype=torch.int64)
+        rows = rows.to(device=device, dtype=torch.int64) + self.row_base
         idx = rows.view(-1, 1) * INDEX_DIM + torch.arange(INDEX_DIM, device=device).view(1, -1)
         if self.index_int:
             return small_int_bf16(self.seed, self.tid(TID_QX), idx)
@@ -244,14 +246,14 @@ class Workload:
     def kx_blocks(self, s: int, blocks: torch.Tensor, device="cpu") -> torch.Tensor:
         """Block keys of sequence s, bf16 [len(blocks)][256]."""
         blocks = blocks.to(device=device, dtype=torch.int64)
-        idx = (s * MAX_BLOCKS + blocks.view(-1, 1)) * INDEX_DIM + torch.arange(INDEX_DIM, device=device).view(1, -1)
+        idx = ((self.seq_base + s) * MAX_BLOCKS + blocks.view(-1, 1)) * INDEX_DIM + torch.arange(INDEX_DIM, device=device).view(1, -1)
         if self.index_int:
             return small_int_bf16(self.seed, self.tid(TID_KX), idx)
         return normal_bf16(self.seed, self.tid(TID_KX), idx)
 
     def _kv_tokens(self, tid: int, s: int, pos: torch.Tensor, device) -> torch.Tensor:
         pos = pos.to(device=device, dtype=torch.int64)
-        idx = ((s * MAX_TOKENS + pos.view(-1, 1, 1)) * N_KV + torch.arange(N_KV, device=device).view(1, -1, 1)) \
+        idx = (((self.seq_base + s) * MAX_TOKENS + pos.view(-1, 1, 1)) * N_KV + torch.arange(N_KV, device=device).view(1, -1, 1)) \
             * HEAD_DIM + torch.arange(HEAD_DIM, device=device).view(1, 1, -1)
         return normal_bf16(self.seed, self.tid(tid), idx)
 
@@ -307,7 +309,7 @@ class Workload:
             s = own_s[p0:p1].clamp(min=0).to(device).view(-1, 1, 1, 1)
             lp = own_p[p0:p1].clamp(min=0).to(device).view(-1, 1, 1, 1)
             pos = lp * PAGE + ar_t
-            idx = ((s * MAX_TOKENS + pos) * N_KV + ar_g) * HEAD_DIM + ar_d
+            idx = (((self.seq_base + s) * MAX_TOKENS + pos) * N_KV + ar_g) * HEAD_DIM + ar_d
             valid = (sel.to(device).view(-1, 1, 1, 1)) & (pos < lens.to(device)[s.view(-1)].view(-1, 1, 1, 1))
             kv = normal_bf16(self.seed, self.tid(TID_K), idx)
             k_pool[p0:p1] = torch.where(valid, kv, torch.zeros((), dtype=torch.bfloat16, device=device))
@@ -337,7 +339,7 @@ class Workload:
             s = own_s[p0:p1].clamp(min=0).to(device).view(-1, 1, 1)
             lp = own_p[p0:p1].clamp(min=0).to(device).view(-1, 1, 1)
             blk = lp * BLOCKS_PER_PAGE + ar_j
-            idx = (s * MAX_BLOCKS + blk) * INDEX_DIM + ar_d
+            idx = ((self.seq_base + s) * MAX_BLOCKS + blk) * INDEX_DIM + ar_d
             valid = used.to(device).view(-1, 1, 1) & (blk < nblk.to(device)[s.view(-1)].view(-1, 1, 1))
             if self.index_int:
                 vals = small_int_bf16(self.seed, tid, idx)
@@ -350,6 +352,17 @@ class Workload:
         """(q bf16 [total_q][64][192], qx bf16 [total_q][256]) for every query row."""
         rows = torch.arange(self.total_q, dtype=torch.int64)
         return self.q_rows(rows, device), self.qx_rows(rows, device)
+
+
+def shard(w: Workload, rank: int, world: int) -> Workload:
+    """The rank-th of `world` contiguous shards of w's sequences.  Values are
+    drawn with global sequence and row ids, so the shards of a batch hold
+    exactly the data of the whole batch."""
+    n = w.batch
+    lo, hi = rank * n // world, (rank + 1) * n // world
+    rows_before = sum(w.nq[:lo])
+    return dataclasses.replace(w, ctx=list(w.ctx[lo:hi]), nq=list(w.nq[lo:hi]), seq_base=w.seq_base + lo,
+                               row_base=w.row_base + rows_before)
 
 
 def uniform_lengths(seed: int, n: int, lo: int, hi: int) -> list:
