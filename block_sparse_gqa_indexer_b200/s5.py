@@ -30,7 +30,8 @@ S5_OK, S5_ERR_INVALID_ARG, S5_ERR_UNSUPPORTED, S5_ERR_CUDA, S5_ERR_DEVICE_BOUNDS
 
 # exported symbols (every declaration of include/s5attn.h)
 SYMBOLS = ("s5_workspace_size", "s5_index_score_topk", "s5_sparse_gqa_attn", "s5_swa_gqa_attn",
-           "s5_reset_device_error", "s5_get_device_error", "s5_status_string", "s5_abi_version")
+           "s5_index_score_topk_noalloc", "s5_reset_device_error", "s5_get_device_error", "s5_status_string",
+           "s5_abi_version")
 
 
 class KvDesc(ctypes.Structure):
@@ -57,6 +58,8 @@ _lib.s5_sparse_gqa_attn.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(Batch
                                     ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.s5_swa_gqa_attn.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(BatchDesc), _P, _I, ctypes.c_float, _P,
                                  _P, _P, ctypes.c_size_t, _P]
+_lib.s5_index_score_topk_noalloc.argtypes = [ctypes.POINTER(IndexDesc), ctypes.POINTER(BatchDesc), _P, _I, _P,
+                                             _P, _P]
 _lib.s5_reset_device_error.argtypes = [_P, _P]
 _lib.s5_get_device_error.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
 _lib.s5_status_string.argtypes = [ctypes.c_int]
@@ -156,6 +159,21 @@ def s5_index_score_topk(key_pool: torch.Tensor, batch: Batch, q_index: torch.Ten
     _check(_lib.s5_index_score_topk(ctypes.byref(idx), ctypes.byref(batch.desc), _ptr(q_index), int(topk),
                                     _ptr(sel), _ptr(sel_count), _ptr(ws), ws.numel(), _stream(stream)),
            "s5_index_score_topk")
+
+
+def s5_index_score_topk_noalloc(key_pool: torch.Tensor, batch: Batch, q_index: torch.Tensor, topk: int,
+                                sel: torch.Tensor, sel_count: torch.Tensor, stream=None):
+    """s5_index_score_topk with the library's fixed scratch array instead of a
+    workspace: for callers that cannot allocate device memory.  Calls that can
+    overlap on the GPU must be serialised by the caller."""
+    _need(key_pool, torch.bfloat16, "key_pool")
+    _need(q_index, torch.bfloat16, "q_index", (batch.total_q, INDEX_DIM))
+    _need(sel, torch.int32, "sel", (batch.total_q, topk))
+    _need(sel_count, torch.int32, "sel_count", (batch.total_q,))
+    idx = IndexDesc(key_pool.data_ptr(), key_pool.shape[0], key_pool.shape[-1])
+    _check(_lib.s5_index_score_topk_noalloc(ctypes.byref(idx), ctypes.byref(batch.desc), _ptr(q_index), int(topk),
+                                            _ptr(sel), _ptr(sel_count), _stream(stream)),
+           "s5_index_score_topk_noalloc")
 
 
 def _kv(k_pool, v_pool):

@@ -162,6 +162,31 @@ s5_status s5_swa_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, cons
                           int32_t window, float sm_scale, void *out, float *lse,
                           void *workspace, size_t workspace_bytes, s5_stream_t stream);
 
+/* s5_index_score_topk without a workspace.  The pages have no counterpart to
+ * this entry point: it exists for callers that cannot allocate device memory
+ * at all, such as code embedded in a host framework that owns every device
+ * allocation and hands over only inputs and outputs, or a process whose
+ * device-memory budget is fixed at start-up.  Results are those of
+ * s5_index_score_topk for the same arguments.
+ *   Scratch: a library-owned 8 MiB device array (file scope), which every GPU
+ *   that loads the library keeps until the process exits.  Limits: at most
+ *   16,384 history blocks per row (max_len <= 131,080) and
+ *   256 + 4 * total_q * ((max_len - 1) / 8) bytes <= 8 MiB; larger requests
+ *   return S5_ERR_WORKSPACE with nothing enqueued.
+ *   The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ *   library routine.  The first call on a device (with that device current)
+ *   looks up the array's device address once; make that first call before
+ *   any stream capture.
+ *   Every call shares the one array and leaves its contents behind; each call
+ *   clears the part that must start at zero.  Calls that can overlap on the
+ *   GPU (other streams, other host threads) race on the array: serialise them.
+ *   Device-data faults are recorded in the array's own error record, which
+ *   this entry point does not expose; diagnose bad inputs with
+ *   s5_index_score_topk and a workspace. */
+s5_status s5_index_score_topk_noalloc(const s5_index_desc *index, const s5_batch_desc *batch,
+                                      const void *q_index, int32_t topk, int32_t *sel, int32_t *sel_count,
+                                      s5_stream_t stream);
+
 /* Zero the device error record (asynchronous, on `stream`). */
 s5_status s5_reset_device_error(void *workspace, s5_stream_t stream);
 
