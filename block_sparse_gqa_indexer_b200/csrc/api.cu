@@ -17,10 +17,10 @@ using namespace s5;
 namespace {
 
 constexpr int kAbiVersion = 100;
-constexpr int kSelCap = 16384;      // one-stage select keeps a row's keys in shared memory
-constexpr int kSeg = 8192;          // two-stage select: blocks per segment
-constexpr int kMaxSeg = 32;         // ... and segments per row (kSeg * kMaxSeg >= S5_MAX_LEN / 8)
-constexpr int kTargetCtas = 2048;   // attention CTAs to aim for (~7 waves of 2 CTAs x 148 SMs)
+constexpr int kSelCap = 16384;      // rows up to this many blocks: one CTA selects the whole row
+constexpr int kSegShort = 4096;     // longer rows: top-k per segment of this many blocks, then a merge
+constexpr int kSeg = 8192;          // ... segments of rows longer than 16,384 blocks
+constexpr int kMaxSeg = 32;         // (kSeg * kMaxSeg >= S5_MAX_LEN / 8)
 constexpr int kMaxSplit = 32;
 constexpr int kScorePagesPerCta = 64;  // indexer CTA: 64 pages = 512 block keys = 256 KB
 
@@ -63,16 +63,17 @@ s5_status check_kv(const s5_kv_desc *kv) {
 
 struct IndexWs {
   size_t scores, cand_key, cand_idx, end;
-  int stride, n_seg;
+  int stride, seg, n_seg;
   bool two_stage;
 };
 
 IndexWs index_ws(const s5_batch_desc *b) {
   IndexWs w{};
-  w.stride = max_blocks(b);
+  w.stride = (max_blocks(b) + 3) & ~3;  // rows start 16-byte aligned
   w.two_stage = w.stride > kSelCap;
-  w.n_seg = w.two_stage ? (w.stride + kSeg - 1) / kSeg : 0;
-  size_t off = kWsHeader;
+  w.seg = (w.stride <= 16384) ? kSegShort : kSeg;
+  w.n_seg = w.two_stage ? (w.stride + w.seg - 1) / w.seg : 0;
+  size_t off = kWsFixed;
   w.scores = off;
   off = align_up(off + (size_t)b->total_q * w.stride * sizeof(float), 256);
   w.cand_key = off;
@@ -83,11 +84,13 @@ IndexWs index_ws(const s5_batch_desc *b) {
   return w;
 }
 
-// Partitions per (row, group): enough CTAs to fill the GPU, each warp at least
-// two block pairs, and no CTA owning more than kMaxList blocks.
-int choose_split(int total_q, int blocks_per_row) {
+// Partitions per (row, group).  The kernel is HBM-bound, so the aim is one
+// wave of equal CTAs (2 resident per SM): as many partitions as fit in that
+// wave, none when the batch alone fills it, each warp keeping at least two
+// block pairs, and no CTA owning more than kMaxList blocks.
+int choose_split(int total_q, int blocks_per_row, int slots) {
   const int units = total_q * kKv;
-  int n = (kTargetCtas + units / 2) / (units > 0 ? units : 1);
+  int n = units > 0 ? slots / units : 1;
   const int by_work = blocks_per_row / (4 * 4);  // 4 warps x 2 pairs x 2 blocks
   n = n < by_work ? n : by_work;
   n = n > kMaxSplit ? kMaxSplit : n;
@@ -96,15 +99,34 @@ int choose_split(int total_q, int blocks_per_row) {
   return n < 1 ? 1 : n;
 }
 
+constexpr int kCtasPerSm = 2;
+constexpr int kSizingSms = 256;  // workspace sizing assumes at most this many SMs
+
+// Attention CTA slots of the current device (cached per device).
+int device_slots() {
+  static std::mutex mu;
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kCtasPerSm * 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
+    if (sms > kSizingSms) sms = kSizingSms;
+    cache[dev] = kCtasPerSm * sms;
+  }
+  return cache[dev];
+}
+
 struct AttnWs {
   size_t part_o, part_lse, end;
   int n_split;
 };
 
-AttnWs attn_ws(const s5_batch_desc *b, int blocks_per_row) {
+AttnWs attn_ws(const s5_batch_desc *b, int blocks_per_row, int slots) {
   AttnWs w{};
-  w.n_split = choose_split(b->total_q, blocks_per_row);
-  size_t off = kWsHeader;
+  w.n_split = choose_split(b->total_q, blocks_per_row, slots);
+  size_t off = kWsFixed;
   w.part_o = off;
   if (w.n_split > 1) {
     off = align_up(off + (size_t)b->total_q * kHeads * w.n_split * kD * sizeof(float), 256);
@@ -174,7 +196,7 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   if (q == nullptr || out == nullptr || !aligned16(q) || !aligned16(out)) return S5_ERR_INVALID_ARG;
   if (mode == kModeSparse && (sel == nullptr || sel_count == nullptr)) return S5_ERR_INVALID_ARG;
   const int bpr = (mode == kModeSparse) ? sparse_blocks_per_row(topk) : swa_blocks_per_row(b, window);
-  const AttnWs w = attn_ws(b, bpr);
+  const AttnWs w = attn_ws(b, bpr, device_slots());
   if (ws_bytes < w.end) return S5_ERR_WORKSPACE;
   CUtensorMap tk, tv;
   if (!make_kv_map(&tk, kv->k_pool, kv->num_pages) || !make_kv_map(&tv, kv->v_pool, kv->num_pages))
@@ -199,6 +221,7 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   a.lse = lse;
   a.part_o = reinterpret_cast<float *>(wsb + w.part_o);
   a.part_lse = reinterpret_cast<float *>(wsb + w.part_lse);
+  a.merge_cnt = (b->total_q <= kMaxMergeRows) ? reinterpret_cast<uint32_t *>(wsb + kWsHeader) : nullptr;
   a.err = reinterpret_cast<int32_t *>(ws);
   return cuda_status(launch_gqa_decode(mode, a, tk, tv, b->total_q, stream));
 }
@@ -213,10 +236,11 @@ s5_status s5_workspace_size(const s5_batch_desc *batch, int32_t window, size_t *
   if (st != S5_OK) return st;
   if (window < 0) return S5_ERR_INVALID_ARG;
   size_t need = index_ws(batch).end;
-  const size_t sp = attn_ws(batch, sparse_blocks_per_row(kMaxTopk)).end;
+  const int slots = kCtasPerSm * kSizingSms;  // an upper bound: no device query here
+  const size_t sp = attn_ws(batch, sparse_blocks_per_row(kMaxTopk), slots).end;
   if (sp > need) need = sp;
   if (window > 0) {
-    const size_t sw = attn_ws(batch, swa_blocks_per_row(batch, window)).end;
+    const size_t sw = attn_ws(batch, swa_blocks_per_row(batch, window), slots).end;
     if (sw > need) need = sw;
   }
   *bytes = need;
@@ -271,7 +295,7 @@ s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *b
   sa.topk = topk;
   sa.sel = sel;
   sa.sel_count = sel_count;
-  sa.seg = kSeg;
+  sa.seg = w.seg;
   sa.n_seg = w.n_seg;
   sa.cand_key = reinterpret_cast<uint32_t *>(wsb + w.cand_key);
   sa.cand_idx = reinterpret_cast<int32_t *>(wsb + w.cand_idx);
@@ -295,7 +319,7 @@ s5_status s5_swa_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, cons
 
 s5_status s5_reset_device_error(void *workspace, s5_stream_t stream) {
   if (workspace == nullptr) return S5_ERR_INVALID_ARG;
-  return cuda_status(cudaMemsetAsync(workspace, 0, sizeof(ErrRec), reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(cudaMemsetAsync(workspace, 0, kWsFixed, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 s5_status s5_get_device_error(void *workspace, s5_stream_t stream, int32_t *code, int32_t *info) {

@@ -40,11 +40,61 @@ constexpr int kListOff = kRingBytes + kQBytes;
 constexpr int kBarOff = kListOff + 2 * kMaxList * 4;
 constexpr int kAttnSmem = kBarOff + kWarps * kStages * 8 + 1024;  // + alignment slack
 constexpr uint64_t kWaitNs = 2000000000ull;                       // 2 s per wait
+constexpr int kMaxSplitMerge = 32;
 
 // byte offset of (token row r, dim d) inside a 128B-swizzled [8][192] bf16 tile
 __device__ __forceinline__ uint32_t swz(int r, int d) {
   const uint32_t off = (uint32_t)((r * 3 + (d >> 6)) * 128 + (d & 63) * 2);
   return off ^ (((off >> 7) & 7u) << 4);
+}
+
+// Merge weights of the partitions of one (row, head): w[p] = exp2(lse_p - M) / L
+// in partition order, and the merged natural-log lse.  The same arithmetic
+// wherever the merge runs, so results do not depend on which partition
+// finished last.
+__device__ __forceinline__ void partition_weights(const float *pl, int n, float *w, float &lse_nat) {
+  float M = -INFINITY;
+  for (int p = 0; p < n; ++p) M = fmaxf(M, __ldcg(pl + p));
+  const float Mu = (M == -INFINITY) ? 0.f : M;
+  float L = 0.f;
+  for (int p = 0; p < n; ++p) {
+    const float lp = __ldcg(pl + p);
+    L += (lp == -INFINITY) ? 0.f : hw_exp2(lp - Mu);
+  }
+  const float inv = (L > 0.f) ? 1.f / L : 0.f;
+  for (int p = 0; p < n; ++p) {
+    const float lp = __ldcg(pl + p);
+    w[p] = (lp == -INFINITY) ? 0.f : hw_exp2(lp - Mu) * inv;
+  }
+  lse_nat = (L > 0.f) ? (M + hw_log2(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+__device__ __forceinline__ void store_bf16x4(__nv_bfloat16 *dst, float4 v) {
+  uint2 w2;
+  w2.x = pack_bf16(v.x, v.y);
+  w2.y = pack_bf16(v.z, v.w);
+  *reinterpret_cast<uint2 *>(dst) = w2;
+}
+
+// Standalone merge for batches whose partitions are not merged in place:
+// one CTA per (row, head), one float4 of dims per thread.
+__global__ void __launch_bounds__(kD / 4) s5_combine_kernel(const AttnArgs a) {
+  const size_t rh = blockIdx.x;
+  const int n = a.n_split;
+  float w[kMaxSplitMerge];
+  float lse;
+  partition_weights(a.part_lse + rh * n, n, w, lse);
+  const int d = threadIdx.x * 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int p = 0; p < n; ++p) {
+    const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (rh * n + p) * kD + d));
+    acc.x = fmaf(w[p], v.x, acc.x);
+    acc.y = fmaf(w[p], v.y, acc.y);
+    acc.z = fmaf(w[p], v.z, acc.z);
+    acc.w = fmaf(w[p], v.w, acc.w);
+  }
+  store_bf16x4(reinterpret_cast<__nv_bfloat16 *>(a.out) + rh * kD + d, acc);
+  if (threadIdx.x == 0 && a.lse != nullptr) a.lse[rh] = lse;
 }
 
 template <int MODE>
@@ -101,32 +151,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   const int i_beg = min(n_list, p * chunk);
   const int n_items = min(n_list, i_beg + chunk) - i_beg;
 
-  // ---- resolve blocks to TMA rows -----------------------------------------------
+  // (block ids and TMA rows are resolved by each warp for its own items, below)
   const int32_t *pt = a.page_table + (size_t)max(s, 0) * a.max_pages;
-  for (int i = tid; i < n_items; i += kWarps * 32) {
-    const int li = i_beg + i;
-    int b;
-    bool ok = true;
-    if (MODE == kModeSparse) {
-      if (li < n_sel) {
-        b = __ldg(a.sel + (size_t)r * a.topk + li);
-        ok = (b >= 0) && (b < c);
-      } else {
-        b = c;
-      }
-    } else {
-      b = b_first + li;
-    }
-    int row = -1;
-    if (ok) {
-      const int ph = __ldg(pt + b / kBpp);
-      if (ph >= 0 && ph < a.num_pages) row = ((ph * kKv + g) * kPage) + (b % kBpp) * kBlk;
-      else ok = false;
-    }
-    if (!ok) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
-    blist[i] = ok ? b : -1;
-    brow[i] = row;
-  }
   // ---- query tile of the group: 16 heads x 192, padded rows -----------------------
   {
     const uint4 *qg = reinterpret_cast<const uint4 *>(a.q) + ((size_t)r * kHeads + g * kHpg) * (kD / 8);
@@ -171,9 +197,39 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       }
     }
   };
+  // resolve this warp's items to block ids and TMA rows (lane k: items k, k+32, ...);
+  // the first 32 are resolved before the first loads are issued
+  auto resolve = [&](int k) {
+    const int li = i_beg + w_beg + k;
+    int b;
+    bool ok = true;
+    if (MODE == kModeSparse) {
+      if (li < n_sel) {
+        b = __ldg(a.sel + (size_t)r * a.topk + li);
+        ok = (b >= 0) && (b < c);
+      } else {
+        b = c;
+      }
+    } else {
+      b = b_first + li;
+    }
+    int row = -1;
+    if (ok) {
+      const int ph = __ldg(pt + b / kBpp);
+      if (ph >= 0 && ph < a.num_pages) row = ((ph * kKv + g) * kPage) + (b % kBpp) * kBlk;
+      else ok = false;
+    }
+    if (!ok) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
+    blist[w_beg + k] = ok ? b : -1;
+    brow[w_beg + k] = row;
+  };
+  if (lane < w_n) resolve(lane);
+  __syncwarp();
   if (lane == 0) {
     for (int j = 0; j < kStages && j < n_pairs; ++j) issue(j);
   }
+  for (int k = lane + 32; k < w_n; k += 32) resolve(k);
+  __syncwarp();
 
   // Q fragments (A operand) for the 12 k-steps of 16 dims
   uint32_t qa[kD / 16][4];
@@ -390,27 +446,60 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       if ((tid & 7) == 0) a.part_lse[rh * a.n_split + p] = lse2;
     }
   }
-}
+  if (a.n_split == 1 || a.merge_cnt == nullptr) return;
 
-// Merge the partitions of every (row, head) in partition order.
-__global__ void __launch_bounds__(kD) s5_combine_kernel(const AttnArgs a) {
-  const size_t rh = blockIdx.x;
-  const int d = threadIdx.x;
-  const int n = a.n_split;
-  const float *pl = a.part_lse + rh * n;
-  float M = -INFINITY;
-  for (int p = 0; p < n; ++p) M = fmaxf(M, pl[p]);
-  const float Mu = (M == -INFINITY) ? 0.f : M;
-  float L = 0.f, acc = 0.f;
-  for (int p = 0; p < n; ++p) {
-    const float lp = pl[p];
-    const float w = (lp == -INFINITY) ? 0.f : hw_exp2(lp - Mu);
-    L += w;
-    acc += w * a.part_o[(rh * n + p) * kD + d];
+  // ---- the last partition CTA of (r, g) to arrive merges every partition ----
+  __shared__ int is_last;
+  __shared__ float w_s[kHpg][kMaxSplitMerge];
+  __shared__ float lse_s[kHpg];
+  __threadfence();  // publish this CTA's partial before counting it
+  __syncthreads();
+  if (tid == 0) {
+    const uint32_t prev = atomicAdd(a.merge_cnt + (size_t)r * kKv + g, 1u);
+    is_last = (prev == (uint32_t)a.n_split - 1);
   }
-  const float res = (L > 0.f) ? acc / L : 0.f;
-  reinterpret_cast<__nv_bfloat16 *>(a.out)[rh * kD + d] = __float2bfloat16_rn(res);
-  if (d == 0 && a.lse != nullptr) a.lse[rh] = (L > 0.f) ? (M + hw_log2(L)) * 0.69314718055994531f : -INFINITY;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const int n = a.n_split;
+  const size_t rh0 = (size_t)r * kHeads + g * kHpg;
+  if (tid < kHpg) partition_weights(a.part_lse + (rh0 + tid) * n, n, w_s[tid], lse_s[tid]);
+  __syncthreads();
+  {
+    const int h = tid >> 3;          // 16 heads x 8 threads
+    const int c0 = (tid & 7) * 6;    // 6 float4 columns each
+    const size_t rh = rh0 + h;
+    const float4 *src = reinterpret_cast<const float4 *>(a.part_o + rh * n * kD) + c0;
+    float4 acc[6];
+#pragma unroll
+    for (int c = 0; c < 6; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p0 = 0; p0 < n; p0 += 4) {
+      float4 v[4][6];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int c = 0; c < 6; ++c)
+          if (p0 + q < n) v[q][c] = __ldcg(src + (size_t)(p0 + q) * (kD / 4) + c);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (p0 + q < n) {
+          const float wp = w_s[h][p0 + q];
+#pragma unroll
+          for (int c = 0; c < 6; ++c) {
+            acc[c].x = fmaf(wp, v[q][c].x, acc[c].x);
+            acc[c].y = fmaf(wp, v[q][c].y, acc[c].y);
+            acc[c].z = fmaf(wp, v[q][c].z, acc[c].z);
+            acc[c].w = fmaf(wp, v[q][c].w, acc[c].w);
+          }
+        }
+      }
+    }
+    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(a.out) + rh * kD;
+#pragma unroll
+    for (int c = 0; c < 6; ++c) store_bf16x4(out + 4 * (c0 + c), acc[c]);
+    if ((tid & 7) == 0 && a.lse != nullptr) a.lse[rh] = lse_s[h];
+  }
+  if (tid == 0) a.merge_cnt[(size_t)r * kKv + g] = 0u;  // ready for the next call
 }
 
 cudaError_t launch_gqa_decode(int mode, const AttnArgs &a, const CUtensorMap &tk, const CUtensorMap &tv,
@@ -428,8 +517,8 @@ cudaError_t launch_gqa_decode(int mode, const AttnArgs &a, const CUtensorMap &tk
     gqa_decode_kernel<kModeSwa><<<grid, kWarps * 32, kAttnSmem, st>>>(a, tk, tv);
   }
   e = cudaGetLastError();
-  if (e != cudaSuccess || a.n_split == 1) return e;
-  s5_combine_kernel<<<(unsigned)total_q * kHeads, kD, 0, st>>>(a);
+  if (e != cudaSuccess || a.n_split == 1 || a.merge_cnt != nullptr) return e;
+  s5_combine_kernel<<<(unsigned)total_q * kHeads, kD / 4, 0, st>>>(a);
   return cudaGetLastError();
 }
 

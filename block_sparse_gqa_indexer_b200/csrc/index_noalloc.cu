@@ -73,7 +73,7 @@ extern "C" s5_status s5_index_score_topk_noalloc(const s5_index_desc *index, con
 
   // scratch layout: error record (256 B), then fp32 scores [total_q][stride]
   const int hist = batch->max_len >= 1 ? (batch->max_len - 1) / kBlk : 0;
-  const int stride = hist > 1 ? hist : 1;
+  const int stride = ((hist > 1 ? hist : 1) + 3) & ~3;  // rows start 16-byte aligned
   if (stride > kNoAllocMaxHistory) return S5_ERR_WORKSPACE;
   const size_t need = kWsHeader + (size_t)batch->total_q * stride * sizeof(float);
   if (need > kNoAllocScratchBytes) return S5_ERR_WORKSPACE;

@@ -153,145 +153,150 @@ __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
 // list position, emitted in list order.
 // ============================================================================
 
+template <int NT>
 struct SelectSmem {
-  uint32_t hist[256];
-  int warp_a[32];
-  int warp_b[32];
+  uint32_t whist[NT / 32][256];  // one private histogram per warp
+  int wsum[32];
+  int scan_a[32];
+  int scan_b[32];
   uint32_t digit, above, bin_cnt;
 };
 
-// keys[0..n) in shared memory.  Calls emit(pos, i) for the k selected list
-// positions i, pos = 0..k-1 in increasing i.  Requires n > k >= 1.
+// Exclusive prefix sum of v over threads in thread order.
+template <int NT>
+__device__ __forceinline__ int block_excl_scan(int v, int *buf) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) buf[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int x = (lane < NT / 32) ? buf[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += o;
+    }
+    if (lane < NT / 32) buf[lane] = x;  // inclusive warp totals
+  }
+  __syncthreads();
+  return (warp > 0 ? buf[warp - 1] : 0) + incl - v;
+}
+
+// Top-k of a list of n keys (n > k >= 1).  Thread t owns list positions
+// t*E .. t*E+E-1, held in shared memory as ks[j * NT + t].  Radix select on
+// 8-bit digits from the top: each pass histograms the digit of the keys that
+// still match the chosen prefix into per-warp histograms (no atomics shared
+// between warps), sums them and picks the bin holding the kk-th largest; it
+// stops early when that whole bin is taken.  Then the keys above the final
+// range and the first kk keys inside it (list order) are emitted as
+// emit(pos, list_position), pos = 0..k-1 in list order.
 template <int NT, typename Emit>
-__device__ void cta_select(const uint32_t *keys, int n, int k, SelectSmem &sm, Emit emit) {
+__device__ void cta_select(const uint32_t *ks, int n, int E, int k, SelectSmem<NT> &sm, Emit emit) {
   constexpr int NW = NT / 32;
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
+  static_assert(NT >= 256, "one thread per bin when summing histograms");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int first = tid * E;
+  const int mine = max(0, min(E, n - first));
   uint32_t prefix = 0, mask = 0;
-  int kk = k;  // rank still to place among keys matching (prefix, mask)
-  uint32_t t_lo = 0, t_hi = 0;
-  bool done = false;
-  for (int shift = 24; shift >= 0 && !done; shift -= 8) {
-    for (int i = tid; i < 256; i += NT) sm.hist[i] = 0;
+  int kk = k;
+  uint32_t *wh = sm.whist[warp];
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = lane; i < 256; i += 32) wh[i] = 0;
+    __syncwarp();
+    for (int j = 0; j < mine; ++j) {
+      const uint32_t key = ks[j * NT + tid];
+      if ((key & mask) == prefix) atomicAdd(&wh[(key >> shift) & 255u], 1u);
+    }
     __syncthreads();
-    for (int base = warp * 32; base < n; base += NT) {
-      const int i = base + lane;
-      const uint32_t key = (i < n) ? keys[i] : 0u;
-      const bool match = (i < n) && ((key & mask) == prefix);
-      const unsigned act = __ballot_sync(0xffffffffu, match);
-      if (match) {
-        const uint32_t d = (key >> shift) & 255u;
-        const unsigned peers = __match_any_sync(act, d);
-        if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[d], (uint32_t)__popc(peers));
+    // thread i < 256 owns bin 255 - i: bins in descending order
+    int cnt = 0;
+    if (tid < 256) {
+      const int b = 255 - tid;
+#pragma unroll 8
+      for (int w = 0; w < NW; ++w) cnt += (int)sm.whist[w][b];
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31 && warp < 8) sm.wsum[warp] = incl;
+    __syncthreads();
+    if (tid < 256) {
+      int base = 0;
+      for (int w = 0; w < warp; ++w) base += sm.wsum[w];
+      const int excl = base + incl - cnt;
+      if (excl < kk && kk <= excl + cnt) {
+        sm.digit = (uint32_t)(255 - tid);
+        sm.above = (uint32_t)excl;
+        sm.bin_cnt = (uint32_t)cnt;
       }
     }
     __syncthreads();
-    if (warp == 0) {
-      // lane l scans bins 255-8l .. 248-8l (descending)
-      uint32_t c8[8];
-      uint32_t sum = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        c8[i] = sm.hist[255 - (lane * 8 + i)];
-        sum += c8[i];
-      }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-      }
-      const uint32_t excl = incl - sum;
-      if (excl < (uint32_t)kk && (uint32_t)kk <= incl) {
-        uint32_t acc = excl;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (acc < (uint32_t)kk && (uint32_t)kk <= acc + c8[i]) {
-            sm.digit = 255 - (lane * 8 + i);
-            sm.above = acc;
-            sm.bin_cnt = c8[i];
-          }
-          acc += c8[i];
-        }
-      }
-    }
-    __syncthreads();
-    const uint32_t d = sm.digit;
     kk -= (int)sm.above;
-    prefix |= d << shift;
+    prefix |= sm.digit << shift;
     mask |= 255u << shift;
-    if ((int)sm.bin_cnt == kk || shift == 0) {
-      // either every key in this bin is taken, or the threshold is exact
-      t_lo = prefix;
-      t_hi = prefix | ~mask;
-      done = true;
-    }
-    __syncthreads();
+    const bool stop = ((int)sm.bin_cnt == kk);
+    __syncthreads();  // sm.digit / above / bin_cnt are rewritten by the next pass
+    if (stop) break;
   }
-  // keys > t_hi are taken; of the keys in [t_lo, t_hi] the first kk in list order
-  const int per_warp = (((n + NW - 1) / NW) + 31) & ~31;
-  const int wbeg = warp * per_warp;
-  const int wend = min(n, wbeg + per_warp);
-  const unsigned lt = (1u << lane) - 1u;
-  int cnt_in = 0;
-  for (int base = wbeg; base < wend; base += 32) {
-    const int i = base + lane;
-    const bool inr = (i < wend) && keys[i] >= t_lo && keys[i] <= t_hi;
-    cnt_in += __popc(__ballot_sync(0xffffffffu, inr));
+  const uint32_t t_lo = prefix, t_hi = prefix | ~mask;  // keys in [t_lo, t_hi] compete for the last kk places
+  int in = 0, gt = 0;
+  for (int j = 0; j < mine; ++j) {
+    const uint32_t key = ks[j * NT + tid];
+    gt += key > t_hi;
+    in += (key >= t_lo) & (key <= t_hi);
   }
-  if (lane == 0) sm.warp_a[warp] = cnt_in;
-  __syncthreads();
-  if (tid == 0) {
-    int acc = 0;
-    for (int w = 0; w < NW; ++w) {
-      const int v = sm.warp_a[w];
-      sm.warp_a[w] = acc;
-      acc += v;
-    }
-  }
-  __syncthreads();
-  int rank = sm.warp_a[warp];
-  int cnt_take = 0;
-  for (int base = wbeg; base < wend; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = (i < wend) ? keys[i] : 0u;
-    const bool gt = (i < wend) && key > t_hi;
-    const bool inr = (i < wend) && key >= t_lo && key <= t_hi;
-    const unsigned bal = __ballot_sync(0xffffffffu, inr);
-    const bool take = gt || (inr && (rank + __popc(bal & lt)) < kk);
-    rank += __popc(bal);
-    cnt_take += __popc(__ballot_sync(0xffffffffu, take));
-  }
-  if (lane == 0) sm.warp_b[warp] = cnt_take;
-  __syncthreads();
-  if (tid == 0) {
-    int acc = 0;
-    for (int w = 0; w < NW; ++w) {
-      const int v = sm.warp_b[w];
-      sm.warp_b[w] = acc;
-      acc += v;
-    }
-  }
-  __syncthreads();
-  rank = sm.warp_a[warp];
-  int pos = sm.warp_b[warp];
-  for (int base = wbeg; base < wend; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = (i < wend) ? keys[i] : 0u;
-    const bool gt = (i < wend) && key > t_hi;
-    const bool inr = (i < wend) && key >= t_lo && key <= t_hi;
-    const unsigned bal = __ballot_sync(0xffffffffu, inr);
-    const bool take = gt || (inr && (rank + __popc(bal & lt)) < kk);
-    const unsigned tb = __ballot_sync(0xffffffffu, take);
-    if (take) emit(pos + __popc(tb & lt), i);
-    pos += __popc(tb);
-    rank += __popc(bal);
+  const int in_before = block_excl_scan<NT>(in, sm.scan_a);
+  const int take = gt + max(0, min(in, kk - in_before));
+  int pos = block_excl_scan<NT>(take, sm.scan_b);
+  int r = in_before;
+  for (int j = 0; j < mine; ++j) {
+    const uint32_t key = ks[j * NT + tid];
+    const bool inr = (key >= t_lo) & (key <= t_hi);
+    const bool tk = key > t_hi || (inr && r < kk);
+    r += inr;
+    if (tk) emit(pos++, first + j);
   }
   __syncthreads();
 }
 
-// Query row -> (history blocks c).  Returns false (and records) on bad batch data.
+// Positions per thread for an n-long list: a multiple of 4 (whole float4 loads).
+template <int NT>
+__host__ __device__ constexpr int owned_per_thread(int n) {
+  return (((n + NT - 1) / NT) + 3) & ~3;
+}
+
+// Stage the n scores row[0..n) as keys in the owner layout; a thread's loads
+// are all in flight together.  row is 16-byte aligned and readable up to the
+// next multiple of 4.
+template <int NT>
+__device__ __forceinline__ void load_keys(const float *row, int n, int E, uint32_t *ks) {
+  const int t = threadIdx.x;
+  const float4 *r4 = reinterpret_cast<const float4 *>(row + (size_t)t * E);
+  constexpr int kMaxQ = 8;  // E <= 32
+  float4 v[kMaxQ];
+#pragma unroll
+  for (int q = 0; q < kMaxQ; ++q)
+    if (4 * q < E && t * E + 4 * q < n) v[q] = __ldcg(r4 + q);
+#pragma unroll
+  for (int q = 0; q < kMaxQ; ++q) {
+    if (4 * q < E) {
+      const int i0 = t * E + 4 * q;
+      const float f[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ks[(4 * q + e) * NT + t] = (i0 + e < n) ? score_key(f[e]) : 0u;
+    }
+  }
+}
+
+// Query row -> (history blocks c).  Returns false on bad batch data.
 __device__ __forceinline__ bool row_history(const SelectArgs &a, int r, int &c) {
   const int s = seq_of_row(a.cu_q, a.batch, r);
   if (s < 0) return false;
@@ -301,31 +306,35 @@ __device__ __forceinline__ bool row_history(const SelectArgs &a, int r, int &c) 
   return true;
 }
 
-// Single stage: one CTA per query row, the row's keys staged in shared memory.
+__device__ __forceinline__ void write_all(int32_t *out, int n, int topk, int nt) {
+  for (int i = threadIdx.x; i < topk; i += nt) out[i] = (i < n) ? i : -1;
+}
+
+// Single stage: one CTA per query row.
 template <int NT>
 __global__ void __launch_bounds__(NT) topk_select_kernel(SelectArgs a) {
-  extern __shared__ __align__(16) uint32_t keys_s[];
-  __shared__ SelectSmem sm;
+  extern __shared__ __align__(16) uint32_t ks[];
+  __shared__ SelectSmem<NT> sm;
   const int r = blockIdx.x;
+  int32_t *out = a.sel + (size_t)r * a.topk;
   int c = 0;
   if (!row_history(a, r, c)) {
     if (threadIdx.x == 0) {
       record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
       a.sel_count[r] = 0;
     }
-    for (int i = threadIdx.x; i < a.topk; i += NT) a.sel[(size_t)r * a.topk + i] = -1;
+    write_all(out, 0, a.topk, NT);
     return;
   }
-  int32_t *out = a.sel + (size_t)r * a.topk;
   if (c <= a.topk) {
-    for (int i = threadIdx.x; i < a.topk; i += NT) out[i] = (i < c) ? i : -1;
+    write_all(out, c, a.topk, NT);
     if (threadIdx.x == 0) a.sel_count[r] = c;
     return;
   }
-  const float *sc = a.scores + (size_t)r * a.score_stride;
-  for (int i = threadIdx.x; i < c; i += NT) keys_s[i] = score_key(__ldg(sc + i));
+  const int E = owned_per_thread<NT>(c);
+  load_keys<NT>(a.scores + (size_t)r * a.score_stride, c, E, ks);
   __syncthreads();
-  cta_select<NT>(keys_s, c, a.topk, sm, [&](int pos, int i) { out[pos] = i; });
+  cta_select<NT>(ks, c, E, a.topk, sm, [&](int pos, int i) { out[pos] = i; });
   if (threadIdx.x == 0) a.sel_count[r] = a.topk;
 }
 
@@ -333,8 +342,8 @@ __global__ void __launch_bounds__(NT) topk_select_kernel(SelectArgs a) {
 // `seg` blocks, as (key, block) candidates in block order.
 template <int NT>
 __global__ void __launch_bounds__(NT) topk_segment_kernel(SelectArgs a) {
-  extern __shared__ __align__(16) uint32_t keys_s[];
-  __shared__ SelectSmem sm;
+  extern __shared__ __align__(16) uint32_t ks[];
+  __shared__ SelectSmem<NT> sm;
   const int r = blockIdx.y;
   const int sg = blockIdx.x;
   int c = 0;
@@ -347,60 +356,69 @@ __global__ void __launch_bounds__(NT) topk_segment_kernel(SelectArgs a) {
   const float *sc = a.scores + (size_t)r * a.score_stride + b0;
   if (n <= a.topk) {
     for (int i = threadIdx.x; i < n; i += NT) {
-      a.cand_key[cbase + i] = score_key(__ldg(sc + i));
+      a.cand_key[cbase + i] = score_key(__ldcg(sc + i));
       a.cand_idx[cbase + i] = b0 + i;
     }
     return;
   }
-  for (int i = threadIdx.x; i < n; i += NT) keys_s[i] = score_key(__ldg(sc + i));
+  const int E = owned_per_thread<NT>(n);
+  load_keys<NT>(sc, n, E, ks);
   __syncthreads();
-  cta_select<NT>(keys_s, n, a.topk, sm, [&](int pos, int i) {
-    a.cand_key[cbase + pos] = keys_s[i];
+  cta_select<NT>(ks, n, E, a.topk, sm, [&](int pos, int i) {
+    a.cand_key[cbase + pos] = ks[(i % E) * NT + i / E];
     a.cand_idx[cbase + pos] = b0 + i;
   });
 }
 
-// Stage 2: the top-k of the concatenated candidates of every segment.
+// Stage 2: the top-k of the concatenated candidates of every segment.  Every
+// segment but the last holds exactly topk candidates, so candidate L of the
+// row sits at slot L % topk of segment L / topk.
 template <int NT>
 __global__ void __launch_bounds__(NT) topk_merge_kernel(SelectArgs a) {
   extern __shared__ __align__(16) uint32_t smem[];
-  __shared__ SelectSmem sm;
+  __shared__ SelectSmem<NT> sm;
   const int r = blockIdx.x;
+  int32_t *out = a.sel + (size_t)r * a.topk;
   int c = 0;
   if (!row_history(a, r, c)) {
     if (threadIdx.x == 0) {
       record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
       a.sel_count[r] = 0;
     }
-    for (int i = threadIdx.x; i < a.topk; i += NT) a.sel[(size_t)r * a.topk + i] = -1;
+    write_all(out, 0, a.topk, NT);
     return;
   }
-  int32_t *out = a.sel + (size_t)r * a.topk;
   if (c <= a.topk) {
-    for (int i = threadIdx.x; i < a.topk; i += NT) out[i] = (i < c) ? i : -1;
+    write_all(out, c, a.topk, NT);
     if (threadIdx.x == 0) a.sel_count[r] = c;
     return;
   }
   const int nseg = (c + a.seg - 1) / a.seg;
-  uint32_t *keys_s = smem;
-  int32_t *idx_s = reinterpret_cast<int32_t *>(smem + (size_t)a.n_seg * a.topk);
-  int n = 0;
-  for (int sg = 0; sg < nseg; ++sg) {
-    const int m = min(a.topk, min(a.seg, c - sg * a.seg));
-    const size_t cbase = ((size_t)r * a.n_seg + sg) * a.topk;
-    for (int i = threadIdx.x; i < m; i += NT) {
-      keys_s[n + i] = a.cand_key[cbase + i];
-      idx_s[n + i] = a.cand_idx[cbase + i];
+  const int last = c - (nseg - 1) * a.seg;
+  const int n = (nseg - 1) * a.topk + min(a.topk, last);
+  const int E = owned_per_thread<NT>(n);
+  uint32_t *ks = smem;
+  int32_t *is = reinterpret_cast<int32_t *>(smem + (size_t)E * NT);
+  const size_t rbase = (size_t)r * a.n_seg * a.topk;
+  for (int j = 0; j < E; ++j) {
+    const int L = threadIdx.x * E + j;
+    if (L < n) {
+      const size_t src = rbase + (size_t)(L / a.topk) * a.topk + (L % a.topk);
+      ks[j * NT + threadIdx.x] = __ldcg(a.cand_key + src);
+      is[j * NT + threadIdx.x] = __ldcg(a.cand_idx + src);
     }
-    n += m;
   }
   __syncthreads();
   if (n <= a.topk) {  // a single segment whose candidates are all taken
-    for (int i = threadIdx.x; i < a.topk; i += NT) out[i] = (i < n) ? idx_s[i] : -1;
+    for (int j = 0; j < E; ++j) {
+      const int L = threadIdx.x * E + j;
+      if (L < n) out[L] = is[j * NT + threadIdx.x];
+    }
+    for (int i = n + threadIdx.x; i < a.topk; i += NT) out[i] = -1;
     if (threadIdx.x == 0) a.sel_count[r] = n;
     return;
   }
-  cta_select<NT>(keys_s, n, a.topk, sm, [&](int pos, int i) { out[pos] = idx_s[i]; });
+  cta_select<NT>(ks, n, E, a.topk, sm, [&](int pos, int i) { out[pos] = is[(i % E) * NT + i / E]; });
   if (threadIdx.x == 0) a.sel_count[r] = a.topk;
 }
 
@@ -417,30 +435,39 @@ cudaError_t launch_index_score(const IndexScoreArgs &a, int max_q, int grid_page
   return cudaGetLastError();
 }
 
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = 1024;  // one CTA per row (rows of up to 16,384 blocks)
+constexpr int kSegThreads = 256;   // stage 1: one CTA per segment (E = seg / 256 <= 32)
+
+template <int NT>
+cudaError_t launch_merge(const SelectArgs &a, int total_q, cudaStream_t st) {
+  const size_t smem = (size_t)owned_per_thread<NT>(a.n_seg * a.topk) * NT * (sizeof(uint32_t) + sizeof(int32_t));
+  cudaError_t e = cudaFuncSetAttribute(topk_merge_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_merge_kernel<NT><<<total_q, NT, smem, st>>>(a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_topk_select(const SelectArgs &a, int total_q, bool two_stage, cudaStream_t st) {
   if (!two_stage) {
-    const size_t smem = (size_t)a.score_stride * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(topk_select_kernel<kSelThreads>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    constexpr int NT = kSelThreads;
+    const size_t smem = (size_t)owned_per_thread<NT>(a.score_stride) * NT * sizeof(uint32_t);
+    cudaError_t e = cudaFuncSetAttribute(topk_select_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    topk_select_kernel<kSelThreads><<<total_q, kSelThreads, smem, st>>>(a);
+    topk_select_kernel<NT><<<total_q, NT, smem, st>>>(a);
     return cudaGetLastError();
   }
-  const size_t smem1 = (size_t)a.seg * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(topk_segment_kernel<kSelThreads>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+  constexpr int NS = kSegThreads;
+  const size_t smem1 = (size_t)owned_per_thread<NS>(a.seg) * NS * sizeof(uint32_t);
+  cudaError_t e = cudaFuncSetAttribute(topk_segment_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem1);
   if (e != cudaSuccess) return e;
-  topk_segment_kernel<kSelThreads><<<dim3(a.n_seg, total_q), kSelThreads, smem1, st>>>(a);
+  topk_segment_kernel<NS><<<dim3(a.n_seg, total_q), NS, smem1, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem2 = (size_t)a.n_seg * a.topk * (sizeof(uint32_t) + sizeof(int32_t));
-  e = cudaFuncSetAttribute(topk_merge_kernel<kSelThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem2);
-  if (e != cudaSuccess) return e;
-  topk_merge_kernel<kSelThreads><<<total_q, kSelThreads, smem2, st>>>(a);
-  return cudaGetLastError();
+  // stage 2: at most 32 owned candidates per thread
+  if (a.n_seg * a.topk <= 32 * 512) return launch_merge<512>(a, total_q, st);
+  return launch_merge<1024>(a, total_q, st);
 }
 
 }  // namespace s5

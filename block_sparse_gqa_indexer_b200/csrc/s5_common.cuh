@@ -20,8 +20,11 @@ constexpr int kDx = S5_INDEX_DIM;           // 256
 constexpr int kMaxTopk = S5_MAX_TOPK;       // 512
 constexpr int kBlockBytes = kBlk * kD * 2;  // 3,072 bytes: one block of one group (K or V)
 
-// Workspace header: the device error record lives in the first 256 bytes.
+// Workspace header: the device error record lives in the first 256 bytes,
+// followed by the attention merge counters (4 per row for up to 1,024 rows).
 constexpr size_t kWsHeader = 256;
+constexpr size_t kWsCounterBytes = 16384;
+constexpr size_t kWsFixed = kWsHeader + kWsCounterBytes;  // first byte of per-call scratch
 
 struct ErrRec {
   int32_t code;

@@ -10,6 +10,7 @@ namespace s5 {
 constexpr int kModeSparse = 0;
 constexpr int kModeSwa = 1;
 constexpr int kMaxList = 544;  // blocks one attention CTA may own (>= 512 + 1)
+constexpr int kMaxMergeRows = 1024;  // rows whose partitions merge inside the attention kernel
 
 struct IndexScoreArgs {
   const void *key_pool;
@@ -64,6 +65,7 @@ struct AttnArgs {
   float *lse;
   float *part_o;    // [total_q * 64][n_split][192]
   float *part_lse;  // [total_q * 64][n_split]   (base-2)
+  uint32_t *merge_cnt;  // [total_q * 4] arrival counters (zero between calls), or null: separate merge kernel
   int32_t *err;
 };
 

@@ -117,8 +117,12 @@ typedef struct {
 
 /* Bytes of device workspace any of the calls below may use for this batch
  * (window: the largest sliding window that will be requested, or 0).  The
- * first 256 bytes hold the device error record: zero them once (or call
- * s5_reset_device_error) before first use; later calls keep them. */
+ * first S5_WS_FIXED_BYTES bytes hold the device error record and the
+ * attention partition counters: zero them once before first use (or call
+ * s5_reset_device_error); every call leaves the counters at zero again.  The
+ * rest is per-call scratch with no state between calls.  Calls that share a
+ * workspace must be ordered (one stream). */
+#define S5_WS_FIXED_BYTES (256 + 16384)
 s5_status s5_workspace_size(const s5_batch_desc *batch, int32_t window, size_t *bytes);
 
 /* Indexer: score every history block of every query row and keep the best
@@ -187,7 +191,8 @@ s5_status s5_index_score_topk_noalloc(const s5_index_desc *index, const s5_batch
                                       const void *q_index, int32_t topk, int32_t *sel, int32_t *sel_count,
                                       s5_stream_t stream);
 
-/* Zero the device error record (asynchronous, on `stream`). */
+/* Zero the first S5_WS_FIXED_BYTES of a workspace: the device error record
+ * and the partition counters (asynchronous, on `stream`). */
 s5_status s5_reset_device_error(void *workspace, s5_stream_t stream);
 
 /* Synchronise `stream` and read the device error record: *code is S5_OK or

@@ -251,3 +251,17 @@ def test_config5_hybrid_1m(lib):
             _check_no_device_error(lib, d)
         del d
         torch.cuda.empty_cache()
+
+
+def test_swa_many_rows_wide_window_separate_merge(lib):
+    # > 1,024 rows whose windows need two partitions each: partitions merge in
+    # the standalone kernel instead of inside the attention kernel
+    w = S.Workload(ctx=[8000], nq=[1100], seed=20)
+    d = DeviceInputs(w, lib, with_index=False)
+    d.ws = lib.new_workspace(d.batch, window=8192)
+    lib.s5_swa_gqa_attn(d.k_pool, d.v_pool, d.batch, d.q, 8192, O.DEFAULT_SM_SCALE, d.out, d.lse, d.ws)
+    rows = sample_rows(w.total_q, 6, 5)
+    want, want_lse = oracle_swa(w, rows, 8192)
+    assert_attn_close(d.out.float().cpu().numpy()[rows], want, "swa W=8192, 1100 rows")
+    assert np.abs(d.lse.cpu().numpy()[rows] - want_lse).max() <= LSE_ABS
+    _check_no_device_error(lib, d)
