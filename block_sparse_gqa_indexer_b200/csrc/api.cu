@@ -61,8 +61,10 @@ s5_status check_kv(const s5_kv_desc *kv) {
 
 // ---------------------------------------------------------------- workspace layout
 
+constexpr int kMaxHistRows = 1024;  // decode / verify batches: rows get a score histogram
+
 struct IndexWs {
-  size_t scores, cand_key, cand_idx, end;
+  size_t scores, cand_key, cand_idx, hist, hist_bytes, end;
   int stride, seg, n_seg;
   bool two_stage;
 };
@@ -80,6 +82,9 @@ IndexWs index_ws(const s5_batch_desc *b) {
   off = align_up(off + (size_t)b->total_q * w.n_seg * kMaxTopk * sizeof(uint32_t), 256);
   w.cand_idx = off;
   off = align_up(off + (size_t)b->total_q * w.n_seg * kMaxTopk * sizeof(int32_t), 256);
+  w.hist = off;
+  w.hist_bytes = (!w.two_stage && b->total_q <= kMaxHistRows) ? (size_t)b->total_q * kHistBins * sizeof(uint32_t) : 0;
+  off = align_up(off + w.hist_bytes, 256);
   w.end = off;
   return w;
 }
@@ -213,6 +218,7 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   a.ctx_lens = b->ctx_lens;
   a.cu_q = b->cu_q;
   a.batch = b->batch;
+  a.total_q = b->total_q;
   a.max_len = b->max_len;
   a.num_pages = kv->num_pages;
   a.scale_log2 = sm_scale * 1.4426950408889634f;
@@ -280,7 +286,9 @@ s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *b
   ia.score_stride = w.stride;
   ia.pages_per_cta = kScorePagesPerCta;
   ia.topk = topk;
+  ia.hist = w.hist_bytes ? reinterpret_cast<uint32_t *>(wsb + w.hist) : nullptr;
   ia.err = err;
+  if (ia.hist != nullptr && cudaMemsetAsync(ia.hist, 0, w.hist_bytes, cs) != cudaSuccess) return S5_ERR_CUDA;
   const int pages = (w.stride + kBpp - 1) / kBpp;
   const int grid_pages = (pages + kScorePagesPerCta - 1) / kScorePagesPerCta;
   cudaError_t e = launch_index_score(ia, batch->max_q, grid_pages, batch->batch, cs);
@@ -292,6 +300,7 @@ s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *b
   sa.ctx_lens = batch->ctx_lens;
   sa.cu_q = batch->cu_q;
   sa.batch = batch->batch;
+  sa.total_q = batch->total_q;
   sa.topk = topk;
   sa.sel = sel;
   sa.sel_count = sel_count;
@@ -299,6 +308,7 @@ s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *b
   sa.n_seg = w.n_seg;
   sa.cand_key = reinterpret_cast<uint32_t *>(wsb + w.cand_key);
   sa.cand_idx = reinterpret_cast<int32_t *>(wsb + w.cand_idx);
+  sa.hist = ia.hist;
   sa.err = err;
   return cuda_status(launch_topk_select(sa, batch->total_q, w.two_stage, cs));
 }

@@ -54,16 +54,16 @@ __device__ __forceinline__ uint32_t swz(int r, int d) {
 // finished last.
 __device__ __forceinline__ void partition_weights(const float *pl, int n, float *w, float &lse_nat) {
   float M = -INFINITY;
-  for (int p = 0; p < n; ++p) M = fmaxf(M, __ldcg(pl + p));
+  for (int p = 0; p < n; ++p) M = fmaxf(M, ld_cg(pl + p));
   const float Mu = (M == -INFINITY) ? 0.f : M;
   float L = 0.f;
   for (int p = 0; p < n; ++p) {
-    const float lp = __ldcg(pl + p);
+    const float lp = ld_cg(pl + p);
     L += (lp == -INFINITY) ? 0.f : hw_exp2(lp - Mu);
   }
   const float inv = (L > 0.f) ? 1.f / L : 0.f;
   for (int p = 0; p < n; ++p) {
-    const float lp = __ldcg(pl + p);
+    const float lp = ld_cg(pl + p);
     w[p] = (lp == -INFINITY) ? 0.f : hw_exp2(lp - Mu) * inv;
   }
   lse_nat = (L > 0.f) ? (M + hw_log2(L)) * 0.69314718055994531f : -INFINITY;
@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(kD / 4) s5_combine_kernel(const AttnArgs a) {
   const int d = threadIdx.x * 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int p = 0; p < n; ++p) {
-    const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (rh * n + p) * kD + d));
+    const float4 v = ld_cg(reinterpret_cast<const float4 *>(a.part_o + (rh * n + p) * kD + d));
     acc.x = fmaf(w[p], v.x, acc.x);
     acc.y = fmaf(w[p], v.y, acc.y);
     acc.z = fmaf(w[p], v.z, acc.z);
@@ -117,17 +117,27 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   const int r = blockIdx.z;
 
   // ---- the unit's token range -------------------------------------------------
-  const int s = seq_of_row(a.cu_q, a.batch, r);
-  int t = -1, lo_tok = 0, n_list = 0, b_first = 0, n_sel = 0;
-  bool bad = (s < 0);
-  if (!bad) {
-    t = __ldg(a.ctx_lens + s) + (r - __ldg(a.cu_q + s));
-    bad = (t < 0) || (t >= a.max_pages * kPage) || (t >= a.max_len);
+  if (tid < kWarps * kStages) mbar_init(bars + tid, 1);
+  fence_mbar_init();
+  // programmatic launch: everything above touches shared memory only; every
+  // global input (batch data, q, the selection) is read after this wait
+  pdl_wait();
+  int s = -1, t = -1, lo_tok = 0, n_list = 0, b_first = 0, n_sel = 0;
+  const int sel_cnt = (MODE == kModeSparse) ? ld_cg(a.sel_count + r) : 0;
+  bool bad = !locate_row(a.cu_q, a.ctx_lens, a.batch, r, row_guess(r, a.batch, a.total_q), s, t);
+  if (!bad) bad = (t < 0) || (t >= a.max_pages * kPage) || (t >= a.max_len);
+  // ---- query tile of the group: 16 heads x 192, padded rows ----
+  {
+    const uint4 *qg = reinterpret_cast<const uint4 *>(a.q) + ((size_t)r * kHeads + g * kHpg) * (kD / 8);
+    for (int i = tid; i < kHpg * (kD / 8); i += kWarps * 32) {
+      const int h = i / (kD / 8), cc = i % (kD / 8);
+      *reinterpret_cast<uint4 *>(q_s + h * kQStride + cc * 16) = ld_cg(qg + i);
+    }
   }
   const int c = bad ? 0 : t / kBlk;
   if (!bad) {
     if (MODE == kModeSparse) {
-      n_sel = __ldg(a.sel_count + r);
+      n_sel = sel_cnt;
       if (n_sel < 0 || n_sel > a.topk || n_sel > c) {
         bad = true;
       } else {
@@ -153,18 +163,6 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
 
   // (block ids and TMA rows are resolved by each warp for its own items, below)
   const int32_t *pt = a.page_table + (size_t)max(s, 0) * a.max_pages;
-  // ---- query tile of the group: 16 heads x 192, padded rows -----------------------
-  {
-    const uint4 *qg = reinterpret_cast<const uint4 *>(a.q) + ((size_t)r * kHeads + g * kHpg) * (kD / 8);
-    for (int i = tid; i < kHpg * (kD / 8); i += kWarps * 32) {
-      const int h = i / (kD / 8), cc = i % (kD / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (n_list > 0) v = __ldg(qg + i);
-      *reinterpret_cast<uint4 *>(q_s + h * kQStride + cc * 16) = v;
-    }
-  }
-  if (tid < kWarps * kStages) mbar_init(bars + tid, 1);
-  fence_mbar_init();
   __syncthreads();
 
   // ---- this warp's share ----------------------------------------------------------
@@ -205,7 +203,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     bool ok = true;
     if (MODE == kModeSparse) {
       if (li < n_sel) {
-        b = __ldg(a.sel + (size_t)r * a.topk + li);
+        b = ld_cg(a.sel + (size_t)r * a.topk + li);
         ok = (b >= 0) && (b < c);
       } else {
         b = c;
@@ -215,7 +213,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     }
     int row = -1;
     if (ok) {
-      const int ph = __ldg(pt + b / kBpp);
+      const int ph = ld_cg(pt + b / kBpp);
       if (ph >= 0 && ph < a.num_pages) row = ((ph * kKv + g) * kPage) + (b % kBpp) * kBlk;
       else ok = false;
     }
@@ -479,7 +477,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int c = 0; c < 6; ++c)
-          if (p0 + q < n) v[q][c] = __ldcg(src + (size_t)(p0 + q) * (kD / 4) + c);
+          if (p0 + q < n) v[q][c] = ld_cg(src + (size_t)(p0 + q) * (kD / 4) + c);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         if (p0 + q < n) {
@@ -506,17 +504,23 @@ cudaError_t launch_gqa_decode(int mode, const AttnArgs &a, const CUtensorMap &tk
                               int total_q, cudaStream_t st) {
   dim3 grid(a.n_split, kKv, total_q);
   cudaError_t e;
-  if (mode == kModeSparse) {
-    e = cudaFuncSetAttribute(gqa_decode_kernel<kModeSparse>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kAttnSmem);
-    if (e != cudaSuccess) return e;
-    gqa_decode_kernel<kModeSparse><<<grid, kWarps * 32, kAttnSmem, st>>>(a, tk, tv);
-  } else {
-    e = cudaFuncSetAttribute(gqa_decode_kernel<kModeSwa>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
-    if (e != cudaSuccess) return e;
-    gqa_decode_kernel<kModeSwa><<<grid, kWarps * 32, kAttnSmem, st>>>(a, tk, tv);
-  }
-  e = cudaGetLastError();
+  auto kernel = (mode == kModeSparse) ? gqa_decode_kernel<kModeSparse> : gqa_decode_kernel<kModeSwa>;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+  if (e != cudaSuccess) return e;
+  // programmatic stream serialization: launch and barrier setup overlap the
+  // previous kernel; the kernel reads no global memory before pdl_wait()
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = kAttnSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kernel, a, tk, tv);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || a.n_split == 1 || a.merge_cnt != nullptr) return e;
   s5_combine_kernel<<<(unsigned)total_q * kHeads, kD / 4, 0, st>>>(a);
   return cudaGetLastError();

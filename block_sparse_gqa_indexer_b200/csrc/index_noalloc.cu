@@ -111,6 +111,7 @@ extern "C" s5_status s5_index_score_topk_noalloc(const s5_index_desc *index, con
   sa.ctx_lens = batch->ctx_lens;
   sa.cu_q = batch->cu_q;
   sa.batch = batch->batch;
+  sa.total_q = batch->total_q;
   sa.topk = topk;
   sa.sel = sel;
   sa.sel_count = sel_count;

@@ -46,6 +46,7 @@ template <int QT, int UNROLL>
 __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
   constexpr int LOGV = (QT == 1) ? 3 : (QT == 2) ? 4 : 5;
   constexpr int V = 1 << LOGV;  // 8 blocks x QT queries
+  pdl_trigger();  // the select may launch now; it waits for these scores before reading them
   const int s = blockIdx.y;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -140,8 +141,10 @@ __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
         const int j = v % kBpp;
         const int b = pp * kBpp + j;
         if (qi < nq && b < (ctx + tile0 + qi) / kBlk) {
-          a.scores[(size_t)(q_beg + tile0 + qi) * a.score_stride + b] =
-              (phys[u] >= 0) ? vals[0] : __int_as_float(0xff800000);  // -inf for an unreadable page
+          const size_t row = (size_t)(q_beg + tile0 + qi);
+          const float sc = (phys[u] >= 0) ? vals[0] : __int_as_float(0xff800000);  // -inf: unreadable page
+          a.scores[row * a.score_stride + b] = sc;
+          if (a.hist != nullptr) atomicAdd(a.hist + row * kHistBins + (score_key(sc) >> 20), 1u);
         }
       }
     }
@@ -187,16 +190,48 @@ __device__ __forceinline__ int block_excl_scan(int v, int *buf) {
   return (warp > 0 ? buf[warp - 1] : 0) + incl - v;
 }
 
+// Emission of a selection: keys > t_hi are taken, and of the keys in
+// [t_lo, t_hi] the first kk in list order; emit(pos, list_position, key) in
+// list order.  One scan of the packed per-thread counts (keys above in the
+// high 16 bits, keys inside in the low 16) gives both prefixes: a thread's
+// first output goes to above_before + min(inside_before, kk).
+template <int NT, int EMAX, typename Emit>
+__device__ __forceinline__ void emit_selected(const uint32_t (&key)[EMAX], int mine, int first, uint32_t t_lo,
+                                              uint32_t t_hi, int kk, int *scan_buf, Emit emit) {
+  int in = 0, gt = 0;
+#pragma unroll
+  for (int j = 0; j < EMAX; ++j) {
+    if (j < mine) {
+      gt += key[j] > t_hi;
+      in += (key[j] >= t_lo) & (key[j] <= t_hi);
+    }
+  }
+  const int before = block_excl_scan<NT>((gt << 16) | in, scan_buf);  // list length <= 65535
+  const int in_before = before & 0xFFFF;
+  int pos = (before >> 16) + min(in_before, kk);
+  int r = in_before;
+#pragma unroll
+  for (int j = 0; j < EMAX; ++j) {
+    if (j < mine) {
+      const bool inr = (key[j] >= t_lo) & (key[j] <= t_hi);
+      const bool tk = key[j] > t_hi || (inr && r < kk);
+      r += inr;
+      if (tk) emit(pos++, first + j, key[j]);
+    }
+  }
+}
+
 // Top-k of a list of n keys (n > k >= 1).  Thread t owns list positions
-// t*E .. t*E+E-1, held in shared memory as ks[j * NT + t].  Radix select on
-// 8-bit digits from the top: each pass histograms the digit of the keys that
-// still match the chosen prefix into per-warp histograms (no atomics shared
-// between warps), sums them and picks the bin holding the kk-th largest; it
-// stops early when that whole bin is taken.  Then the keys above the final
-// range and the first kk keys inside it (list order) are emitted as
-// emit(pos, list_position), pos = 0..k-1 in list order.
-template <int NT, typename Emit>
-__device__ void cta_select(const uint32_t *ks, int n, int E, int k, SelectSmem<NT> &sm, Emit emit) {
+// t*E .. t*E+E-1 (E <= EMAX, a multiple of 4) and holds their keys in
+// registers.  Radix select on 8-bit digits from the top: each pass histograms
+// the digit of the keys still matching the chosen prefix into per-warp
+// histograms (no atomics shared between warps), sums them and picks the bin
+// holding the kk-th largest; it stops early when that whole bin is taken.
+// Then the keys above the final range and the first kk keys inside it (list
+// order) are emitted as emit(pos, list_position, key), pos = 0..k-1 in list
+// order.
+template <int NT, int EMAX, typename Emit>
+__device__ void cta_select(const uint32_t (&key)[EMAX], int n, int E, int k, SelectSmem<NT> &sm, Emit emit) {
   constexpr int NW = NT / 32;
   static_assert(NT >= 256, "one thread per bin when summing histograms");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -206,12 +241,12 @@ __device__ void cta_select(const uint32_t *ks, int n, int E, int k, SelectSmem<N
   int kk = k;
   uint32_t *wh = sm.whist[warp];
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = lane; i < 256; i += 32) wh[i] = 0;
+#pragma unroll
+    for (int i = 0; i < 256 / 32; ++i) wh[lane + 32 * i] = 0;
     __syncwarp();
-    for (int j = 0; j < mine; ++j) {
-      const uint32_t key = ks[j * NT + tid];
-      if ((key & mask) == prefix) atomicAdd(&wh[(key >> shift) & 255u], 1u);
-    }
+#pragma unroll
+    for (int j = 0; j < EMAX; ++j)
+      if (j < mine && (key[j] & mask) == prefix) atomicAdd(&wh[(key[j] >> shift) & 255u], 1u);
     __syncthreads();
     // thread i < 256 owns bin 255 - i: bins in descending order
     int cnt = 0;
@@ -246,25 +281,7 @@ __device__ void cta_select(const uint32_t *ks, int n, int E, int k, SelectSmem<N
     __syncthreads();  // sm.digit / above / bin_cnt are rewritten by the next pass
     if (stop) break;
   }
-  const uint32_t t_lo = prefix, t_hi = prefix | ~mask;  // keys in [t_lo, t_hi] compete for the last kk places
-  int in = 0, gt = 0;
-  for (int j = 0; j < mine; ++j) {
-    const uint32_t key = ks[j * NT + tid];
-    gt += key > t_hi;
-    in += (key >= t_lo) & (key <= t_hi);
-  }
-  const int in_before = block_excl_scan<NT>(in, sm.scan_a);
-  const int take = gt + max(0, min(in, kk - in_before));
-  int pos = block_excl_scan<NT>(take, sm.scan_b);
-  int r = in_before;
-  for (int j = 0; j < mine; ++j) {
-    const uint32_t key = ks[j * NT + tid];
-    const bool inr = (key >= t_lo) & (key <= t_hi);
-    const bool tk = key > t_hi || (inr && r < kk);
-    r += inr;
-    if (tk) emit(pos++, first + j);
-  }
-  __syncthreads();
+  emit_selected<NT, EMAX>(key, mine, first, prefix, prefix | ~mask, kk, sm.scan_a, emit);
 }
 
 // Positions per thread for an n-long list: a multiple of 4 (whole float4 loads).
@@ -273,34 +290,30 @@ __host__ __device__ constexpr int owned_per_thread(int n) {
   return (((n + NT - 1) / NT) + 3) & ~3;
 }
 
-// Stage the n scores row[0..n) as keys in the owner layout; a thread's loads
-// are all in flight together.  row is 16-byte aligned and readable up to the
+// The keys of scores row[0..n) owned by this thread (positions t*E ..), all
+// loads in flight together.  row is 16-byte aligned and readable up to the
 // next multiple of 4.
-template <int NT>
-__device__ __forceinline__ void load_keys(const float *row, int n, int E, uint32_t *ks) {
+template <int NT, int EMAX>
+__device__ __forceinline__ void load_keys(const float *row, int n, int E, uint32_t (&key)[EMAX]) {
   const int t = threadIdx.x;
   const float4 *r4 = reinterpret_cast<const float4 *>(row + (size_t)t * E);
-  constexpr int kMaxQ = 8;  // E <= 32
-  float4 v[kMaxQ];
+  float4 v[EMAX / 4];
 #pragma unroll
-  for (int q = 0; q < kMaxQ; ++q)
-    if (4 * q < E && t * E + 4 * q < n) v[q] = __ldcg(r4 + q);
+  for (int q = 0; q < EMAX / 4; ++q)
+    if (4 * q < E && t * E + 4 * q < n) v[q] = ld_cg(r4 + q);
 #pragma unroll
-  for (int q = 0; q < kMaxQ; ++q) {
-    if (4 * q < E) {
-      const int i0 = t * E + 4 * q;
-      const float f[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) ks[(4 * q + e) * NT + t] = (i0 + e < n) ? score_key(f[e]) : 0u;
-    }
+  for (int q = 0; q < EMAX / 4; ++q) {
+    key[4 * q] = score_key(v[q].x);
+    key[4 * q + 1] = score_key(v[q].y);
+    key[4 * q + 2] = score_key(v[q].z);
+    key[4 * q + 3] = score_key(v[q].w);
   }
 }
 
 // Query row -> (history blocks c).  Returns false on bad batch data.
 __device__ __forceinline__ bool row_history(const SelectArgs &a, int r, int &c) {
-  const int s = seq_of_row(a.cu_q, a.batch, r);
-  if (s < 0) return false;
-  const int t = __ldg(a.ctx_lens + s) + (r - __ldg(a.cu_q + s));
+  int s, t;
+  if (!locate_row(a.cu_q, a.ctx_lens, a.batch, r, row_guess(r, a.batch, a.total_q), s, t)) return false;
   if (t < 0 || t / kBlk > a.score_stride) return false;
   c = t / kBlk;
   return true;
@@ -310,15 +323,17 @@ __device__ __forceinline__ void write_all(int32_t *out, int n, int topk, int nt)
   for (int i = threadIdx.x; i < topk; i += nt) out[i] = (i < n) ? i : -1;
 }
 
-// Single stage: one CTA per query row.
-template <int NT>
+// Single stage: one CTA per query row (rows of up to NT * EMAX blocks).
+template <int NT, int EMAX>
 __global__ void __launch_bounds__(NT) topk_select_kernel(SelectArgs a) {
-  extern __shared__ __align__(16) uint32_t ks[];
   __shared__ SelectSmem<NT> sm;
   const int r = blockIdx.x;
   int32_t *out = a.sel + (size_t)r * a.topk;
+  pdl_trigger();
+  pdl_wait();
   int c = 0;
-  if (!row_history(a, r, c)) {
+  const bool row_ok = row_history(a, r, c) && c <= NT * EMAX;
+  if (!row_ok) {
     if (threadIdx.x == 0) {
       record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
       a.sel_count[r] = 0;
@@ -332,20 +347,176 @@ __global__ void __launch_bounds__(NT) topk_select_kernel(SelectArgs a) {
     return;
   }
   const int E = owned_per_thread<NT>(c);
-  load_keys<NT>(a.scores + (size_t)r * a.score_stride, c, E, ks);
-  __syncthreads();
-  cta_select<NT>(ks, c, E, a.topk, sm, [&](int pos, int i) { out[pos] = i; });
+  uint32_t key[EMAX];
+  load_keys<NT, EMAX>(a.scores + (size_t)r * a.score_stride, c, E, key);
+  cta_select<NT, EMAX>(key, c, E, a.topk, sm, [&](int pos, int i, uint32_t) { out[pos] = i; });
   if (threadIdx.x == 0) a.sel_count[r] = a.topk;
+}
+
+constexpr int kWarpRefine = 2048;  // threshold bins up to this size are refined by one warp
+
+struct HistSmem {
+  uint32_t h2[1024];            // block-wide refinement of a large threshold bin
+  uint32_t cand[kWarpRefine];   // keys of the threshold bin (any order)
+  int scan_a[32];
+  int ncand;
+  uint32_t digit, above, bin_cnt;
+  uint32_t t_val;
+  int t_kk;
+};
+
+// Bin of the kk-th largest key when thread t owns the NB consecutive bins
+// counted from the top, starting at bin (top - t * NB); c[i] is the count of
+// bin top - t * NB - i.  Results in sm.digit / above / bin_cnt.
+template <int NT, int NB>
+__device__ __forceinline__ void find_bin_desc(const uint32_t (&c)[NB], int top, int kk, HistSmem &sm) {
+  int cnt = 0;
+#pragma unroll
+  for (int i = 0; i < NB; ++i) cnt += (int)c[i];
+  const int excl = block_excl_scan<NT>(cnt, sm.scan_a);
+  if (excl < kk && kk <= excl + cnt) {
+    int acc = excl;
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+      if (acc < kk && kk <= acc + (int)c[i]) {
+        sm.digit = (uint32_t)(top - (int)threadIdx.x * NB - i);
+        sm.above = (uint32_t)acc;
+        sm.bin_cnt = c[i];
+      }
+      acc += (int)c[i];
+    }
+  }
+  __syncthreads();
+}
+
+// Single stage from a row histogram of the top 12 key bits (built while the
+// scores were produced).  The histogram gives the threshold bin; its keys are
+// then resolved either by one warp (a bit-by-bit search over the remaining 20
+// bits, when the bin holds at most kWarpRefine keys and WARP_REFINE is set) or
+// by two more block-wide radix passes of 10 bits.
+template <int NT, int EMAX, bool WARP_REFINE>
+__global__ void __launch_bounds__(NT) topk_select_hist_kernel(SelectArgs a) {
+  static_assert(NT == 512 || NT == 1024, "row-histogram and refinement bins are split evenly over threads");
+  constexpr int NB1 = kHistBins / NT;  // row-histogram bins per thread
+  constexpr int NB2 = 1024 / NT;       // refinement bins per thread
+  __shared__ HistSmem sm;
+  const int r = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  int32_t *out = a.sel + (size_t)r * a.topk;
+  pdl_trigger();
+  pdl_wait();  // every input (batch data, scores, histograms) is read after this point
+  int c = 0;
+  const bool row_ok = row_history(a, r, c) && c <= NT * EMAX;
+  // this thread's row-histogram bins, top first: 4095 - NB1*t .. (loaded with the keys)
+  uint32_t cc1[NB1];
+  {
+    const uint4 *h4 = reinterpret_cast<const uint4 *>(a.hist + (size_t)r * kHistBins);
+#pragma unroll
+    for (int q = 0; q < NB1 / 4; ++q) {
+      const uint4 hv = ld_cg(h4 + (kHistBins / 4 - 1 - (NB1 / 4) * tid - q));
+      cc1[4 * q] = hv.w;
+      cc1[4 * q + 1] = hv.z;
+      cc1[4 * q + 2] = hv.y;
+      cc1[4 * q + 3] = hv.x;
+    }
+  }
+  if (!row_ok) {
+    if (tid == 0) {
+      record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
+      a.sel_count[r] = 0;
+    }
+    write_all(out, 0, a.topk, NT);
+    return;
+  }
+  if (c <= a.topk) {
+    write_all(out, c, a.topk, NT);
+    if (tid == 0) a.sel_count[r] = c;
+    return;
+  }
+  const int E = owned_per_thread<NT>(c);
+  const int first = tid * E;
+  const int mine = max(0, min(E, c - first));
+  uint32_t key[EMAX];
+  load_keys<NT, EMAX>(a.scores + (size_t)r * a.score_stride, c, E, key);
+  if (tid == 0) sm.ncand = 0;
+  find_bin_desc<NT, NB1>(cc1, kHistBins - 1, a.topk, sm);
+  int kk = a.topk - (int)sm.above;
+  const uint32_t b1 = sm.digit;
+  const int nb = (int)sm.bin_cnt;
+  uint32_t t_lo = b1 << 20, t_hi = t_lo | 0xFFFFFu;
+  if (nb != kk) {
+    if (WARP_REFINE && nb <= kWarpRefine) {
+      // gather the bin's keys, then one warp finds the kk-th largest among them
+#pragma unroll
+      for (int j = 0; j < EMAX; ++j)
+        if (j < mine && (key[j] >> 20) == b1) {
+          const int slot = atomicAdd(&sm.ncand, 1);
+          if (slot < kWarpRefine) sm.cand[slot] = key[j];
+        }
+      __syncthreads();
+      if (warp == 0) {
+        const int ncand = min(sm.ncand, kWarpRefine);
+        uint32_t T = b1 << 20;
+        int ab = 0;
+        for (int b = 19; b >= 0; --b) {
+          const uint32_t cand = T | (1u << b);
+          int ge = 0;
+          for (int i = lane; i < ncand; i += 32) {
+            const uint32_t x = sm.cand[i];
+            ge += ((x >> (b + 1)) == (T >> (b + 1))) & (x >= cand);
+          }
+          ge = __reduce_add_sync(0xffffffffu, ge);
+          if (ab + ge >= kk) T = cand;
+          else ab += ge;
+        }
+        if (lane == 0) {
+          sm.t_val = T;
+          sm.t_kk = kk - ab;
+        }
+      }
+      __syncthreads();
+      t_lo = t_hi = sm.t_val;
+      kk = sm.t_kk;
+    } else {
+      uint32_t prefix = b1 << 20, mask = 0xFFF00000u;
+      bool stop = false;
+      __syncthreads();
+      for (int shift = 10; shift >= 0 && !stop; shift -= 10) {
+#pragma unroll
+        for (int i = 0; i < NB2; ++i) sm.h2[tid + i * NT] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < EMAX; ++j)
+          if (j < mine && (key[j] & mask) == prefix) atomicAdd(&sm.h2[(key[j] >> shift) & 1023u], 1u);
+        __syncthreads();
+        uint32_t cc2[NB2];
+#pragma unroll
+        for (int i = 0; i < NB2; ++i) cc2[i] = sm.h2[1023 - NB2 * tid - i];
+        find_bin_desc<NT, NB2>(cc2, 1023, kk, sm);
+        kk -= (int)sm.above;
+        prefix |= sm.digit << shift;
+        mask |= 1023u << shift;
+        stop = ((int)sm.bin_cnt == kk);
+        __syncthreads();
+      }
+      t_lo = prefix;
+      t_hi = prefix | ~mask;
+    }
+  }
+  emit_selected<NT, EMAX>(key, mine, first, t_lo, t_hi, kk, sm.scan_a, [&](int pos, int i, uint32_t) { out[pos] = i; });
+  if (tid == 0) a.sel_count[r] = a.topk;
 }
 
 // Two stages for long histories.  Stage 1: the top-k of each segment of
 // `seg` blocks, as (key, block) candidates in block order.
-template <int NT>
+template <int NT, int EMAX>
 __global__ void __launch_bounds__(NT) topk_segment_kernel(SelectArgs a) {
-  extern __shared__ __align__(16) uint32_t ks[];
   __shared__ SelectSmem<NT> sm;
   const int r = blockIdx.y;
   const int sg = blockIdx.x;
+  pdl_trigger();
+  pdl_wait();
   int c = 0;
   if (!row_history(a, r, c)) return;  // recorded by the final stage
   if (c <= a.topk) return;
@@ -356,29 +527,30 @@ __global__ void __launch_bounds__(NT) topk_segment_kernel(SelectArgs a) {
   const float *sc = a.scores + (size_t)r * a.score_stride + b0;
   if (n <= a.topk) {
     for (int i = threadIdx.x; i < n; i += NT) {
-      a.cand_key[cbase + i] = score_key(__ldcg(sc + i));
+      a.cand_key[cbase + i] = score_key(ld_cg(sc + i));
       a.cand_idx[cbase + i] = b0 + i;
     }
     return;
   }
   const int E = owned_per_thread<NT>(n);
-  load_keys<NT>(sc, n, E, ks);
-  __syncthreads();
-  cta_select<NT>(ks, n, E, a.topk, sm, [&](int pos, int i) {
-    a.cand_key[cbase + pos] = ks[(i % E) * NT + i / E];
+  uint32_t key[EMAX];
+  load_keys<NT, EMAX>(sc, n, E, key);
+  cta_select<NT, EMAX>(key, n, E, a.topk, sm, [&](int pos, int i, uint32_t kv) {
+    a.cand_key[cbase + pos] = kv;
     a.cand_idx[cbase + pos] = b0 + i;
   });
 }
 
 // Stage 2: the top-k of the concatenated candidates of every segment.  Every
 // segment but the last holds exactly topk candidates, so candidate L of the
-// row sits at slot L % topk of segment L / topk.
-template <int NT>
+// row is entry L of the row's candidate arrays.
+template <int NT, int EMAX>
 __global__ void __launch_bounds__(NT) topk_merge_kernel(SelectArgs a) {
-  extern __shared__ __align__(16) uint32_t smem[];
   __shared__ SelectSmem<NT> sm;
   const int r = blockIdx.x;
   int32_t *out = a.sel + (size_t)r * a.topk;
+  pdl_trigger();
+  pdl_wait();
   int c = 0;
   if (!row_history(a, r, c)) {
     if (threadIdx.x == 0) {
@@ -396,29 +568,21 @@ __global__ void __launch_bounds__(NT) topk_merge_kernel(SelectArgs a) {
   const int nseg = (c + a.seg - 1) / a.seg;
   const int last = c - (nseg - 1) * a.seg;
   const int n = (nseg - 1) * a.topk + min(a.topk, last);
-  const int E = owned_per_thread<NT>(n);
-  uint32_t *ks = smem;
-  int32_t *is = reinterpret_cast<int32_t *>(smem + (size_t)E * NT);
   const size_t rbase = (size_t)r * a.n_seg * a.topk;
-  for (int j = 0; j < E; ++j) {
-    const int L = threadIdx.x * E + j;
-    if (L < n) {
-      const size_t src = rbase + (size_t)(L / a.topk) * a.topk + (L % a.topk);
-      ks[j * NT + threadIdx.x] = __ldcg(a.cand_key + src);
-      is[j * NT + threadIdx.x] = __ldcg(a.cand_idx + src);
-    }
-  }
-  __syncthreads();
   if (n <= a.topk) {  // a single segment whose candidates are all taken
-    for (int j = 0; j < E; ++j) {
-      const int L = threadIdx.x * E + j;
-      if (L < n) out[L] = is[j * NT + threadIdx.x];
-    }
-    for (int i = n + threadIdx.x; i < a.topk; i += NT) out[i] = -1;
+    for (int i = threadIdx.x; i < a.topk; i += NT) out[i] = (i < n) ? ld_cg(a.cand_idx + rbase + i) : -1;
     if (threadIdx.x == 0) a.sel_count[r] = n;
     return;
   }
-  cta_select<NT>(ks, n, E, a.topk, sm, [&](int pos, int i) { out[pos] = is[(i % E) * NT + i / E]; });
+  const int E = owned_per_thread<NT>(n);
+  uint32_t key[EMAX];
+#pragma unroll
+  for (int j = 0; j < EMAX; ++j) {
+    const int L = threadIdx.x * E + j;
+    key[j] = (j < E && L < n) ? ld_cg(a.cand_key + rbase + L) : 0u;
+  }
+  cta_select<NT, EMAX>(key, n, E, a.topk, sm,
+                       [&](int pos, int i, uint32_t) { out[pos] = ld_cg(a.cand_idx + rbase + i); });
   if (threadIdx.x == 0) a.sel_count[r] = a.topk;
 }
 
@@ -435,39 +599,37 @@ cudaError_t launch_index_score(const IndexScoreArgs &a, int max_q, int grid_page
   return cudaGetLastError();
 }
 
-constexpr int kSelThreads = 1024;  // one CTA per row (rows of up to 16,384 blocks)
-constexpr int kSegThreads = 256;   // stage 1: one CTA per segment (E = seg / 256 <= 32)
+constexpr int kSelThreads = 1024;  // one CTA per row: rows of up to 16,384 blocks
+constexpr int kSegThreads = 256;   // stage 1: one CTA per segment of up to 8,192 blocks
 
-template <int NT>
-cudaError_t launch_merge(const SelectArgs &a, int total_q, cudaStream_t st) {
-  const size_t smem = (size_t)owned_per_thread<NT>(a.n_seg * a.topk) * NT * (sizeof(uint32_t) + sizeof(int32_t));
-  cudaError_t e = cudaFuncSetAttribute(topk_merge_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  topk_merge_kernel<NT><<<total_q, NT, smem, st>>>(a);
-  return cudaGetLastError();
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous kernel of the stream drains; it calls pdl_wait() before it
+// reads any global memory.
+template <typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 cudaError_t launch_topk_select(const SelectArgs &a, int total_q, bool two_stage, cudaStream_t st) {
   if (!two_stage) {
-    constexpr int NT = kSelThreads;
-    const size_t smem = (size_t)owned_per_thread<NT>(a.score_stride) * NT * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(topk_select_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    topk_select_kernel<NT><<<total_q, NT, smem, st>>>(a);
-    return cudaGetLastError();
+    if (a.hist != nullptr)
+      return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false>, dim3(total_q), dim3(kSelThreads), st, a);
+    return launch_pdl(topk_select_kernel<kSelThreads, 16>, dim3(total_q), dim3(kSelThreads), st, a);
   }
-  constexpr int NS = kSegThreads;
-  const size_t smem1 = (size_t)owned_per_thread<NS>(a.seg) * NS * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(topk_segment_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem1);
+  cudaError_t e = launch_pdl(topk_segment_kernel<kSegThreads, 32>, dim3(a.n_seg, total_q), dim3(kSegThreads), st, a);
   if (e != cudaSuccess) return e;
-  topk_segment_kernel<NS><<<dim3(a.n_seg, total_q), NS, smem1, st>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // stage 2: at most 32 owned candidates per thread
-  if (a.n_seg * a.topk <= 32 * 512) return launch_merge<512>(a, total_q, st);
-  return launch_merge<1024>(a, total_q, st);
+  if (a.n_seg * a.topk <= 512 * 16) return launch_pdl(topk_merge_kernel<512, 16>, dim3(total_q), dim3(512), st, a);
+  return launch_pdl(topk_merge_kernel<1024, 20>, dim3(total_q), dim3(1024), st, a);
 }
 
 }  // namespace s5

@@ -26,6 +26,36 @@ constexpr size_t kWsHeader = 256;
 constexpr size_t kWsCounterBytes = 16384;
 constexpr size_t kWsFixed = kWsHeader + kWsCounterBytes;  // first byte of per-call scratch
 
+// Loads that stay after a preceding wait or fence in program order (asm
+// volatile, L2-coherent).  Used for every read of data another kernel or CTA
+// may have just written: plain __ldg loads are treated as invariant and may be
+// hoisted above griddepcontrol.wait or a fence.
+__device__ __forceinline__ int32_t ld_cg(const int32_t *p) {
+  int32_t v;
+  asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_cg(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_cg(const float *p) {
+  float v;
+  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 ld_cg(const uint4 *p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_cg(const float4 *p) {
+  float4 v;
+  asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p) : "memory");
+  return v;
+}
+
 struct ErrRec {
   int32_t code;
   int32_t info;
@@ -42,12 +72,36 @@ __device__ __forceinline__ void record_error(int32_t *err, int code, int info) {
 // non-decreasing).  Returns -1 when r is outside [cu_q[0], cu_q[batch]).
 __device__ __forceinline__ int seq_of_row(const int32_t *cu_q, int batch, int r) {
   int lo = 0, hi = batch;  // invariant: cu_q[lo] <= r < cu_q[hi]
-  if (r < __ldg(cu_q) || r >= __ldg(cu_q + batch)) return -1;
+  if (r < ld_cg(cu_q) || r >= ld_cg(cu_q + batch)) return -1;
   while (hi - lo > 1) {
     int mid = (lo + hi) >> 1;
-    if (__ldg(cu_q + mid) <= r) lo = mid; else hi = mid;
+    if (ld_cg(cu_q + mid) <= r) lo = mid; else hi = mid;
   }
   return lo;
+}
+
+// Sequence s and absolute position t of query row r.  `guess` is tried
+// first (one round trip: cu_q[g], cu_q[g+1], ctx_lens[g] are independent
+// loads); a miss falls back to the binary search.  False on bad batch data.
+__device__ __forceinline__ bool locate_row(const int32_t *cu_q, const int32_t *ctx_lens, int batch, int r,
+                                           int guess, int &s, int &t) {
+  const int g = min(max(guess, 0), batch - 1);
+  const int lo = ld_cg(cu_q + g), hi = ld_cg(cu_q + g + 1), ctx = ld_cg(ctx_lens + g);
+  if (lo <= r && r < hi) {
+    s = g;
+    t = ctx + (r - lo);
+    return true;
+  }
+  s = seq_of_row(cu_q, batch, r);
+  if (s < 0) return false;
+  t = ld_cg(ctx_lens + s) + (r - ld_cg(cu_q + s));
+  return true;
+}
+
+// Proportional guess of the sequence of row r (exact when every sequence has
+// the same number of query rows).
+__device__ __forceinline__ int row_guess(int r, int batch, int total_q) {
+  return total_q > 0 ? (int)(((long long)r * batch) / total_q) : 0;
 }
 
 // ---------------------------------------------------------------- small PTX wrappers
@@ -55,6 +109,14 @@ __device__ __forceinline__ int seq_of_row(const int32_t *cu_q, int batch, int r)
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before the previous kernel in the stream finishes;
+// pdl_wait() blocks until that kernel has completed and its writes are
+// visible (a no-op for ordinary launches).  pdl_trigger() lets the next such
+// kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

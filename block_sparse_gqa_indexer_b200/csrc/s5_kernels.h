@@ -26,8 +26,11 @@ struct IndexScoreArgs {
   int score_stride;  // >= history blocks of any row
   int pages_per_cta;
   int topk;
+  uint32_t *hist;  // [total_q][4096] counts of score keys by their top 12 bits (zeroed before), or null
   int32_t *err;
 };
+
+constexpr int kHistBins = 4096;  // row histogram of the top 12 bits of the score keys
 
 struct SelectArgs {
   const float *scores;
@@ -35,6 +38,7 @@ struct SelectArgs {
   const int32_t *ctx_lens;
   const int32_t *cu_q;
   int batch;
+  int total_q;
   int topk;
   int32_t *sel;
   int32_t *sel_count;
@@ -43,6 +47,7 @@ struct SelectArgs {
   int n_seg;  // segments per row (stride of the candidate arrays)
   uint32_t *cand_key;
   int32_t *cand_idx;
+  const uint32_t *hist;  // row histograms built by the scoring kernel, or null
   int32_t *err;
 };
 
@@ -57,6 +62,7 @@ struct AttnArgs {
   const int32_t *ctx_lens;
   const int32_t *cu_q;
   int batch;
+  int total_q;
   int max_len;
   int num_pages;
   float scale_log2;  // sm_scale * log2(e)
