@@ -238,3 +238,59 @@ def sparse_layer_step_host(key_pool, k_pool, v_pool, batch: Batch, q_host, qx_ho
         s5_sparse_gqa_attn(k_pool, v_pool, batch, q_dev, sel, sel_count, topk, sm_scale, out_dev, lse_dev, ws, st)
         out_host.copy_(out_dev, non_blocking=True)
         lse_host.copy_(lse_dev, non_blocking=True)
+
+
+class SparseLayerPipeline:
+    """Sparse-layer decode steps whose per-step inputs (q, q_index) arrive in
+    pinned host memory and whose outputs (out, lse) go back to pinned host
+    memory, with the KV cache and block keys resident on the device.
+
+    Two device buffer sets and three streams overlap the host->device copy
+    of step i+1 and the device->host copy of step i-1 with the compute of
+    step i (s5_index_score_topk + s5_sparse_gqa_attn on the compute stream).
+    """
+
+    def __init__(self, key_pool, k_pool, v_pool, batch: Batch, ws, topk: int = MAX_TOPK,
+                 sm_scale: float = DEFAULT_SM_SCALE):
+        dev = k_pool.device
+        self.key_pool, self.k_pool, self.v_pool, self.batch, self.ws = key_pool, k_pool, v_pool, batch, ws
+        self.topk, self.sm_scale = topk, sm_scale
+        tq = batch.total_q
+        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        self.q = [torch.empty((tq, N_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.qx = [torch.empty((tq, INDEX_DIM), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.sel = [torch.empty((tq, topk), dtype=torch.int32, device=dev) for _ in range(2)]
+        self.cnt = [torch.empty((tq,), dtype=torch.int32, device=dev) for _ in range(2)]
+        self.out = [torch.empty((tq, N_HEADS, HEAD_DIM), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.lse = [torch.empty((tq, N_HEADS), dtype=torch.float32, device=dev) for _ in range(2)]
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]
+        self.ev_comp = [torch.cuda.Event() for _ in range(2)]
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]
+        self.n = 0
+
+    def step(self, q_host, qx_host, out_host, lse_host):
+        b = self.n % 2
+        if self.n >= 2:  # buffer set b was last used two steps ago
+            self.s_in.wait_event(self.ev_comp[b])
+        with torch.cuda.stream(self.s_in):
+            self.q[b].copy_(q_host, non_blocking=True)
+            self.qx[b].copy_(qx_host, non_blocking=True)
+            self.ev_in[b].record(self.s_in)
+        self.s_comp.wait_event(self.ev_in[b])
+        if self.n >= 2:
+            self.s_comp.wait_event(self.ev_out[b])
+        s5_index_score_topk(self.key_pool, self.batch, self.qx[b], self.topk, self.sel[b], self.cnt[b], self.ws,
+                            self.s_comp)
+        s5_sparse_gqa_attn(self.k_pool, self.v_pool, self.batch, self.q[b], self.sel[b], self.cnt[b], self.topk,
+                           self.sm_scale, self.out[b], self.lse[b], self.ws, self.s_comp)
+        self.ev_comp[b].record(self.s_comp)
+        self.s_out.wait_event(self.ev_comp[b])
+        with torch.cuda.stream(self.s_out):
+            out_host.copy_(self.out[b], non_blocking=True)
+            lse_host.copy_(self.lse[b], non_blocking=True)
+            self.ev_out[b].record(self.s_out)
+        self.n += 1
+
+    def synchronize(self):
+        for st in (self.s_in, self.s_comp, self.s_out):
+            st.synchronize()

@@ -175,7 +175,8 @@ s5_status s5_swa_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, cons
  *   Scratch: a library-owned 8 MiB device array (file scope), which every GPU
  *   that loads the library keeps until the process exits.  Limits: at most
  *   16,384 history blocks per row (max_len <= 131,080) and
- *   256 + 4 * total_q * ((max_len - 1) / 8) bytes <= 8 MiB; larger requests
+ *   256 + 4 * total_q * S bytes <= 8 MiB, S = (max_len - 1) / 8 rounded up to a
+ *   multiple of 4; larger requests
  *   return S5_ERR_WORKSPACE with nothing enqueued.
  *   The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
  *   library routine.  The first call on a device (with that device current)
