@@ -389,6 +389,74 @@ def run_ours(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_config(args) -> None:
+    """Time one step of numbered configuration `args.config` (1..5) on this GPU and
+    print a JSON line with its own bytes / FLOPs (a measurement aid; the bench
+    line is the default mode)."""
+    from block_sparse_gqa_indexer_b200 import s5
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    layers = S.config_workloads(args.config)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / (192 ** 0.5)
+    calls, kinds, bytes_total, flops_total = [], [], 0, 0
+    for li, w in enumerate(layers):
+        swa = (args.config == 2) or (args.config == 5 and li < 3)
+        pt = w.page_table()
+        k_pool, v_pool = w.kv_pools(dev, pt, window_only=S.WINDOW if swa else None)
+        batch = s5.Batch.from_host(pt, w.ctx, w.nq, dev)
+        ws = s5.new_workspace(batch, window=S.WINDOW, device=dev)
+        q, qx = w.queries(dev)
+        out = torch.empty((w.total_q, 64, 192), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((w.total_q, 64), dtype=torch.float32, device=dev)
+        if swa:
+            calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, o=out, l=lse, ws=ws:
+                         s5.s5_swa_gqa_attn(k, v, b, q, S.WINDOW, scale, o, l, ws, stream))
+            kinds.append("swa")
+            bytes_total += R.swa_decode_bytes(w.ctx, w.nq)["total"]
+            flops_total += sum(R.attn_flops(R.swa_tokens(c + j)) for c, n in zip(w.ctx, w.nq) for j in range(n))
+        else:
+            key_pool = w.index_pool(dev, pt)
+            sel = torch.empty((w.total_q, S.TOPK), dtype=torch.int32, device=dev)
+            cnt = torch.empty((w.total_q,), dtype=torch.int32, device=dev)
+            calls.append(lambda kp=key_pool, b=batch, qx=qx, sel=sel, cnt=cnt, ws=ws:
+                         s5.s5_index_score_topk(kp, b, qx, S.TOPK, sel, cnt, ws, stream))
+            kinds.append("index")
+            calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, sel=sel, cnt=cnt, o=out, l=lse, ws=ws:
+                         s5.s5_sparse_gqa_attn(k, v, b, q, sel, cnt, S.TOPK, scale, o, l, ws, stream))
+            kinds.append("sparse")
+            bytes_total += R.sparse_decode_bytes(w.ctx, w.nq)["total"]
+            flops_total += R.sparse_flops(w.ctx, w.nq)["total"]
+    for _ in range(args.warmup):
+        for c in calls:
+            c()
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        for c in calls:
+            c()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / args.steps
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        for j, c in enumerate(calls):
+            c()
+            ev[i][j + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    per_call = [statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps))
+                for j in range(len(calls))]
+    peak, kind = _peaks()
+    line = {"config": args.config, "ms_per_step": ms, "calls_ms": dict(zip([f"{k}{i}" for i, k in enumerate(kinds)],
+                                                                           per_call)),
+            "algorithmic_bytes": bytes_total, "useful_flops": flops_total,
+            "gbs": bytes_total / (ms * 1e-3) / 1e9, "pct_hbm_peak": 100 * bytes_total / (ms * 1e-3) / 1e9 / peak,
+            "useful_tflops": flops_total / (ms * 1e-3) / 1e12, "steps": args.steps, "warmup": args.warmup}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -397,12 +465,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--batch", type=int, default=64, help="sequences per GPU (64 = the stated workload)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
+    ap.add_argument("--config", type=int, default=0, help="time numbered configuration 1..5 instead")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         args.steps = min(args.steps, 20)
         run_reference(args)
+    elif args.config:
+        run_config(args)
     else:
         run_ours(args)
 

@@ -62,9 +62,11 @@ s5_status check_kv(const s5_kv_desc *kv) {
 // ---------------------------------------------------------------- workspace layout
 
 constexpr int kMaxHistRows = 1024;  // decode / verify batches: rows get a score histogram
+constexpr int kGemmMinRows = 64;    // sequences with more query rows score on the tensor cores
+constexpr int kGemmTilesPerCta = 32;
 
 struct IndexWs {
-  size_t scores, cand_key, cand_idx, hist, hist_bytes, end;
+  size_t scores, cand_key, cand_idx, hist, hist_bytes, kxs, kxs_bytes, end;
   int stride, seg, n_seg;
   bool two_stage;
 };
@@ -83,8 +85,14 @@ IndexWs index_ws(const s5_batch_desc *b) {
   w.cand_idx = off;
   off = align_up(off + (size_t)b->total_q * w.n_seg * kMaxTopk * sizeof(int32_t), 256);
   w.hist = off;
-  w.hist_bytes = (!w.two_stage && b->total_q <= kMaxHistRows) ? (size_t)b->total_q * kHistBins * sizeof(uint32_t) : 0;
+  // the histograms are built by the CUDA-core scoring kernel (not by the tensor-core GEMM)
+  const bool gemm = b->max_q > kGemmMinRows;
+  w.hist_bytes = (!gemm && !w.two_stage && b->total_q <= kMaxHistRows)
+                     ? (size_t)b->total_q * kHistBins * sizeof(uint32_t) : 0;
   off = align_up(off + w.hist_bytes, 256);
+  w.kxs = off;
+  w.kxs_bytes = gemm ? (size_t)b->batch * w.stride * kDx * 2 : 0;
+  off = align_up(off + w.kxs_bytes, 1024);
   w.end = off;
   return w;
 }
@@ -180,6 +188,21 @@ bool make_kv_map(CUtensorMap *m, const void *pool, int num_pages) {
   cuuint32_t box[3] = {64, 3, (cuuint32_t)kBlk};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(pool), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// A bf16 matrix [rows][256] tiled as 64 x 128 boxes with the 128-byte swizzle
+// (one K block of a K-major tcgen05 operand per box).
+bool make_k256_map(CUtensorMap *m, const void *base, long long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kDx, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kDx * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -289,10 +312,36 @@ s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *b
   ia.hist = w.hist_bytes ? reinterpret_cast<uint32_t *>(wsb + w.hist) : nullptr;
   ia.err = err;
   if (ia.hist != nullptr && cudaMemsetAsync(ia.hist, 0, w.hist_bytes, cs) != cudaSuccess) return S5_ERR_CUDA;
-  const int pages = (w.stride + kBpp - 1) / kBpp;
-  const int grid_pages = (pages + kScorePagesPerCta - 1) / kScorePagesPerCta;
-  cudaError_t e = launch_index_score(ia, batch->max_q, grid_pages, batch->batch, cs);
-  if (e != cudaSuccess) return S5_ERR_CUDA;
+  if (w.kxs_bytes > 0) {
+    // prefill-sized: gather each sequence's keys, then tensor-core GEMM
+    GatherArgs ga{};
+    ga.key_pool = index->key_pool;
+    ga.num_pages = index->num_pages;
+    ga.page_table = batch->page_table;
+    ga.max_pages = batch->max_pages;
+    ga.kxs = wsb + w.kxs;
+    ga.max_blocks = w.stride;
+    if (launch_gather_keys(ga, batch->batch, cs) != cudaSuccess) return S5_ERR_CUDA;
+    CUtensorMap tq, tk;
+    if (!make_k256_map(&tq, q_index, batch->total_q) ||
+        !make_k256_map(&tk, ga.kxs, (long long)batch->batch * w.stride))
+      return S5_ERR_CUDA;
+    GemmArgs gm{};
+    gm.ctx_lens = batch->ctx_lens;
+    gm.cu_q = batch->cu_q;
+    gm.batch = batch->batch;
+    gm.total_q = batch->total_q;
+    gm.scores = ia.scores;
+    gm.score_stride = w.stride;
+    gm.max_blocks = w.stride;
+    gm.tiles_per_cta = kGemmTilesPerCta;
+    gm.err = err;
+    if (launch_index_gemm(gm, tq, tk, batch->batch, batch->max_q, cs) != cudaSuccess) return S5_ERR_CUDA;
+  } else {
+    const int pages = (w.stride + kBpp - 1) / kBpp;
+    const int grid_pages = (pages + kScorePagesPerCta - 1) / kScorePagesPerCta;
+    if (launch_index_score(ia, batch->max_q, grid_pages, batch->batch, cs) != cudaSuccess) return S5_ERR_CUDA;
+  }
 
   SelectArgs sa{};
   sa.scores = ia.scores;

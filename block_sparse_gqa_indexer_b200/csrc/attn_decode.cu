@@ -112,9 +112,12 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const int p = blockIdx.x;
-  const int g = blockIdx.y;
-  const int r = blockIdx.z;
+  // flattened grid, partition fastest, then row, then group: rows running
+  // together share one group's KV (100 MB per 128K-token sequence, L2-sized)
+  const int p = blockIdx.x % a.n_split;
+  const int rg = blockIdx.x / a.n_split;
+  const int r = rg % a.total_q;
+  const int g = rg / a.total_q;
 
   // ---- the unit's token range -------------------------------------------------
   if (tid < kWarps * kStages) mbar_init(bars + tid, 1);
@@ -502,7 +505,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
 
 cudaError_t launch_gqa_decode(int mode, const AttnArgs &a, const CUtensorMap &tk, const CUtensorMap &tv,
                               int total_q, cudaStream_t st) {
-  dim3 grid(a.n_split, kKv, total_q);
+  const long long n_cta = (long long)a.n_split * total_q * kKv;
+  if (n_cta > 0x7fffffffLL) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)n_cta);
   cudaError_t e;
   auto kernel = (mode == kModeSparse) ? gqa_decode_kernel<kModeSparse> : gqa_decode_kernel<kModeSwa>;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);

@@ -197,7 +197,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int *buf) {
 // first output goes to above_before + min(inside_before, kk).
 template <int NT, int EMAX, typename Emit>
 __device__ __forceinline__ void emit_selected(const uint32_t (&key)[EMAX], int mine, int first, uint32_t t_lo,
-                                              uint32_t t_hi, int kk, int *scan_buf, Emit emit) {
+                                              uint32_t t_hi, int kk, int k_out, int *scan_buf, Emit emit) {
   int in = 0, gt = 0;
 #pragma unroll
   for (int j = 0; j < EMAX; ++j) {
@@ -216,7 +216,8 @@ __device__ __forceinline__ void emit_selected(const uint32_t (&key)[EMAX], int m
       const bool inr = (key[j] >= t_lo) & (key[j] <= t_hi);
       const bool tk = key[j] > t_hi || (inr && r < kk);
       r += inr;
-      if (tk) emit(pos++, first + j, key[j]);
+      if (tk && pos < k_out) emit(pos, first + j, key[j]);  // never past the k outputs
+      pos += tk;
     }
   }
 }
@@ -281,7 +282,7 @@ __device__ void cta_select(const uint32_t (&key)[EMAX], int n, int E, int k, Sel
     __syncthreads();  // sm.digit / above / bin_cnt are rewritten by the next pass
     if (stop) break;
   }
-  emit_selected<NT, EMAX>(key, mine, first, prefix, prefix | ~mask, kk, sm.scan_a, emit);
+  emit_selected<NT, EMAX>(key, mine, first, prefix, prefix | ~mask, kk, k, sm.scan_a, emit);
 }
 
 // Positions per thread for an n-long list: a multiple of 4 (whole float4 loads).
@@ -370,6 +371,11 @@ struct HistSmem {
 // bin top - t * NB - i.  Results in sm.digit / above / bin_cnt.
 template <int NT, int NB>
 __device__ __forceinline__ void find_bin_desc(const uint32_t (&c)[NB], int top, int kk, HistSmem &sm) {
+  if (threadIdx.x == 0) {  // defined results even if no bin holds the kk-th key
+    sm.digit = 0;
+    sm.above = 0;
+    sm.bin_cnt = 0;
+  }
   int cnt = 0;
 #pragma unroll
   for (int i = 0; i < NB; ++i) cnt += (int)c[i];
@@ -504,7 +510,8 @@ __global__ void __launch_bounds__(NT) topk_select_hist_kernel(SelectArgs a) {
       t_hi = prefix | ~mask;
     }
   }
-  emit_selected<NT, EMAX>(key, mine, first, t_lo, t_hi, kk, sm.scan_a, [&](int pos, int i, uint32_t) { out[pos] = i; });
+  emit_selected<NT, EMAX>(key, mine, first, t_lo, t_hi, kk, a.topk, sm.scan_a,
+                          [&](int pos, int i, uint32_t) { out[pos] = i; });
   if (tid == 0) a.sel_count[r] = a.topk;
 }
 

@@ -75,7 +75,32 @@ struct AttnArgs {
   int32_t *err;
 };
 
+// Prefill-sized batches: block keys gathered per sequence, then a tcgen05 GEMM.
+struct GatherArgs {
+  const void *key_pool;
+  int num_pages;
+  const int32_t *page_table;
+  int max_pages;
+  void *kxs;       // bf16 [batch][max_blocks][256]
+  int max_blocks;  // rows per sequence in kxs
+};
+
+struct GemmArgs {
+  const int32_t *ctx_lens;
+  const int32_t *cu_q;
+  int batch;
+  int total_q;
+  float *scores;  // [total_q][score_stride]
+  int score_stride;
+  int max_blocks;     // rows per sequence of the gathered keys
+  int tiles_per_cta;  // 128-block N tiles per CTA
+  int32_t *err;
+};
+
 cudaError_t launch_index_score(const IndexScoreArgs &a, int max_q, int grid_pages, int n_seq, cudaStream_t st);
+cudaError_t launch_gather_keys(const GatherArgs &a, int batch, cudaStream_t st);
+cudaError_t launch_index_gemm(const GemmArgs &a, const CUtensorMap &tq, const CUtensorMap &tk, int batch, int max_q,
+                              cudaStream_t st);
 cudaError_t launch_topk_select(const SelectArgs &a, int total_q, bool two_stage, cudaStream_t st);
 cudaError_t launch_gqa_decode(int mode, const AttnArgs &a, const CUtensorMap &tk, const CUtensorMap &tv,
                               int total_q, cudaStream_t st);

@@ -265,3 +265,19 @@ def test_swa_many_rows_wide_window_separate_merge(lib):
     assert_attn_close(d.out.float().cpu().numpy()[rows], want, "swa W=8192, 1100 rows")
     assert np.abs(d.lse.cpu().numpy()[rows] - want_lse).max() <= LSE_ABS
     _check_no_device_error(lib, d)
+
+
+@pytest.mark.parametrize("ctx,nq", [
+    ([3000, 70000], [300, 200]),    # more than 64 rows per sequence: tensor-core scoring
+    ([100, 20000, 9], [129, 1, 70]),
+])
+def test_prefill_sized_batches_all_selections(lib, ctx, nq):
+    w = S.Workload(ctx=ctx, nq=nq, seed=22)
+    d = DeviceInputs(w, lib)
+    _run_index(lib, d)
+    _run_sparse(lib, d)
+    rows = list(range(w.total_q))
+    want_sel = _check_selection(lib, d, rows)
+    some = sample_rows(w.total_q, 8, 3)
+    _check_sparse_out(d, some, want_sel[some], f"prefill-sized ctx={ctx} nq={nq}")
+    _check_no_device_error(lib, d)
