@@ -390,13 +390,13 @@ def run_ours(args) -> None:
 
 
 def run_config(args) -> None:
-    """Time one step of numbered configuration `args.config` (1..5) on this GPU and
+    """Time one step of numbered configuration `args.config` (1..6) on this GPU and
     print a JSON line with its own bytes / FLOPs (a measurement aid; the bench
     line is the default mode)."""
     from block_sparse_gqa_indexer_b200 import s5
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    layers = S.config_workloads(args.config)
+    layers = [S.shard(w, 0, args.shard) for w in S.config_workloads(args.config)]
     stream = torch.cuda.current_stream(dev)
     scale = 1.0 / (192 ** 0.5)
     calls, kinds, bytes_total, flops_total = [], [], 0, 0
@@ -465,7 +465,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--batch", type=int, default=64, help="sequences per GPU (64 = the stated workload)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
-    ap.add_argument("--config", type=int, default=0, help="time numbered configuration 1..5 instead")
+    ap.add_argument("--config", type=int, default=0, help="time numbered configuration 1..6 instead")
+    ap.add_argument("--shard", type=int, default=1, help="with --config: run the first of this many batch shards")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

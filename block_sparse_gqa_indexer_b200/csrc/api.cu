@@ -152,6 +152,69 @@ AttnWs attn_ws(const s5_batch_desc *b, int blocks_per_row, int slots) {
   return w;
 }
 
+// ---- multi-row tiles (verify / prefill) on the tensor cores ----
+constexpr int kTileRows = 4;
+
+struct TileWs {
+  size_t count, ent, tile_on, row_skip, part_o, part_lse, end;
+  int tiles_per_seq, n_tiles, union_cap, bitmap_words, n_split;
+};
+
+// Tile CTAs hold 210 KB of shared memory: one per SM.  With `sizing`, the
+// partials are reserved for the largest partition count any device may pick.
+// The region starts at `base`: below it lie the per-row kernel's partials,
+// which that kernel writes while other CTAs still read the tile flags.
+TileWs tile_ws(const s5_batch_desc *b, int topk, int slots_1cta, bool sizing, size_t base) {
+  TileWs w{};
+  w.tiles_per_seq = (b->max_q + kTileRows - 1) / kTileRows;
+  w.n_tiles = b->batch * w.tiles_per_seq;
+  w.union_cap = kTileRows * topk + kTileRows;
+  w.bitmap_words = (b->max_len / kBlk) / 32 + 2;
+  // partitions: fewest waves per unit of work (ceil(n * units / slots) / n), n <= 8,
+  // ties to fewer partitions; merge counters cover 1,024 tiles
+  const long long units = (long long)w.n_tiles * kKv;
+  int best = 1;
+  if (w.n_tiles <= kMaxMergeRows && units > 0 && slots_1cta > 0) {
+    double best_cost = 1e30;
+    for (int n = 1; n <= 8; ++n) {
+      const double cost = (double)((n * units + slots_1cta - 1) / slots_1cta) / n;
+      if (cost < best_cost - 1e-9) {
+        best_cost = cost;
+        best = n;
+      }
+    }
+  }
+  w.n_split = best;
+  size_t off = align_up(base, 256);
+  w.count = off;
+  off = align_up(off + (size_t)w.n_tiles * sizeof(int), 256);
+  w.tile_on = off;
+  off = align_up(off + (size_t)w.n_tiles * sizeof(int32_t), 256);
+  w.row_skip = off;
+  off = align_up(off + (size_t)b->total_q * sizeof(int32_t), 256);
+  w.ent = off;
+  off = align_up(off + (size_t)w.n_tiles * w.union_cap * sizeof(uint32_t), 256);
+  w.part_o = w.part_lse = off;
+  const int n_res = (sizing && w.n_tiles <= kMaxMergeRows) ? 8 : w.n_split;
+  if (n_res > 1) {
+    off = align_up(off + (size_t)b->total_q * kHeads * n_res * kD * sizeof(float), 256);
+    w.part_lse = off;
+    off = align_up(off + (size_t)b->total_q * kHeads * n_res * sizeof(float), 256);
+  }
+  w.end = off;
+  return w;
+}
+
+// Multi-token batches go through the union kernel, which sends each 4-row
+// tile to the shared-set tile kernel or to the per-row kernel.
+bool use_tiles(const s5_batch_desc *b) { return b->max_q >= 2; }
+
+// Crossover of the two paths, measured on B200: a shared-set chunk of 8 union
+// blocks (4 rows x 16 heads on the tensor cores) costs about as much as 5.6
+// per-row blocks, so a tile takes the shared set when its union has at most
+// 70 % as many blocks as its rows read one by one.
+constexpr int kTileUnionPct = 70;
+
 int sparse_blocks_per_row(int topk) { return topk + 1; }
 int swa_blocks_per_row(const s5_batch_desc *b, int window) {
   long long w = window < b->max_len ? window : b->max_len;
@@ -193,6 +256,40 @@ bool make_kv_map(CUtensorMap *m, const void *pool, int num_pages) {
   return r == CUDA_SUCCESS;
 }
 
+// A bf16 matrix [rows][192] tiled as 64-wide boxes of `box_rows` rows with the
+// 128-byte swizzle (one 64-dim plane of a K/V block or of 16 query heads).
+bool make_d192_map(CUtensorMap *m, const void *base, long long rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// A K or V pool as rows of 192 dims, each 8-row box landing plane-major: box
+// {64 dims, 8 rows, 3 planes} with the planes (128 B apart in memory) as the
+// outermost box dimension, so one copy places a whole 8-token block as three
+// 1,024-byte swizzled planes [plane][token][64 dims].  The plane stride is
+// smaller than the row stride; the box addresses stay inside the pool either
+// way (every coordinate is range-checked against its own extent).
+bool make_kv_plane_map(CUtensorMap *m, const void *pool, int num_pages) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)num_pages * kKv * kPage, 3};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)kBlk, 3};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(pool), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // A bf16 matrix [rows][256] tiled as 64 x 128 boxes with the 128-byte swizzle
 // (one K block of a K-major tcgen05 operand per box).
 bool make_k256_map(CUtensorMap *m, const void *base, long long rows) {
@@ -223,6 +320,7 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   if (b->total_q == 0) return S5_OK;
   if (q == nullptr || out == nullptr || !aligned16(q) || !aligned16(out)) return S5_ERR_INVALID_ARG;
   if (mode == kModeSparse && (sel == nullptr || sel_count == nullptr)) return S5_ERR_INVALID_ARG;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
   const int bpr = (mode == kModeSparse) ? sparse_blocks_per_row(topk) : swa_blocks_per_row(b, window);
   const AttnWs w = attn_ws(b, bpr, device_slots());
   if (ws_bytes < w.end) return S5_ERR_WORKSPACE;
@@ -230,7 +328,6 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   if (!make_kv_map(&tk, kv->k_pool, kv->num_pages) || !make_kv_map(&tv, kv->v_pool, kv->num_pages))
     return S5_ERR_CUDA;
   AttnArgs a{};
-  uint8_t *wsb = static_cast<uint8_t *>(ws);
   a.q = q;
   a.sel = sel;
   a.sel_count = sel_count;
@@ -251,7 +348,51 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   a.part_o = reinterpret_cast<float *>(wsb + w.part_o);
   a.part_lse = reinterpret_cast<float *>(wsb + w.part_lse);
   a.merge_cnt = (b->total_q <= kMaxMergeRows) ? reinterpret_cast<uint32_t *>(wsb + kWsHeader) : nullptr;
+  a.row_skip = nullptr;
   a.err = reinterpret_cast<int32_t *>(ws);
+
+  if (mode == kModeSparse && use_tiles(b)) {
+    // union lists and per-tile choice, then the shared-set tiles; the per-row
+    // kernel below skips the rows those tiles computed
+    const TileWs tw = tile_ws(b, topk, device_slots() / kCtasPerSm, false, w.end);
+    if (ws_bytes < tw.end) return S5_ERR_WORKSPACE;
+    CUtensorMap tq, tpk, tpv;
+    if (!make_d192_map(&tq, q, (long long)b->total_q * kHeads, kHpg) ||
+        !make_kv_plane_map(&tpk, kv->k_pool, kv->num_pages) || !make_kv_plane_map(&tpv, kv->v_pool, kv->num_pages))
+      return S5_ERR_CUDA;
+    TileArgs t{};
+    t.q = q;
+    t.sel = sel;
+    t.sel_count = sel_count;
+    t.topk = topk;
+    t.page_table = b->page_table;
+    t.max_pages = b->max_pages;
+    t.ctx_lens = b->ctx_lens;
+    t.cu_q = b->cu_q;
+    t.batch = b->batch;
+    t.total_q = b->total_q;
+    t.num_pages = kv->num_pages;
+    t.scale_log2 = a.scale_log2;
+    t.tiles_per_seq = tw.tiles_per_seq;
+    t.n_tiles = tw.n_tiles;
+    t.n_split = tw.n_split;
+    t.bitmap_words = tw.bitmap_words;
+    t.union_cap = tw.union_cap;
+    t.union_count = reinterpret_cast<int *>(wsb + tw.count);
+    t.union_ent = reinterpret_cast<uint32_t *>(wsb + tw.ent);
+    t.out = out;
+    t.lse = lse;
+    t.part_o = reinterpret_cast<float *>(wsb + tw.part_o);
+    t.part_lse = reinterpret_cast<float *>(wsb + tw.part_lse);
+    t.merge_cnt = reinterpret_cast<uint32_t *>(wsb + kWsHeader);
+    t.union_pct = kTileUnionPct;
+    t.tile_on = reinterpret_cast<int32_t *>(wsb + tw.tile_on);
+    t.row_skip = reinterpret_cast<int32_t *>(wsb + tw.row_skip);
+    t.err = a.err;
+    if (launch_tile_union(t, b->batch, stream) != cudaSuccess) return S5_ERR_CUDA;
+    if (launch_gqa_tile(t, tq, tpk, tpv, stream) != cudaSuccess) return S5_ERR_CUDA;
+    a.row_skip = t.row_skip;
+  }
   return cuda_status(launch_gqa_decode(mode, a, tk, tv, b->total_q, stream));
 }
 
@@ -266,7 +407,8 @@ s5_status s5_workspace_size(const s5_batch_desc *batch, int32_t window, size_t *
   if (window < 0) return S5_ERR_INVALID_ARG;
   size_t need = index_ws(batch).end;
   const int slots = kCtasPerSm * kSizingSms;  // an upper bound: no device query here
-  const size_t sp = attn_ws(batch, sparse_blocks_per_row(kMaxTopk), slots).end;
+  size_t sp = attn_ws(batch, sparse_blocks_per_row(kMaxTopk), slots).end;
+  if (use_tiles(batch)) sp = tile_ws(batch, kMaxTopk, kSizingSms, true, sp).end;
   if (sp > need) need = sp;
   if (window > 0) {
     const size_t sw = attn_ws(batch, swa_blocks_per_row(batch, window), slots).end;

@@ -80,6 +80,7 @@ __device__ __forceinline__ void store_bf16x4(__nv_bfloat16 *dst, float4 v) {
 // one CTA per (row, head), one float4 of dims per thread.
 __global__ void __launch_bounds__(kD / 4) s5_combine_kernel(const AttnArgs a) {
   const size_t rh = blockIdx.x;
+  if (a.row_skip != nullptr && ld_cg(a.row_skip + rh / kHeads) != 0) return;  // row computed by the tile kernel
   const int n = a.n_split;
   float w[kMaxSplitMerge];
   float lse;
@@ -125,6 +126,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   // programmatic launch: everything above touches shared memory only; every
   // global input (batch data, q, the selection) is read after this wait
   pdl_wait();
+  if (a.row_skip != nullptr && ld_cg(a.row_skip + r) != 0) return;  // row computed by the tile kernel
   int s = -1, t = -1, lo_tok = 0, n_list = 0, b_first = 0, n_sel = 0;
   const int sel_cnt = (MODE == kModeSparse) ? ld_cg(a.sel_count + r) : 0;
   bool bad = !locate_row(a.cu_q, a.ctx_lens, a.batch, r, row_guess(r, a.batch, a.total_q), s, t);

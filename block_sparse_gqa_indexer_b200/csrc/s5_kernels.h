@@ -72,6 +72,7 @@ struct AttnArgs {
   float *part_o;    // [total_q * 64][n_split][192]
   float *part_lse;  // [total_q * 64][n_split]   (base-2)
   uint32_t *merge_cnt;  // [total_q * 4] arrival counters (zero between calls), or null: separate merge kernel
+  const int32_t *row_skip;  // [total_q]: nonzero for rows the shared-set tile kernel computes, or null
   int32_t *err;
 };
 
@@ -96,6 +97,45 @@ struct GemmArgs {
   int tiles_per_cta;  // 128-block N tiles per CTA
   int32_t *err;
 };
+
+// Multi-row tiles (verify / prefill): shared-set attention on the tensor cores.
+constexpr int kMaxTileEntries = 2056;  // blocks one tile CTA may own (>= 4 x 512 + 4, multiple of 8)
+constexpr int kMaxTileSplit = 32;
+
+struct TileArgs {
+  const void *q;
+  const int32_t *sel;
+  const int32_t *sel_count;
+  int topk;
+  const int32_t *page_table;
+  int max_pages;
+  const int32_t *ctx_lens;
+  const int32_t *cu_q;
+  int batch;
+  int total_q;
+  int num_pages;
+  float scale_log2;
+  int tiles_per_seq;   // ceil(max_q / 4)
+  int n_tiles;         // batch * tiles_per_seq
+  int n_split;         // partitions of a tile's block list
+  int bitmap_words;    // 32-bit words per row bitmap in the union kernel
+  int union_cap;       // entries per tile in the union lists
+  int *union_count;    // [n_tiles]
+  uint32_t *union_ent; // [n_tiles][union_cap]
+  void *out;
+  float *lse;
+  float *part_o;
+  float *part_lse;
+  uint32_t *merge_cnt;
+  int union_pct;       // a tile takes the shared-set path when 100 * |union| <= union_pct * sum of rows' blocks
+  int32_t *tile_on;    // [n_tiles] written by the union kernel: 1 = shared-set path
+  int32_t *row_skip;   // [total_q] written by the union kernel: 1 = row computed by the tile kernel
+  int32_t *err;
+};
+
+cudaError_t launch_tile_union(const TileArgs &a, int batch, cudaStream_t st);
+cudaError_t launch_gqa_tile(const TileArgs &a, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                            cudaStream_t st);
 
 cudaError_t launch_index_score(const IndexScoreArgs &a, int max_q, int grid_pages, int n_seq, cudaStream_t st);
 cudaError_t launch_gather_keys(const GatherArgs &a, int batch, cudaStream_t st);

@@ -57,7 +57,7 @@ MAX_TOKENS = 1 << 21
 MAX_BLOCKS = MAX_TOKENS // BLOCK
 
 # tensor ids (one stream per tensor kind, per layer: id + 16 * layer)
-TID_Q, TID_QX, TID_K, TID_V, TID_KX, TID_LEN, TID_PERM = 1, 2, 3, 4, 5, 6, 7
+TID_Q, TID_QX, TID_K, TID_V, TID_KX, TID_LEN, TID_PERM, TID_QXN = 1, 2, 3, 4, 5, 6, 7, 8
 
 _M32 = 0xFFFFFFFF
 _M64 = (1 << 64) - 1
@@ -154,9 +154,15 @@ class Workload:
     perm_pages: bool = True  # shuffle physical pages
     seq_base: int = 0  # global id of sequence 0 (a shard of a larger batch)
     row_base: int = 0  # global id of query row 0
+    # 0: independent indexer queries per token.  W > 0: "block-coherent"
+    # indexer queries: the tokens of each W-token window of a sequence share
+    # one base query, and each token adds +-1 to about 1/16 of its
+    # dimensions, so neighbouring tokens select mostly the same blocks.
+    qx_coherent: int = 0
 
     def __post_init__(self):
         assert len(self.ctx) == len(self.nq)
+        assert self.qx_coherent <= 0 or self.index_int, "block-coherent indexer queries are integer-valued"
         for c, n in zip(self.ctx, self.nq):
             assert c >= 0 and n >= 0 and c + n <= MAX_TOKENS
 
@@ -235,13 +241,31 @@ class Workload:
             + torch.arange(HEAD_DIM, device=device).view(1, 1, -1)
         return normal_bf16(self.seed, self.tid(TID_Q), idx)
 
+    def row_seq_pos(self, rows: torch.Tensor):
+        """(sequence, absolute position) of local query rows ``rows`` (int64 tensors)."""
+        dev = rows.device
+        cu = torch.tensor(self.cu_q, dtype=torch.int64, device=dev)
+        seq = torch.searchsorted(cu[1:], rows, right=True)
+        ctx = torch.tensor(self.ctx, dtype=torch.int64, device=dev)
+        return seq, ctx[seq] + rows - cu[seq]
+
     def qx_rows(self, rows: torch.Tensor, device="cpu") -> torch.Tensor:
         """Indexer queries, bf16 [len(rows)][256] (one per query token, shared by all heads)."""
-        rows = rows.to(device=device, dtype=torch.int64) + self.row_base
-        idx = rows.view(-1, 1) * INDEX_DIM + torch.arange(INDEX_DIM, device=device).view(1, -1)
-        if self.index_int:
-            return small_int_bf16(self.seed, self.tid(TID_QX), idx)
-        return normal_bf16(self.seed, self.tid(TID_QX), idx)
+        rows = rows.to(device=device, dtype=torch.int64)
+        dims = torch.arange(INDEX_DIM, device=device).view(1, -1)
+        grows = rows + self.row_base
+        idx = grows.view(-1, 1) * INDEX_DIM + dims
+        if self.qx_coherent <= 0:
+            if self.index_int:
+                return small_int_bf16(self.seed, self.tid(TID_QX), idx)
+            return normal_bf16(self.seed, self.tid(TID_QX), idx)
+        seq, pos = self.row_seq_pos(rows)
+        windows = MAX_TOKENS // self.qx_coherent + 1
+        bidx = ((seq + self.seq_base) * windows + pos // self.qx_coherent).view(-1, 1) * INDEX_DIM + dims
+        base = uniform_int(self.seed, self.tid(TID_QX), bidx, -4, 4)
+        u = uniform_int(self.seed, self.tid(TID_QXN), idx, 0, 31)
+        noise = (u == 0).to(torch.int64) - (u == 1).to(torch.int64)
+        return (base + noise).to(torch.bfloat16)
 
     def kx_blocks(self, s: int, blocks: torch.Tensor, device="cpu") -> torch.Tensor:
         """Block keys of sequence s, bf16 [len(blocks)][256]."""
@@ -384,7 +408,10 @@ def config_workloads(which: int, seed: Optional[int] = None) -> list:
     3  sparse multi-token verify, B=64, lengths U[32K, 128K], 4 queries each;
     4  sparse chunked prefill, 16,384 queries appended at offset 114,688;
     5  hybrid group (3 sliding-window layers + 1 sparse layer), B=4, 1,048,576 cached tokens.
-    0  the headline: sparse decode, B=64, 131,072 cached tokens each, one query.
+    0  the headline: sparse decode, B=64, 131,072 cached tokens each, one query;
+    6  config 4 with block-coherent indexer queries (64-token windows share a
+       base query), a labelled secondary input on which neighbouring queries'
+       selections overlap as the shared-set prefill design expects.
     """
     sd = (0x5E5 + which) if seed is None else seed
     if which == 0:
@@ -399,6 +426,8 @@ def config_workloads(which: int, seed: Optional[int] = None) -> list:
         return [Workload(ctx=[114688], nq=[16384], seed=sd)]
     if which == 5:
         return [Workload(ctx=[1048576] * 4, nq=[1] * 4, seed=sd, layer=l) for l in range(4)]
+    if which == 6:
+        return [Workload(ctx=[114688], nq=[16384], seed=sd, qx_coherent=64)]
     raise ValueError(which)
 
 

@@ -281,3 +281,88 @@ def test_prefill_sized_batches_all_selections(lib, ctx, nq):
     some = sample_rows(w.total_q, 8, 3)
     _check_sparse_out(d, some, want_sel[some], f"prefill-sized ctx={ctx} nq={nq}")
     _check_no_device_error(lib, d)
+
+
+def test_tile_late_max_rescale(lib):
+    # verify rows (4 per sequence, block-coherent indexer queries so the tiles
+    # take the shared-set tensor-core path): the keys of the last
+    # block read (the current block, highest index) are made to align strongly
+    # with head 0 of every group, so that row maximum jumps late and the
+    # accumulated output must be rescaled
+    w = S.Workload(ctx=[9000, 20000], nq=[4, 4], seed=23, qx_coherent=64)
+    d = DeviceInputs(w, lib)
+    seqs, pos = w.query_seq_pos()
+    q_cpu = d.q.float().cpu()
+    k_cpu = {}
+    for r in range(w.total_q):
+        s, t = seqs[r], pos[r]
+        for tok in range((t // 8) * 8, t + 1):
+            page = int(d.pt[s, tok // 64])
+            for g in range(4):
+                vec = (6.0 * q_cpu[r, 16 * g]).to(torch.bfloat16)
+                d.k_pool[page, g, tok % 64] = vec.to(d.k_pool.device)
+                k_cpu[(s, tok, g)] = vec.double().numpy()
+    _run_index(lib, d)
+    _run_sparse(lib, d)
+    torch.cuda.synchronize()
+    sel = d.sel.cpu().numpy()
+    got = d.out.float().cpu().numpy()
+    for r in range(w.total_q):
+        s, t = seqs[r], pos[r]
+        T = O.sparse_token_set(sel[r], t)
+        K = w.k_tokens(s, torch.as_tensor(T)).double().numpy()
+        for i, tok in enumerate(T.tolist()):
+            for g in range(4):
+                if (s, tok, g) in k_cpu:
+                    K[i, g] = k_cpu[(s, tok, g)]
+        V = w.v_tokens(s, torch.as_tensor(T)).double().numpy()
+        want, _ = O.gqa_attention(q_cpu[r].double().numpy(), K, V, O.DEFAULT_SM_SCALE)
+        assert_attn_close(got[r], O.round_bf16(want), f"row {r}")
+    _check_no_device_error(lib, d)
+
+
+def _tiles_by_path(w, sel):
+    """(shared-set tiles, per-row tiles) of a batch under the library's
+    crossover rule: a 4-row tile takes the shared set when its union of blocks
+    (selected + current) is at most 70 % of the blocks its rows read one by one."""
+    seqs, pos = w.query_seq_pos()
+    shared = per_row = 0
+    r = 0
+    for s in range(w.batch):
+        for k in range(0, w.nq[s], 4):
+            rows = range(r + k, r + min(k + 4, w.nq[s]))
+            union, total = set(), 0
+            for i in rows:
+                blocks = set(int(b) for b in sel[i] if b >= 0) | {pos[i] // 8}
+                union |= blocks
+                total += len(blocks)
+            if 100 * len(union) <= 70 * total:
+                shared += 1
+            else:
+                per_row += 1
+        r += w.nq[s]
+    return shared, per_row
+
+
+@pytest.mark.parametrize("ctx,nq,coherent", [
+    ([20000, 3000, 70000], [300, 77, 45], 64),  # block-coherent queries: mostly shared-set tiles
+    ([9000, 4000, 30000], [40, 9, 23], 0),      # independent queries: per-row tiles past 512 blocks
+])
+def test_prefill_both_paths(lib, ctx, nq, coherent):
+    w = S.Workload(ctx=ctx, nq=nq, seed=24, qx_coherent=coherent)
+    d = DeviceInputs(w, lib)
+    lib.s5_reset_device_error(d.ws)
+    _run_index(lib, d)
+    _run_sparse(lib, d)
+    rows = list(range(w.total_q))
+    want_sel = _check_selection(lib, d, rows)
+    shared, per_row = _tiles_by_path(w, want_sel)
+    assert shared > 0 and per_row > 0, (shared, per_row)
+    some = sample_rows(w.total_q, 16, 4)
+    _check_sparse_out(d, some, want_sel[some], f"prefill ctx={ctx} nq={nq} coherent={coherent}")
+    _check_no_device_error(lib, d)
+
+
+@pytest.mark.slow
+def test_config6_block_coherent_prefill_16k(lib):
+    _config_sparse(lib, 6, 6)
