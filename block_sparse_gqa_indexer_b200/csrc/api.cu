@@ -153,14 +153,13 @@ AttnWs attn_ws(const s5_batch_desc *b, int blocks_per_row, int slots) {
 }
 
 // ---- multi-row tiles (verify / prefill) on the tensor cores ----
-constexpr int kTileRows = 4;
 
 struct TileWs {
   size_t count, ent, tile_on, row_skip, part_o, part_lse, end;
-  int tiles_per_seq, n_tiles, union_cap, bitmap_words, n_split;
+  int tiles_per_seq, n_tiles, union_cap, map_words, n_split;
 };
 
-// Tile CTAs hold 210 KB of shared memory: one per SM.  With `sizing`, the
+// Tile CTAs hold 213 KB of shared memory: one per SM.  With `sizing`, the
 // partials are reserved for the largest partition count any device may pick.
 // The region starts at `base`: below it lie the per-row kernel's partials,
 // which that kernel writes while other CTAs still read the tile flags.
@@ -169,9 +168,11 @@ TileWs tile_ws(const s5_batch_desc *b, int topk, int slots_1cta, bool sizing, si
   w.tiles_per_seq = (b->max_q + kTileRows - 1) / kTileRows;
   w.n_tiles = b->batch * w.tiles_per_seq;
   w.union_cap = kTileRows * topk + kTileRows;
-  w.bitmap_words = (b->max_len / kBlk) / 32 + 2;
-  // partitions: fewest waves per unit of work (ceil(n * units / slots) / n), n <= 8,
-  // ties to fewer partitions; merge counters cover 1,024 tiles
+  const long long words = (long long)(b->max_len / kBlk) / 4 + 2;
+  w.map_words = (int)(words < kUnionMapWords ? words : kUnionMapWords);
+  // partitions: fewest waves of the persistent CTAs per unit of work
+  // (ceil(n * units / slots) / n), n <= 8, ties to fewer partitions; merge
+  // counters cover 1,024 tiles
   const long long units = (long long)w.n_tiles * kKv;
   int best = 1;
   if (w.n_tiles <= kMaxMergeRows && units > 0 && slots_1cta > 0) {
@@ -205,14 +206,12 @@ TileWs tile_ws(const s5_batch_desc *b, int topk, int slots_1cta, bool sizing, si
   return w;
 }
 
-// Multi-token batches go through the union kernel, which sends each 4-row
+// Multi-token batches go through the union kernel, which sends each 8-row
 // tile to the shared-set tile kernel or to the per-row kernel.
 bool use_tiles(const s5_batch_desc *b) { return b->max_q >= 2; }
 
-// Crossover of the two paths, measured on B200: a shared-set chunk of 8 union
-// blocks (4 rows x 16 heads on the tensor cores) costs about as much as 5.6
-// per-row blocks, so a tile takes the shared set when its union has at most
-// 70 % as many blocks as its rows read one by one.
+// Crossover of the two paths: a tile takes the shared set when its union has
+// at most this percentage of the blocks its rows read one by one.
 constexpr int kTileUnionPct = 70;
 
 int sparse_blocks_per_row(int topk) { return topk + 1; }
@@ -251,21 +250,6 @@ bool make_kv_map(CUtensorMap *m, const void *pool, int num_pages) {
   cuuint32_t box[3] = {64, 3, (cuuint32_t)kBlk};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(pool), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-// A bf16 matrix [rows][192] tiled as 64-wide boxes of `box_rows` rows with the
-// 128-byte swizzle (one 64-dim plane of a K/V block or of 16 query heads).
-bool make_d192_map(CUtensorMap *m, const void *base, long long rows, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -356,9 +340,8 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
     // kernel below skips the rows those tiles computed
     const TileWs tw = tile_ws(b, topk, device_slots() / kCtasPerSm, false, w.end);
     if (ws_bytes < tw.end) return S5_ERR_WORKSPACE;
-    CUtensorMap tq, tpk, tpv;
-    if (!make_d192_map(&tq, q, (long long)b->total_q * kHeads, kHpg) ||
-        !make_kv_plane_map(&tpk, kv->k_pool, kv->num_pages) || !make_kv_plane_map(&tpv, kv->v_pool, kv->num_pages))
+    CUtensorMap tpk, tpv;
+    if (!make_kv_plane_map(&tpk, kv->k_pool, kv->num_pages) || !make_kv_plane_map(&tpv, kv->v_pool, kv->num_pages))
       return S5_ERR_CUDA;
     TileArgs t{};
     t.q = q;
@@ -376,7 +359,7 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
     t.tiles_per_seq = tw.tiles_per_seq;
     t.n_tiles = tw.n_tiles;
     t.n_split = tw.n_split;
-    t.bitmap_words = tw.bitmap_words;
+    t.map_words = tw.map_words;
     t.union_cap = tw.union_cap;
     t.union_count = reinterpret_cast<int *>(wsb + tw.count);
     t.union_ent = reinterpret_cast<uint32_t *>(wsb + tw.ent);
@@ -390,7 +373,7 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
     t.row_skip = reinterpret_cast<int32_t *>(wsb + tw.row_skip);
     t.err = a.err;
     if (launch_tile_union(t, b->batch, stream) != cudaSuccess) return S5_ERR_CUDA;
-    if (launch_gqa_tile(t, tq, tpk, tpv, stream) != cudaSuccess) return S5_ERR_CUDA;
+    if (launch_gqa_tile(t, tpk, tpv, device_slots() / kCtasPerSm, stream) != cudaSuccess) return S5_ERR_CUDA;
     a.row_skip = t.row_skip;
   }
   return cuda_status(launch_gqa_decode(mode, a, tk, tv, b->total_q, stream));

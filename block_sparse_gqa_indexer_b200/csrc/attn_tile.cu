@@ -1,28 +1,36 @@
-// Sparse attention for multi-token verify and chunked prefill on the
+// Sparse attention for chunked prefill and multi-token verify on the
 // 5th-generation tensor cores, over the shared set of selected blocks.
 //
 // SGLang day-0 blog ("Step 5 Preview: Day-0 Inference and RL Support with
 // SGLang and Miles"), "Kernels from StepFun": sparse prefill gathers the blocks
 // selected for a batch of queries into one shared set and runs attention over
-// that set with per-query masks.  Here the batch is a tile of up to 4
-// consecutive query rows of one sequence (the 4 tokens of a verify step, or 4
-// neighbouring prefill tokens):
+// that set with per-query masks.  Here the batch is a tile of up to 8
+// consecutive query rows of one sequence:
 //
 //   tile_union_kernel   builds, per tile, the ascending list of distinct blocks
-//                       the tile's rows read (selected history blocks and the
-//                       rows' current blocks), each entry carrying which rows
-//                       read all 8 of its tokens and which read it causally;
-//   gqa_tile_kernel     one CTA per (tile, KV group, partition of that list):
-//                       the 4 rows x 16 heads of the group are the M = 64 rows
-//                       of tcgen05 MMAs.  Warp 4 streams 8-block chunks of K
-//                       and V by TMA; warp 5 issues S = Q K^T (M=64, N=64,
-//                       K=192) into two tensor-memory buffers and
-//                       O += P V (M=64, N=192, K=64) into a tensor-memory
-//                       accumulator; warps 0-3 (warp w = row w of the tile)
-//                       mask, run the online softmax with lazy rescaling of O,
-//                       and write P as the bf16 A operand of the next MMA.
+//                       its rows read (selected history blocks and the rows'
+//                       current blocks), each entry carrying which rows
+//                       selected it, and decides per tile whether the shared
+//                       set pays (its union is small next to the blocks the
+//                       rows read one by one) or the rows go to the per-row
+//                       kernel;
+//   gqa_tile_kernel     a persistent kernel, one CTA per SM, walking work items
+//                       (tile, KV group, partition of the tile's list).  The
+//                       8 rows x 16 heads of a group are the M = 128 rows of
+//                       the MMAs.  Warp 8 streams 8-block chunks of K and warp
+//                       9 of V by TMA (one 3 KB copy per block, plane-major,
+//                       128-byte swizzled) through 4-stage rings; warp 10
+//                       issues S = Q K^T (N = 64 tokens, K = 192) into two
+//                       tensor-memory buffers and warp 11 O += P V, both with
+//                       their A operand (Q, P) in tensor memory (two issuing
+//                       threads, so S of a later chunk never waits behind the
+//                       PV of an earlier one); warps 0-7 load Q into
+//                       tensor memory, run the masked online softmax (two
+//                       warps per 32 rows, one per half of the chunk's
+//                       columns), write P back to tensor memory as bf16 and
+//                       finish each item.
 //
-// Each shared block is read once for the tile instead of once per row; the
+// Each shared block is read once per tile instead of once per row; the
 // masked-out products are the price of dense tiles.
 #include <cuda.h>
 
@@ -32,29 +40,55 @@
 
 namespace s5 {
 
-constexpr int kTRows = 4;                 // query rows per tile
-constexpr int kTM = kTRows * kHpg;        // 64 MMA rows
-constexpr int kTChunkBlocks = 8;          // blocks per chunk
-constexpr int kTN = kTChunkBlocks * kBlk; // 64 tokens per chunk
-constexpr int kTStages = 3;
-constexpr int kTQBytes = 3 * kTM * 128;                       // [3 K-blocks][64 rows][128 B]
-constexpr int kTKvBytes = kTChunkBlocks * kBlockBytes;        // K (or V) of one chunk
-constexpr int kTStageBytes = 2 * kTKvBytes;                   // K then V
-constexpr int kTPBytes = kTM * 128;                           // P: [64 rows][64 tokens] bf16
-constexpr int kTPBufs = 3;                                    // P buffers (chunk c uses c % 3)
-constexpr int kTThreads = 192;
-constexpr uint32_t kTTmemCols = 512;                          // S0 [0,64), S1 [64,128), O [128,320)
+constexpr int kTRows = kTileRows;          // query rows per tile
+constexpr int kTM = kTRows * kHpg;         // 128 MMA rows = tensor-memory lanes
+constexpr int kTChunkBlocks = 8;           // blocks per chunk
+constexpr int kTN = kTChunkBlocks * kBlk;  // 64 tokens per chunk
+constexpr int kTStages = 4;                // depth of the K ring and of the V ring
+constexpr int kTKvBytes = kTChunkBlocks * kBlockBytes;  // K (or V) of one chunk
+constexpr int kTSoftWarps = 8;
+constexpr int kTSoftThreads = kTSoftWarps * 32;
+constexpr int kTWarpK = 8, kTWarpV = 9, kTWarpS = 10, kTWarpPv = 11;
+constexpr int kTThreads = 12 * 32;
+constexpr uint32_t kTTmemCols = 512;
+constexpr uint32_t kTmemS = 0;    // 2 x 64 columns: S of chunk gc in buffer gc % 2
+constexpr uint32_t kTmemP = 128;  // 2 x 32 columns: bf16 P of chunk gc in buffer gc % 2
+constexpr uint32_t kTmemO = 192;  // 192 columns: O
+constexpr uint32_t kTmemQ = 384;  // 96 columns: Q (two bf16 dims per column)
 constexpr uint64_t kTWaitNs = 2000000000ull;
-constexpr float kLazyRescale = 8.0f;                          // log2 units
+constexpr float kLazyRescale = 8.0f;  // log2 units
+
+// shared memory (offsets from a 1,024-byte aligned base)
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kTStages * kTKvBytes;
+constexpr int kOffXm = kOffV + kTStages * kTKvBytes;  // float [2 buffers][2 halves][128 rows]
+constexpr int kOffXl = kOffXm + 2 * 2 * kTM * 4;      // float [2 halves][128 rows]
+constexpr int kOffBar = kOffXl + 2 * kTM * 4;
+constexpr int kNumBars = 44;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kOffList = kOffMisc + 64;            // int [kMaxListTiles]: shared-set tiles, ascending
+constexpr int kMaxListTiles = 4096;
+constexpr int kTileSmem = kOffList + kMaxListTiles * 4 + 1024;  // + alignment slack
+
+// barriers
+constexpr int kBQFull = 0, kBQEmpty = 1;
+constexpr int kBKFull = 2, kBKEmpty = kBKFull + kTStages;  // [kTStages] each
+constexpr int kBVFull = kBKEmpty + kTStages, kBVEmpty = kBVFull + kTStages;
+constexpr int kBSFull = kBVEmpty + kTStages, kBSEmpty = kBSFull + 2;  // [2] each
+constexpr int kBPFull = kBSEmpty + 2, kBPFree = kBPFull + 2;
+constexpr int kBOEmpty = kBPFree + 2;
+constexpr int kBXm = kBOEmpty + 1;  // [4 lane quarters][2 buffers]
+constexpr int kBXl = kBXm + 8;      // [4 lane quarters]
+constexpr int kBMgAll = kBXl + 4, kBMgDec = kBMgAll + 1, kBFinal = kBMgDec + 1;
+static_assert(kBFinal < kNumBars, "barrier slots");
 
 // ---------------------------------------------------------------- union lists
 
-// Entry: block (bits 0..23) | rows reading all 8 tokens << 24 | rows reading it
-// as their current block << 28.
+// Entry: block (bits 0..23) | rows that selected it << 24 (bit j = row j).
 __global__ void __launch_bounds__(256) tile_union_kernel(const TileArgs a) {
-  extern __shared__ uint32_t bm[];  // [4 rows][words]
+  extern __shared__ uint32_t bmap[];  // byte b: rows that selected block b
   __shared__ int cur_blk[kTRows];
-  __shared__ int scan[32];
+  __shared__ int scan[8];
   const int s = blockIdx.y, k = blockIdx.x;
   const int tile = s * a.tiles_per_seq + k;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -73,10 +107,13 @@ __global__ void __launch_bounds__(256) tile_union_kernel(const TileArgs a) {
     return;
   }
   const int c_last = (ctx + k * kTRows + nr - 1) / kBlk;  // largest current block of the tile
-  const int words = c_last / 32 + 1;
-  if (ctx < 0 || r0 + nr > a.total_q || words > a.bitmap_words) {
+  const int words = c_last / 4 + 1;
+  const bool bad = ctx < 0 || r0 < 0 || r0 + nr > a.total_q;
+  if (bad || words > a.map_words) {
+    // bad batch data (recorded; the per-row kernel reports it too), or a
+    // history too long for the shared map: the rows go to the per-row kernel
     if (tid == 0) {
-      record_error(a.err, S5_ERR_DEVICE_BOUNDS, max(r0, 0));
+      if (bad) record_error(a.err, S5_ERR_DEVICE_BOUNDS, max(r0, 0));
       *count = 0;
       a.tile_on[tile] = 0;
       for (int j = 0; j < nr; ++j)
@@ -84,7 +121,7 @@ __global__ void __launch_bounds__(256) tile_union_kernel(const TileArgs a) {
     }
     return;
   }
-  for (int i = tid; i < kTRows * words; i += 256) bm[i] = 0;
+  for (int i = tid; i < words; i += 256) bmap[i] = 0;
   if (tid < kTRows) cur_blk[tid] = (tid < nr) ? (ctx + k * kTRows + tid) / kBlk : -1;
   __syncthreads();
   int row_blocks = 0;  // sum over the tile's rows of (selected blocks + current block)
@@ -99,22 +136,25 @@ __global__ void __launch_bounds__(256) tile_union_kernel(const TileArgs a) {
     row_blocks += n + 1;
     for (int i = tid; i < n; i += 256) {
       const int b = ld_cg(a.sel + (size_t)r * a.topk + i);
-      if (b >= 0 && b < c) atomicOr(bm + j * words + (b >> 5), 1u << (b & 31));
+      if (b >= 0 && b < c) atomicOr(bmap + (b >> 2), (1u << j) << ((b & 3) * 8));
       else record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
     }
   }
   __syncthreads();
-  // ascending compaction of the union of the 4 bitmaps and the current blocks
-  const int per = (words + 255) / 256;  // words per thread, in order
-  int cnt = 0;
-  for (int w = tid * per; w < min(words, tid * per + per); ++w) {
-    uint32_t u = 0;
-    for (int j = 0; j < kTRows; ++j) u |= bm[j * words + w];
+  // ascending compaction of the selected blocks and the current blocks
+  auto in_union = [&](int b, uint32_t byte) {
+    if (byte != 0) return true;
     for (int j = 0; j < nr; ++j)
-      if ((cur_blk[j] >> 5) == w) u |= 1u << (cur_blk[j] & 31);
-    cnt += __popc(u);
+      if (cur_blk[j] == b) return true;
+    return false;
+  };
+  const int per = (words + 255) / 256;  // words per thread, in order
+  const int w_lo = min(words, tid * per), w_hi = min(words, tid * per + per);
+  int cnt = 0;
+  for (int w = w_lo; w < w_hi; ++w) {
+    const uint32_t u = bmap[w];
+    for (int q = 0; q < 4; ++q) cnt += in_union(4 * w + q, (u >> (8 * q)) & 0xFFu) ? 1 : 0;
   }
-  // exclusive scan of per-thread counts
   int incl = cnt;
   for (int off = 1; off < 32; off <<= 1) {
     const int o = __shfl_up_sync(0xffffffffu, incl, off);
@@ -133,21 +173,13 @@ __global__ void __launch_bounds__(256) tile_union_kernel(const TileArgs a) {
   __syncthreads();
   int pos = (warp > 0 ? scan[warp - 1] : 0) + incl - cnt;
   const int total = scan[7];
-  for (int w = tid * per; w < min(words, tid * per + per); ++w) {
-    uint32_t u = 0;
-    for (int j = 0; j < kTRows; ++j) u |= bm[j * words + w];
-    for (int j = 0; j < nr; ++j)
-      if ((cur_blk[j] >> 5) == w) u |= 1u << (cur_blk[j] & 31);
-    while (u != 0) {
-      const int bit = __ffs(u) - 1;
-      u &= u - 1;
-      const int b = w * 32 + bit;
-      uint32_t full = 0, cur = 0;
-      for (int j = 0; j < nr; ++j) {
-        if (bm[j * words + w] & (1u << bit)) full |= 1u << j;
-        if (cur_blk[j] == b) cur |= 1u << j;
-      }
-      if (pos < a.union_cap) ent[pos] = (uint32_t)b | (full << 24) | (cur << 28);
+  for (int w = w_lo; w < w_hi; ++w) {
+    const uint32_t u = bmap[w];
+    for (int q = 0; q < 4; ++q) {
+      const int b = 4 * w + q;
+      const uint32_t byte = (u >> (8 * q)) & 0xFFu;
+      if (!in_union(b, byte)) continue;
+      if (pos < a.union_cap) ent[pos] = (uint32_t)b | (byte << 24);
       ++pos;
     }
   }
@@ -162,14 +194,54 @@ __global__ void __launch_bounds__(256) tile_union_kernel(const TileArgs a) {
 
 // ---------------------------------------------------------------- attention tiles
 
-// byte offset of element (row, col) of a K-major 128-byte-swizzled [rows][64] bf16 tile
-__device__ __forceinline__ uint32_t sw128(int row, int col) {
-  const uint32_t off = (uint32_t)(row * 128 + col * 2);
-  return off ^ (((off >> 7) & 7u) << 4);
+struct TileItem {
+  int tile, g, p, s, k, r0, nr, ctx, e0, ne, n_chunks;
+  bool on;
+};
+
+// Work item idx: partition fastest, then tile, then KV group (CTAs working at
+// the same time share one group's blocks of neighbouring tiles in L2).  The
+// tiles are the n_list shared-set tiles in `list` (ascending), or all tiles
+// when list is null.
+__device__ __forceinline__ TileItem decode_item(const TileArgs &a, const int *list, int n_list, int idx) {
+  TileItem it;
+  it.p = idx % a.n_split;
+  const int tg = idx / a.n_split;
+  const int rank = tg % n_list;
+  it.tile = (list != nullptr) ? list[rank] : rank;
+  it.g = tg / n_list;
+  it.s = it.tile / a.tiles_per_seq;
+  it.k = it.tile % a.tiles_per_seq;
+  const int q_beg = ld_cg(a.cu_q + it.s);
+  const int nq = ld_cg(a.cu_q + it.s + 1) - q_beg;
+  it.ctx = ld_cg(a.ctx_lens + it.s);
+  it.r0 = q_beg + it.k * kTRows;
+  it.nr = max(0, min(kTRows, nq - it.k * kTRows));
+  it.on = it.nr > 0 && ld_cg(a.tile_on + it.tile) != 0;
+  it.e0 = it.ne = it.n_chunks = 0;
+  if (it.on) {
+    const int n_ent = max(0, min(ld_cg(a.union_count + it.tile), a.union_cap));
+    const int per = (n_ent + a.n_split - 1) / a.n_split;
+    const int chunk_e = (per + kTChunkBlocks - 1) / kTChunkBlocks * kTChunkBlocks;
+    it.e0 = min(n_ent, it.p * chunk_e);
+    it.ne = min(n_ent, it.e0 + chunk_e) - it.e0;
+    it.n_chunks = (it.ne + kTChunkBlocks - 1) / kTChunkBlocks;
+  }
+  return it;
+}
+
+// TMA row of a union entry in group it.g of the paged pool, or -1 (recorded).
+__device__ __forceinline__ int entry_row(const TileArgs &a, const TileItem &it, uint32_t e) {
+  const int b = (int)(e & 0xFFFFFFu);
+  const int pg = b / kBpp;
+  const int ph = (pg < a.max_pages) ? ld_cg(a.page_table + (size_t)it.s * a.max_pages + pg) : -1;
+  if (ph >= 0 && ph < a.num_pages) return ((ph * kKv + it.g) * kPage) + (b % kBpp) * kBlk;
+  record_error(a.err, S5_ERR_DEVICE_BOUNDS, it.r0);
+  return -1;
 }
 
 // Merge weights of the partitions of one (row, head): the same arithmetic as
-// the decode kernel's merge, in partition order.
+// the per-row kernel's merge, in partition order.
 __device__ __forceinline__ void tile_partition_weights(const float *pl, int n, float *w, float &lse_nat) {
   float M = -INFINITY;
   for (int p = 0; p < n; ++p) M = fmaxf(M, ld_cg(pl + p));
@@ -188,438 +260,509 @@ __device__ __forceinline__ void tile_partition_weights(const float *pl, int n, f
 }
 
 __global__ void __launch_bounds__(kTThreads, 1)
-    gqa_tile_kernel(const TileArgs a, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v) {
+    gqa_tile_kernel(const TileArgs a, const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sq = smem;                                   // Q tile
-  uint8_t *skv = sq + kTQBytes;                         // K/V stages
-  uint8_t *sp = skv + kTStages * kTStageBytes;          // P buffers [3]
-  int32_t *erow = reinterpret_cast<int32_t *>(sp + kTPBufs * kTPBytes);  // TMA row per entry (-1: absent)
-  uint32_t *eent = reinterpret_cast<uint32_t *>(erow + kMaxTileEntries);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(eent + kMaxTileEntries);
-  uint64_t *bar_q = bars + 0;
-  uint64_t *bar_kv_full = bars + 1;    // [3]
-  uint64_t *bar_kv_empty = bars + 4;   // [3]
-  uint64_t *bar_s_full = bars + 7;     // [2]
-  uint64_t *bar_s_empty = bars + 9;    // [2]
-  uint64_t *bar_p_full = bars + 11;    // [3] P_c written (chunk c uses buffer c % 3)
-  uint64_t *bar_p_free = bars + 14;    // [3] PV_c done: P buffer c % 3 and O through chunk c
-  uint64_t *bar_final = bars + 17;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
-  int *abort_flag = reinterpret_cast<int *>(bars + 19);
-  int *is_last = abort_flag + 1;
+  uint8_t *sk = smem + kOffK;
+  uint8_t *sv = smem + kOffV;
+  float *xm = reinterpret_cast<float *>(smem + kOffXm);
+  float *xl = reinterpret_cast<float *>(smem + kOffXl);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+  int *abort_flag = reinterpret_cast<int *>(smem + kOffMisc + 4);
+  int *is_last = reinterpret_cast<int *>(smem + kOffMisc + 8);
+
+  int *list_s = reinterpret_cast<int *>(smem + kOffList);
+  int *wsum = reinterpret_cast<int *>(smem + kOffMisc + 16);  // [11] per-warp counts
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // flattened grid: partition fastest, then tile, then group
-  const int p = blockIdx.x % a.n_split;
-  const int tg = blockIdx.x / a.n_split;
-  const int tile = tg % a.n_tiles;
-  const int g = tg / a.n_tiles;
-  pdl_wait();  // (no-op for an ordinary launch) every global read below follows it
 
-  // ---- the tile ----
-  const int s = tile / a.tiles_per_seq, k = tile % a.tiles_per_seq;
-  const int q_beg = ld_cg(a.cu_q + s);
-  const int nq = ld_cg(a.cu_q + s + 1) - q_beg;
-  const int ctx = ld_cg(a.ctx_lens + s);
-  const int r0 = q_beg + k * kTRows;
-  const int nr = max(0, min(kTRows, nq - k * kTRows));
-  if (nr == 0) return;  // a tile slot past this sequence's rows
-  if (ld_cg(a.tile_on + tile) == 0) return;  // the per-row kernel computes this tile's rows
-  const int n_ent = ld_cg(a.union_count + tile);
+  // ---- the shared-set tiles, in order (most batches of independent queries have none) ----
+  const int *list = nullptr;
+  int n_list = a.n_tiles;
+  if (a.n_tiles <= kMaxListTiles) {
+    int base = 0;
+    for (int i0 = 0; i0 < a.n_tiles; i0 += kTThreads) {
+      const int i = i0 + tid;
+      const bool on = i < a.n_tiles && ld_cg(a.tile_on + i) != 0;
+      const uint32_t bal = __ballot_sync(0xffffffffu, on);
+      if (lane == 0) wsum[warp] = __popc(bal);
+      __syncthreads();
+      int before = base;
+      for (int w = 0; w < warp; ++w) before += wsum[w];
+      if (on) list_s[before + __popc(bal & ((1u << lane) - 1u))] = i;
+      int tot = 0;
+      for (int w = 0; w < kTThreads / 32; ++w) tot += wsum[w];
+      __syncthreads();
+      base += tot;
+    }
+    list = list_s;
+    n_list = base;
+    if (n_list == 0) return;  // every tile goes to the per-row kernel
+  }
+  const int n_items = n_list * kKv * a.n_split;
 
+  // K/V slots that no copy fills (padding, an unmapped page) must hold finite
+  // values: start from zeros
+  for (int i = tid; i < (2 * kTStages * kTKvBytes) / 16; i += kTThreads)
+    reinterpret_cast<uint4 *>(sk)[i] = make_uint4(0, 0, 0, 0);
   if (warp == 0) tc::tmem_alloc(tmem_slot, kTTmemCols);
   if (tid == 0) {
-    mbar_init(bar_q, 1);
+    mbar_init(bars + kBQFull, kTSoftWarps);
+    mbar_init(bars + kBQEmpty, 1);
     for (int i = 0; i < kTStages; ++i) {
-      mbar_init(bar_kv_full + i, 1);
-      mbar_init(bar_kv_empty + i, 1);
+      mbar_init(bars + kBKFull + i, 1);
+      mbar_init(bars + kBKEmpty + i, 1);
+      mbar_init(bars + kBVFull + i, 1);
+      mbar_init(bars + kBVEmpty + i, 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_s_full + i, 1);
-      mbar_init(bar_s_empty + i, 4);
+      mbar_init(bars + kBSFull + i, 1);
+      mbar_init(bars + kBSEmpty + i, kTSoftWarps);
+      mbar_init(bars + kBPFull + i, kTSoftWarps);
+      mbar_init(bars + kBPFree + i, 1);
     }
-    for (int i = 0; i < kTPBufs; ++i) {
-      mbar_init(bar_p_full + i, 4);
-      mbar_init(bar_p_free + i, 1);
-    }
-    mbar_init(bar_final, 1);
+    mbar_init(bars + kBOEmpty, kTSoftWarps);
+    for (int i = 0; i < 8; ++i) mbar_init(bars + kBXm + i, 64);
+    for (int i = 0; i < 4; ++i) mbar_init(bars + kBXl + i, 64);
+    mbar_init(bars + kBMgAll, kTSoftThreads);
+    mbar_init(bars + kBMgDec, 1);
+    mbar_init(bars + kBFinal, 2);  // one commit from each MMA issuer
     *abort_flag = 0;
   }
   fence_mbar_init();
+  fence_proxy_async_smem();  // the zero fill before any copy or MMA touches those bytes
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int chunk_e = ((n_ent + a.n_split - 1) / a.n_split + kTChunkBlocks - 1) / kTChunkBlocks * kTChunkBlocks;
-  const int e0 = min(n_ent, p * chunk_e);
-  const int ne = min(n_ent, e0 + chunk_e) - e0;  // this CTA's entries (<= kMaxTileEntries: host sizes n_split)
-  const int n_chunks = (ne + kTChunkBlocks - 1) / kTChunkBlocks;
-  const int32_t *pt = a.page_table + (size_t)s * a.max_pages;
-  // resolve entries to TMA rows
-  for (int i = tid; i < n_chunks * kTChunkBlocks; i += kTThreads) {
-    int row = -1;
-    uint32_t e = 0;
-    if (i < ne) {
-      e = ld_cg(a.union_ent + (size_t)tile * a.union_cap + e0 + i);
-      const int b = (int)(e & 0xFFFFFFu);
-      const int pg = b / kBpp;
-      const int ph = (pg < a.max_pages) ? ld_cg(pt + pg) : -1;
-      if (ph >= 0 && ph < a.num_pages) row = ((ph * kKv + g) * kPage) + (b % kBpp) * kBlk;
-      else record_error(a.err, S5_ERR_DEVICE_BOUNDS, r0);
-    }
-    erow[i] = row;
-    eent[i] = (row >= 0) ? e : 0u;
-  }
-  __syncthreads();
 
   auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
     if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
     if (mbar_wait_bounded(bar, parity, kTWaitNs)) return true;
     *reinterpret_cast<volatile int *>(abort_flag) = 1;
-    record_error(a.err, S5_ERR_TIMEOUT, max(r0, 0));
+    record_error(a.err, S5_ERR_TIMEOUT, 0);
     return false;
   };
 
-  if (warp == 4) {
-    // ---------------- TMA producer ----------------
-    // A chunk is 8 blocks x (K, V): 16 copies of one whole block (3 planes of
-    // 1 KB), issued in parallel by lanes 0..15 (lane = 8 * tensor + block);
-    // lane 0 keeps the barrier bookkeeping.
-    if (n_chunks > 0) {
-      if (lane == 0) {
-        // Q: rows (query j, head 16g + h) -> smem row 16j + h; 3 K-blocks of 64 dims
-        mbar_arrive_expect_tx(bar_q, kTQBytes);
-        for (int j = 0; j < kTRows; ++j)
-          for (int cb = 0; cb < 3; ++cb)
-            tma_load_2d(sq + cb * kTM * 128 + j * kHpg * 128, &tm_q, cb * 64,
-                        (min(r0 + j, a.total_q - 1)) * kHeads + g * kHpg, bar_q);
-      }
-      const uint64_t policy = policy_evict_normal();
-      const int lb = lane & 7, lt = (lane >> 3) & 1;  // block and tensor (0 = K, 1 = V) of this lane
-      int issued = 0;
-      for (int c = 0; c < n_chunks; ++c) {
-        const int st = c % kTStages;
+  if (warp == kTWarpK || warp == kTWarpV) {
+    // ---------------- TMA producers: warp 8 K, warp 9 V ----------------
+    // Lane b < 8 copies block b of each chunk (one 3 KB box: 3 planes x 8
+    // tokens x 64 dims); lane 0 keeps the barrier bookkeeping.
+    const bool is_k = warp == kTWarpK;
+    uint8_t *ring = is_k ? sk : sv;
+    const CUtensorMap *map = is_k ? &tm_k : &tm_v;
+    uint64_t *full = bars + (is_k ? kBKFull : kBVFull);
+    uint64_t *empty = bars + (is_k ? kBKEmpty : kBVEmpty);
+    const uint64_t policy = policy_evict_normal();
+    int gc = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      const TileItem it = decode_item(a, list, n_list, idx);
+      if (it.n_chunks == 0) continue;
+      const uint32_t *ent = a.union_ent + (size_t)it.tile * a.union_cap + it.e0;
+      for (int c = 0; c < it.n_chunks; ++c, ++gc) {
+        const int st = gc % kTStages;
         int go = 1;
-        if (lane == 0 && c >= kTStages) go = wait(bar_kv_empty + st, ((c / kTStages) - 1) & 1) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, go, 0)) break;
-        const int row = (lane < 16) ? erow[c * kTChunkBlocks + lb] : -1;
+        if (lane == 0 && gc >= kTStages) go = wait(empty + st, ((gc / kTStages) - 1) & 1) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, go, 0)) {
+          ok = false;
+          break;
+        }
+        const int i = c * kTChunkBlocks + lane;
+        const int row = (lane < kTChunkBlocks && i < it.ne) ? entry_row(a, it, ld_cg(ent + i)) : -1;
         uint32_t bytes = (row >= 0) ? (uint32_t)kBlockBytes : 0u;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, off);
-        if (lane == 0) mbar_arrive_expect_tx(bar_kv_full + st, bytes);
+        if (lane == 0) mbar_arrive_expect_tx(full + st, bytes);
         __syncwarp();
-        if (row >= 0)
-          tma_load_3d(skv + st * kTStageBytes + lt * kTKvBytes + lb * kBlockBytes, lt ? &tm_v : &tm_k, 0, row, 0,
-                      bar_kv_full + st, policy);
-        ++issued;
-      }
-      if (lane == 0 && *reinterpret_cast<volatile int *>(abort_flag)) {  // drain copies still in flight
-        mbar_wait_bounded(bar_q, 0, kTWaitNs);
-        for (int c = max(0, issued - kTStages); c < issued; ++c)
-          mbar_wait_bounded(bar_kv_full + c % kTStages, (c / kTStages) & 1, kTWaitNs);
+        if (row >= 0) tma_load_3d(ring + st * kTKvBytes + lane * kBlockBytes, map, 0, row, 0, full + st, policy);
       }
     }
-  } else if (warp == 5) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0 && n_chunks > 0) {
+    // no copy may still be writing shared memory when the CTA retires
+    if (lane == 0) {
+      for (int c = max(0, gc - kTStages); c < gc; ++c)
+        mbar_wait_bounded(full + c % kTStages, (c / kTStages) & 1, kTWaitNs);
+    }
+  } else if (warp == kTWarpS) {
+    // ---------------- S issuer ----------------
+    if (lane == 0) {
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(kTM, kTN);
-      constexpr uint32_t idesc_o = tc::idesc_bf16_f32_bmn(kTM, kD);  // B = V, MN-major
-      const uint32_t q_base = smem_u32(sq), kv_base = smem_u32(skv), p_base = smem_u32(sp);
-      const uint32_t t_o = tmem + 128;
-      auto issue_pv = [&](int c) -> bool {  // O += P_c V_c
-        const int pb = c % kTPBufs;
-        if (!wait(bar_p_full + pb, (c / kTPBufs) & 1)) return false;
-        tc::fence_after_sync();
-        const int st = c % kTStages;
-#pragma unroll
-        for (int ks = 0; ks < kTN / 16; ++ks) {
-          // A = P [64 rows][64 tokens], K-major; B = V, N = 192 dims MN-major over the chunk's 64 tokens:
-          // 64-dim chunks 1,024 B apart (leading), 8-token groups 3,072 B apart (stride)
-          const uint64_t ad = tc::smem_desc_k_sw128(p_base + pb * kTPBytes + ks * 32);
-          const uint64_t bd = tc::smem_desc_mn_sw128(kv_base + st * kTStageBytes + kTKvBytes + ks * 2 * kBlockBytes,
-                                                     1024, kBlockBytes);
-          tc::mma_bf16(t_o, ad, bd, idesc_o, c > 0 || ks > 0);
-        }
-        tc::commit(bar_kv_empty + st);
-        tc::commit(bar_p_free + pb);
-        return true;
-      };
-      if (wait(bar_q, 0)) {
-        bool ok = true;
-        for (int c = 0; c < n_chunks && ok; ++c) {
-          const int st = c % kTStages, sb = c & 1;
-          if (!wait(bar_kv_full + st, (c / kTStages) & 1)) break;
-          if (c >= 2 && !wait(bar_s_empty + sb, ((c >> 1) - 1) & 1)) break;
-          tc::fence_after_sync();
-          // S_c = Q K_c^T: K = 192 as 3 swizzle blocks of 64; the chunk's 8 blocks
-          // are 8-token groups 3,072 B apart, each block's 64-dim chunk cb at cb * 1,024
-#pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const int cb = ks >> 2, kk = ks & 3;
-            const uint64_t ad = tc::smem_desc_k_sw128(q_base + cb * kTM * 128 + kk * 32);
-            const uint64_t bd =
-                tc::smem_desc_k_sw128_stride(kv_base + st * kTStageBytes + cb * 1024 + kk * 32, kBlockBytes);
-            tc::mma_bf16(tmem + sb * kTN, ad, bd, idesc_s, ks > 0);
+      const uint32_t k_base = smem_u32(sk);
+      int gc = 0, qi = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+        const TileItem it = decode_item(a, list, n_list, idx);
+        if (it.n_chunks == 0) continue;
+        if (!wait(bars + kBQFull, qi & 1)) break;
+        for (int c = 0; c < it.n_chunks; ++c, ++gc) {
+          const int st = gc % kTStages, sb = gc & 1;
+          if (!wait(bars + kBKFull + st, (gc / kTStages) & 1) ||
+              (gc >= 2 && !wait(bars + kBSEmpty + sb, ((gc >> 1) - 1) & 1))) {
+            ok = false;
+            break;
           }
-          tc::commit(bar_s_full + sb);
-          if (c > 0) ok = issue_pv(c - 1);
+          tc::fence_after_sync();
+          // S = Q K^T: Q from tensor memory (K-step kk = 8 columns); K = 192
+          // as 3 swizzled planes of 64; the chunk's blocks are 8-token groups
+          // 3,072 B apart, plane cb of a block at cb * 1,024
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const int cb = kk >> 2, k4 = kk & 3;
+            const uint64_t bd =
+                tc::smem_desc_k_sw128_stride(k_base + st * kTKvBytes + cb * 1024 + k4 * 32, kBlockBytes);
+            tc::mma_bf16_ts(tmem + kTmemS + sb * kTN, tmem + kTmemQ + kk * 8, bd, idesc_s, kk > 0);
+          }
+          tc::commit(bars + kBKEmpty + st);
+          tc::commit(bars + kBSFull + sb);
+          if (c == it.n_chunks - 1) tc::commit(bars + kBQEmpty);
         }
-        if (ok && !*reinterpret_cast<volatile int *>(abort_flag)) issue_pv(n_chunks - 1);
+        ++qi;
       }
-      tc::commit(bar_final);  // arrives once every MMA issued above has completed
+      tc::commit(bars + kBFinal);  // arrives once every MMA issued above has completed
+    }
+  } else if (warp == kTWarpPv) {
+    // ---------------- PV issuer ----------------
+    // O += P_x V_x (P: tensor memory, 64 tokens = 4 K-steps of 8 columns; V:
+    // 64-dim planes 1,024 B apart (leading), 8-token blocks 3,072 B apart (stride))
+    if (lane == 0) {
+      constexpr uint32_t idesc_o = tc::idesc_bf16_f32_bmn(kTM, kD);  // B = V, MN-major
+      const uint32_t v_base = smem_u32(sv);
+      int gc = 0, qi = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+        const TileItem it = decode_item(a, list, n_list, idx);
+        if (it.n_chunks == 0) continue;
+        for (int c = 0; c < it.n_chunks; ++c, ++gc) {
+          const bool first = c == 0;
+          if (!wait(bars + kBPFull + (gc & 1), (gc >> 1) & 1) ||
+              !wait(bars + kBVFull + gc % kTStages, (gc / kTStages) & 1) ||
+              (first && qi > 0 && !wait(bars + kBOEmpty, (qi - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const int vs = gc % kTStages;
+#pragma unroll
+          for (int ks = 0; ks < kTN / 16; ++ks) {
+            const uint64_t bd =
+                tc::smem_desc_mn_sw128(v_base + vs * kTKvBytes + ks * 2 * kBlockBytes, 1024, kBlockBytes);
+            tc::mma_bf16_ts(tmem + kTmemO, tmem + kTmemP + (gc & 1) * 32 + ks * 8, bd, idesc_o, !first || ks > 0);
+          }
+          tc::commit(bars + kBVEmpty + vs);
+          tc::commit(bars + kBPFree + (gc & 1));
+        }
+        ++qi;
+      }
+      tc::commit(bars + kBFinal);
     }
   } else {
-    // ---------------- softmax / epilogue: warp w = query row w of the tile ----------------
-    // With the 16x256b tensor-memory shape, thread t holds heads h0 = t/4 and
-    // h1 = t/4 + 8 of this query, columns 8i + 2(t%4) and +1 (i = 0..7) of a
-    // 64-column tile: a head's row is spread over the 4 threads of a quad.
-    const int j = warp;  // row of the tile handled by this warp
-    const int h0 = lane >> 2, h1 = h0 + 8, cq = 2 * (lane & 3);
-    const int t = ctx + k * kTRows + j;
-    const bool row_ok = j < nr;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // ---------------- softmax / epilogue: warps 0-7 ----------------
+    // Warp w reads lanes 32 (w % 4) .. + 31 (tile rows m = lane index: query
+    // j = m / 16, head h = m % 16) and columns 32 (w / 4) .. + 31 of each S.
+    const int q4 = warp & 3, half = warp >> 2;
+    const int m = q4 * 32 + lane;
+    const int j = m >> 4, h = m & 15;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const float sl2 = a.scale_log2;
-    const int t_max = ctx + k * kTRows + nr - 1;  // last position of the tile
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    int gc = 0, qi = 0, mi = 0;
     bool ok = true;
-    for (int c = 0; c < n_chunks; ++c) {
-      const int st = c % kTStages, sb = c & 1;
-      if (!wait(bar_s_full + sb, (c >> 1) & 1)) {
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-      uint32_t v[32];
-      tc::ld_16x256b_x8(tmem + lane_base + sb * kTN, v);
-      tc::wait_ld();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_s_empty + sb);
-      // column i of this thread: 8 i + cq (+1) = token 8 i + cq (+1) of block i of the chunk
-      float sv[2][16];
-      float mx[2] = {-INFINITY, -INFINITY};
-      bool need_zero = false;
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      const TileItem it = decode_item(a, list, n_list, idx);
+      if (!it.on) continue;
+      const bool row_ok = j < it.nr;
+      const int t = it.ctx + it.k * kTRows + j;  // this row's position
+      const int cj = t / kBlk;                    // and its current block
+      const int t_max = it.ctx + it.k * kTRows + it.nr - 1;
+      const uint32_t *ent = a.union_ent + (size_t)it.tile * a.union_cap + it.e0;
+      float m_ref = -INFINITY, l = 0.f;
+      if (it.n_chunks > 0) {
+        // Q of the item into tensor memory: this thread's row (query j, head
+        // 16g + h), dims 96 half .. + 95 (zeros past the tile's rows); the
+        // previous item's last S must be done with the old Q
+        if (qi > 0 && !wait(bars + kBQEmpty, (qi - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        uint32_t qv[48];
+        const uint4 *qs = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.q) +
+                                                          ((size_t)(it.r0 + j) * kHeads + it.g * kHpg + h) * kD +
+                                                          half * 96);
 #pragma unroll
-      for (int i = 0; i < kTChunkBlocks; ++i) {
-        const uint32_t e = eent[c * kTChunkBlocks + i];
-        const int blk = (int)(e & 0xFFFFFFu);
-        need_zero |= (erow[c * kTChunkBlocks + i] < 0) || (blk * kBlk + kBlk - 1 > t_max);
-        bool vis0 = false, vis1 = false;
-        if (row_ok) {
-          if ((e >> (24 + j)) & 1u) {
-            vis0 = vis1 = true;
-          } else if ((e >> (28 + j)) & 1u) {
-            vis0 = blk * kBlk + cq <= t;
-            vis1 = blk * kBlk + cq + 1 <= t;
-          }
+        for (int x = 0; x < 12; ++x) {
+          const uint4 u = row_ok ? ld_cg(qs + x) : make_uint4(0, 0, 0, 0);
+          qv[4 * x] = u.x;
+          qv[4 * x + 1] = u.y;
+          qv[4 * x + 2] = u.z;
+          qv[4 * x + 3] = u.w;
         }
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float s0 = vis0 ? __uint_as_float(v[4 * i + 2 * r]) * sl2 : -INFINITY;
-          const float s1 = vis1 ? __uint_as_float(v[4 * i + 2 * r + 1]) * sl2 : -INFINITY;
-          sv[r][2 * i] = s0;
-          sv[r][2 * i + 1] = s1;
-          mx[r] = fmaxf(mx[r], fmaxf(s0, s1));
+        for (int x = 0; x < 3; ++x) {
+          uint32_t w16[16];
+#pragma unroll
+          for (int y = 0; y < 16; ++y) w16[y] = qv[16 * x + y];
+          tc::st_16cols(tmem + lane_base + kTmemQ + half * 48 + x * 16, w16);
         }
+        tc::wait_st();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + kBQFull);
       }
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {  // row max over the quad
-        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-      }
-      // lazy rescale: keep the reference max unless a row's max grows by more than 2^8
-      float corr[2];
-      bool any_rescale = false;
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const bool grow = mx[r] > m[r] + kLazyRescale;
-        const float m_new = grow ? mx[r] : m[r];
-        corr[r] = (grow && m[r] != -INFINITY) ? hw_exp2(m[r] - m_new) : 1.f;
-        any_rescale |= grow && m[r] != -INFINITY;
-        m[r] = m_new;
-      }
-      if (__any_sync(0xffffffffu, any_rescale) && c > 0) {
-        // O holds chunks 0 .. c-1: wait for PV_{c-1} (in-order completion covers the rest)
-        if (!wait(bar_p_free + (c - 1) % kTPBufs, ((c - 1) / kTPBufs) & 1)) {
+      // lanes 0..3 hold the entries of this half's 4 blocks of the next chunk
+      uint32_t e_next = 0u;
+      if (lane < 4 && half * 4 + lane < it.ne) e_next = ld_cg(ent + half * 4 + lane);
+      for (int c = 0; c < it.n_chunks; ++c, ++gc) {
+        const uint32_t e_cur = e_next;
+        {
+          const int i = (c + 1) * kTChunkBlocks + half * 4 + lane;
+          e_next = (lane < 4 && c + 1 < it.n_chunks && i < it.ne) ? ld_cg(ent + i) : 0u;
+        }
+        const int sb = gc & 1;
+        if (!wait(bars + kBSFull + sb, (gc >> 1) & 1)) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        for (int cb = 0; cb < kD / 64; ++cb) {
-          uint32_t o[32];
-          tc::ld_16x256b_x8(tmem + lane_base + 128 + cb * 64, o);
-          tc::wait_ld();
+        uint32_t v[32];
+        tc::ld_32cols(tmem + lane_base + kTmemS + sb * kTN + half * 32, v);
+        tc::wait_ld();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + kBSEmpty + sb);
+        // mask: column x = 8 ib + tok is token tok of block (4 half + ib) of the chunk
+        float sc[32];  // scaled, masked scores
+        float mx = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            o[4 * i] = __float_as_uint(__uint_as_float(o[4 * i]) * corr[0]);
-            o[4 * i + 1] = __float_as_uint(__uint_as_float(o[4 * i + 1]) * corr[0]);
-            o[4 * i + 2] = __float_as_uint(__uint_as_float(o[4 * i + 2]) * corr[1]);
-            o[4 * i + 3] = __float_as_uint(__uint_as_float(o[4 * i + 3]) * corr[1]);
+        for (int ib = 0; ib < 4; ++ib) {
+          const uint32_t e = __shfl_sync(0xffffffffu, e_cur, ib);
+          const bool valid = row_ok && (c * kTChunkBlocks + half * 4 + ib < it.ne);
+          const int blk = (int)(e & 0xFFFFFFu);
+          const bool sel = valid && ((e >> (24 + j)) & 1u);
+          const int lim = sel ? kBlk - 1 : ((valid && blk == cj) ? t - blk * kBlk : -1);  // tokens 0..lim visible
+#pragma unroll
+          for (int tok = 0; tok < kBlk; ++tok) {
+            const float s = (tok <= lim) ? __uint_as_float(v[ib * kBlk + tok]) * sl2 : -INFINITY;
+            sc[ib * kBlk + tok] = s;
+            mx = fmaxf(mx, s);
           }
-          tc::st_16x256b_x8(tmem + lane_base + 128 + cb * 64, o);
+        }
+        // row max over both halves
+        float *xmb = xm + sb * 2 * kTM;
+        xmb[half * kTM + m] = mx;
+        mbar_arrive(bars + kBXm + q4 * 2 + sb);
+        if (!wait(bars + kBXm + q4 * 2 + sb, (gc >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        const float rmax = fmaxf(mx, xmb[(1 - half) * kTM + m]);
+        // lazy rescale: keep the reference max unless the row max grows by more than 2^8
+        const bool grow = rmax > m_ref + kLazyRescale;
+        const bool resc = grow && m_ref != -INFINITY;
+        const float corr = resc ? hw_exp2(m_ref - rmax) : 1.f;
+        if (grow) m_ref = rmax;
+        if (__any_sync(0xffffffffu, resc) && c > 0) {
+          // O holds chunks up to gc - 1: wait for that PV (in-order completion covers the rest)
+          if (!wait(bars + kBPFree + ((gc - 1) & 1), ((gc - 1) >> 1) & 1)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+#pragma unroll 1
+          for (int cb = 0; cb < 3; ++cb) {
+            uint32_t o[32];
+            const uint32_t ta = tmem + lane_base + kTmemO + half * 96 + cb * 32;
+            tc::ld_32cols(ta, o);
+            tc::wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * corr);
+            tc::st_32cols(ta, o);
+          }
+          tc::wait_st();
+        }
+        l *= corr;
+        // P (bf16) into tensor-memory buffer sb, last read by the PV of chunk gc - 2
+        if (gc >= 2 && !wait(bars + kBPFree + sb, ((gc >> 1) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+        uint32_t pk[16];
+        float ps = 0.f;
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const float p0 = hw_exp2(sc[2 * x] - mu);
+          const float p1 = hw_exp2(sc[2 * x + 1] - mu);
+          ps += p0 + p1;
+          pk[x] = pack_bf16(p0, p1);
+        }
+        l += ps;
+        tc::st_16cols(tmem + lane_base + kTmemP + sb * 32 + half * 16, pk);
+        // V rows no row may read (padding slots, tokens past the tile's last
+        // position, all in the item's last chunk) must be finite: zero them
+        // (P is 0 there, but 0 * NaN is NaN).  Warp w checks block w.
+        if (c == it.n_chunks - 1) {
+          const int ir = c * kTChunkBlocks + warp;
+          const int blk = (ir < it.ne) ? (int)(ld_cg(ent + ir) & 0xFFFFFFu) : -1;
+          const int first_bad = (blk < 0) ? 0 : t_max - blk * kBlk + 1;  // tokens >= first_bad are zeroed
+          if (first_bad < kBlk) {
+            if (!wait(bars + kBVFull + gc % kTStages, (gc / kTStages) & 1)) {
+              ok = false;
+              break;
+            }
+            uint8_t *vb = sv + (gc % kTStages) * kTKvBytes + warp * kBlockBytes;
+            for (int x = lane; x < 3 * kBlk * 8; x += 32) {  // plane, token, 16-byte chunk
+              const int tok = (x >> 3) & 7;
+              if (tok >= first_bad)
+                *reinterpret_cast<uint4 *>(vb + (x >> 6) * 1024 + tok * 128 + (x & 7) * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+          }
         }
         tc::wait_st();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + kBPFull + sb);
       }
-      // P (bf16) into P buffer c % 3, last read by PV_{c-3}
-      const int pbi = c % kTPBufs;
-      if (c >= kTPBufs && !wait(bar_p_free + pbi, ((c / kTPBufs) - 1) & 1)) {
+      if (!ok) break;
+      // ---- epilogue: O / l of the item ----
+      float lt = 0.f;
+      const bool have = it.n_chunks > 0;
+      if (have) {
+        xl[half * kTM + m] = l;
+        mbar_arrive(bars + kBXl + q4);
+        if (!wait(bars + kBXl + q4, qi & 1)) {
+          ok = false;
+          break;
+        }
+        lt = l + xl[(1 - half) * kTM + m];
+        if (!wait(bars + kBPFree + ((gc - 1) & 1), ((gc - 1) >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+      }
+      const float inv = (lt > 0.f) ? 1.f / lt : 0.f;
+      const float lse2 = (lt > 0.f) ? m_ref + hw_log2(lt) : -INFINITY;
+      const size_t rh = (size_t)(it.r0 + j) * kHeads + it.g * kHpg + h;
+#pragma unroll 1
+      for (int cb = 0; cb < 3; ++cb) {
+        uint32_t o[32];
+        if (have) {
+          tc::ld_32cols(tmem + lane_base + kTmemO + half * 96 + cb * 32, o);
+          tc::wait_ld();
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = 0u;
+        }
+        if (row_ok) {
+          const int d0 = half * 96 + cb * 32;
+          if (a.n_split == 1) {
+            uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(a.out) + rh * kD + d0);
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+              dst[x] = make_uint4(pack_bf16(__uint_as_float(o[8 * x]) * inv, __uint_as_float(o[8 * x + 1]) * inv),
+                                  pack_bf16(__uint_as_float(o[8 * x + 2]) * inv, __uint_as_float(o[8 * x + 3]) * inv),
+                                  pack_bf16(__uint_as_float(o[8 * x + 4]) * inv, __uint_as_float(o[8 * x + 5]) * inv),
+                                  pack_bf16(__uint_as_float(o[8 * x + 6]) * inv, __uint_as_float(o[8 * x + 7]) * inv));
+          } else {
+            float4 *dst = reinterpret_cast<float4 *>(a.part_o + (rh * a.n_split + it.p) * kD + d0);
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              dst[x] = make_float4(__uint_as_float(o[4 * x]) * inv, __uint_as_float(o[4 * x + 1]) * inv,
+                                   __uint_as_float(o[4 * x + 2]) * inv, __uint_as_float(o[4 * x + 3]) * inv);
+          }
+        }
+      }
+      if (have) {
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + kBOEmpty);
+        ++qi;
+      }
+      if (row_ok && half == 0) {
+        if (a.n_split == 1) {
+          if (a.lse != nullptr) a.lse[rh] = lse2 * 0.69314718055994531f;
+        } else {
+          a.part_lse[rh * a.n_split + it.p] = lse2;
+        }
+      }
+      if (a.n_split == 1) continue;
+      // ---- the last partition to finish (tile, group) merges every partition ----
+      __threadfence();
+      mbar_arrive(bars + kBMgAll);
+      if (tid == 0) {
+        int last = 0;
+        if (wait(bars + kBMgAll, mi & 1)) {
+          uint32_t *cnt = a.merge_cnt + (size_t)it.tile * kKv + it.g;
+          const uint32_t prev = atomicAdd(cnt, 1u);
+          last = (prev == (uint32_t)a.n_split - 1) ? 1 : 0;
+          if (last) *cnt = 0u;  // every partition has arrived: ready for the next call
+        }
+        *is_last = last;
+        mbar_arrive(bars + kBMgDec);
+      }
+      if (!wait(bars + kBMgDec, mi & 1)) {
         ok = false;
         break;
       }
-      uint8_t *pb = sp + pbi * kTPBytes;
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const float mu = (m[r] == -INFINITY) ? 0.f : m[r];
-        const int row = j * kHpg + (r ? h1 : h0);
-        float psum = 0.f;
-#pragma unroll
-        for (int i = 0; i < kTChunkBlocks; ++i) {
-          const float p0 = hw_exp2(sv[r][2 * i] - mu);
-          const float p1 = hw_exp2(sv[r][2 * i + 1] - mu);
-          psum += p0 + p1;
-          *reinterpret_cast<uint32_t *>(pb + sw128(row, 8 * i + cq)) = pack_bf16(p0, p1);
-        }
-        psum += __shfl_xor_sync(0xffffffffu, psum, 1);
-        psum += __shfl_xor_sync(0xffffffffu, psum, 2);
-        l[r] = l[r] * corr[r] + psum;
-      }
-      // V rows no row of the tile may read (absent blocks, tokens past the tile's
-      // last position) must be finite: zero them (P is 0 there, but 0 * NaN is NaN)
-      if (__any_sync(0xffffffffu, need_zero)) {
-        uint8_t *vb = skv + st * kTStageBytes + kTKvBytes;
-        for (int b = j; b < kTChunkBlocks; b += 4) {
-          const int idx = c * kTChunkBlocks + b;
-          const int blk = (int)(eent[idx] & 0xFFFFFFu);
-          const bool absent = erow[idx] < 0;
-          if (!absent && blk * kBlk + kBlk - 1 <= t_max) continue;
-          for (int x = lane; x < 3 * kBlk * 8; x += 32) {  // 3 planes x 8 tokens x 8 16-byte chunks
-            const int tok = (x >> 3) & 7;
-            if (absent || blk * kBlk + tok > t_max)
-              *reinterpret_cast<uint4 *>(vb + b * kBlockBytes + (x >> 6) * 1024 + tok * 128 + (x & 7) * 16) =
-                  make_uint4(0, 0, 0, 0);
-          }
-        }
-      }
-      fence_proxy_async_smem();  // generic writes (P, zeroed V rows) before the tensor core reads them
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p_full + pbi);
-    }
-    // ---- epilogue: O / l ----
-    if (!ok) *reinterpret_cast<volatile int *>(abort_flag) = 1;
-    const bool have = ok && n_chunks > 0 &&
-                      wait(bar_p_free + (n_chunks - 1) % kTPBufs, ((n_chunks - 1) / kTPBufs) & 1);
-    if (have) tc::fence_after_sync();
-    float inv[2], lse2[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const float lr = have ? l[r] : 0.f;
-      inv[r] = (lr > 0.f) ? 1.f / lr : 0.f;
-      lse2[r] = (lr > 0.f) ? (m[r] + hw_log2(lr)) : -INFINITY;
-    }
-    for (int cb = 0; cb < kD / 64; ++cb) {
-      uint32_t o[32];
-      if (have) {
-        tc::ld_16x256b_x8(tmem + lane_base + 128 + cb * 64, o);
-        tc::wait_ld();
-      } else {
-#pragma unroll
-        for (int x = 0; x < 32; ++x) o[x] = 0u;
-      }
-      if (row_ok) {
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const size_t rh = (size_t)(r0 + j) * kHeads + g * kHpg + (r ? h1 : h0);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int d = cb * 64 + 8 * i + cq;
-            const float o0 = __uint_as_float(o[4 * i + 2 * r]) * inv[r];
-            const float o1 = __uint_as_float(o[4 * i + 2 * r + 1]) * inv[r];
-            if (a.n_split == 1) {
-              *reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(a.out) + rh * kD + d) = pack_bf16(o0, o1);
-            } else {
-              *reinterpret_cast<float2 *>(a.part_o + (rh * a.n_split + p) * kD + d) = make_float2(o0, o1);
+      ++mi;
+      if (*is_last) {
+        __threadfence();
+        const int mm = tid >> 1, dh = (tid & 1) * 96;
+        const int jj = mm >> 4, hh = mm & 15;
+        if (jj < it.nr) {
+          const size_t rh2 = (size_t)(it.r0 + jj) * kHeads + it.g * kHpg + hh;
+          float w[kMaxTileSplit];
+          float lse;
+          tile_partition_weights(a.part_lse + rh2 * a.n_split, a.n_split, w, lse);
+          __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(a.out) + rh2 * kD + dh;
+          for (int x = 0; x < 96; x += 4) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int q = 0; q < a.n_split; ++q) {
+              const float4 pv = ld_cg(reinterpret_cast<const float4 *>(a.part_o + (rh2 * a.n_split + q) * kD + dh + x));
+              acc.x = fmaf(w[q], pv.x, acc.x);
+              acc.y = fmaf(w[q], pv.y, acc.y);
+              acc.z = fmaf(w[q], pv.z, acc.z);
+              acc.w = fmaf(w[q], pv.w, acc.w);
             }
+            uint2 w2;
+            w2.x = pack_bf16(acc.x, acc.y);
+            w2.y = pack_bf16(acc.z, acc.w);
+            *reinterpret_cast<uint2 *>(out + x) = w2;
           }
-        }
-      }
-    }
-    if (row_ok && (lane & 3) == 0) {
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const size_t rh = (size_t)(r0 + j) * kHeads + g * kHpg + (r ? h1 : h0);
-        if (a.n_split == 1) {
-          if (a.lse != nullptr) a.lse[rh] = lse2[r] * 0.69314718055994531f;
-        } else {
-          a.part_lse[rh * a.n_split + p] = lse2[r];
+          if ((tid & 1) == 0 && a.lse != nullptr) a.lse[rh2] = lse;
         }
       }
     }
   }
+
   // ---- teardown: no MMA may be writing tensor memory when it is released ----
-  if (warp == 0 && n_chunks > 0) mbar_wait_bounded(bar_final, 0, kTWaitNs);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (warp == 0) tc::tmem_dealloc(tmem, kTTmemCols);
-  if (a.n_split == 1 || a.merge_cnt == nullptr) return;
-
-  // ---- the last partition CTA of (tile, group) merges every partition ----
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const uint32_t prev = atomicAdd(a.merge_cnt + (size_t)tile * kKv + g, 1u);
-    *is_last = (prev == (uint32_t)a.n_split - 1);
+  if (warp == 0) {
+    mbar_wait_bounded(bars + kBFinal, 0, kTWaitNs);
+    tc::tmem_dealloc(tmem, kTTmemCols);
   }
-  __syncthreads();
-  if (!*is_last) return;
-  __threadfence();
-  if (tid < kTM) {
-    const int jj = tid / kHpg, hh = tid % kHpg;
-    if (jj < nr) {
-      const size_t rh = (size_t)(r0 + jj) * kHeads + g * kHpg + hh;
-      float w[kMaxTileSplit];
-      float lse;
-      tile_partition_weights(a.part_lse + rh * a.n_split, a.n_split, w, lse);
-      __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(a.out) + rh * kD;
-      for (int x = 0; x < kD; x += 4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q = 0; q < a.n_split; ++q) {
-          const float4 v = ld_cg(reinterpret_cast<const float4 *>(a.part_o + (rh * a.n_split + q) * kD + x));
-          acc.x = fmaf(w[q], v.x, acc.x);
-          acc.y = fmaf(w[q], v.y, acc.y);
-          acc.z = fmaf(w[q], v.z, acc.z);
-          acc.w = fmaf(w[q], v.w, acc.w);
-        }
-        uint2 w2;
-        w2.x = pack_bf16(acc.x, acc.y);
-        w2.y = pack_bf16(acc.z, acc.w);
-        *reinterpret_cast<uint2 *>(out + x) = w2;
-      }
-      if (a.lse != nullptr) a.lse[rh] = lse;
-    }
-  }
-  if (tid == 0) a.merge_cnt[(size_t)tile * kKv + g] = 0u;
 }
 
-constexpr int kTileSmem = kTQBytes + kTStages * kTStageBytes + kTPBufs * kTPBytes + 2 * kMaxTileEntries * 4 + 256 + 1024;
-
 cudaError_t launch_tile_union(const TileArgs &a, int batch, cudaStream_t st) {
-  const size_t smem = (size_t)kTRows * a.bitmap_words * sizeof(uint32_t);
+  const size_t smem = (size_t)a.map_words * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(tile_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   tile_union_kernel<<<dim3(a.tiles_per_seq, batch), 256, smem, st>>>(a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gqa_tile(const TileArgs &a, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+cudaError_t launch_gqa_tile(const TileArgs &a, const CUtensorMap &tk, const CUtensorMap &tv, int n_ctas,
                             cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(gqa_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileSmem);
   if (e != cudaSuccess) return e;
-  const long long n_cta = (long long)a.n_split * a.n_tiles * kKv;
-  if (n_cta > 0x7fffffffLL) return cudaErrorInvalidValue;
-  gqa_tile_kernel<<<(unsigned)n_cta, kTThreads, kTileSmem, st>>>(a, tq, tk, tv);
+  const long long n_items = (long long)a.n_split * a.n_tiles * kKv;  // upper bound: every tile shared-set
+  if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const int grid = (int)(n_items < n_ctas ? n_items : n_ctas);
+  if (grid < 1) return cudaSuccess;
+  gqa_tile_kernel<<<grid, kTThreads, kTileSmem, st>>>(a, tk, tv);
   return cudaGetLastError();
 }
 

@@ -99,8 +99,9 @@ struct GemmArgs {
 };
 
 // Multi-row tiles (verify / prefill): shared-set attention on the tensor cores.
-constexpr int kMaxTileEntries = 2056;  // blocks one tile CTA may own (>= 4 x 512 + 4, multiple of 8)
+constexpr int kTileRows = 8;           // query rows per shared-set tile (8 rows x 16 heads = M 128)
 constexpr int kMaxTileSplit = 32;
+constexpr int kUnionMapWords = 49152;  // shared byte map of the union kernel: blocks < 196,608
 
 struct TileArgs {
   const void *q;
@@ -115,10 +116,10 @@ struct TileArgs {
   int total_q;
   int num_pages;
   float scale_log2;
-  int tiles_per_seq;   // ceil(max_q / 4)
+  int tiles_per_seq;   // ceil(max_q / kTileRows)
   int n_tiles;         // batch * tiles_per_seq
   int n_split;         // partitions of a tile's block list
-  int bitmap_words;    // 32-bit words per row bitmap in the union kernel
+  int map_words;       // 32-bit words of the union kernel's byte map (one byte per block)
   int union_cap;       // entries per tile in the union lists
   int *union_count;    // [n_tiles]
   uint32_t *union_ent; // [n_tiles][union_cap]
@@ -134,7 +135,7 @@ struct TileArgs {
 };
 
 cudaError_t launch_tile_union(const TileArgs &a, int batch, cudaStream_t st);
-cudaError_t launch_gqa_tile(const TileArgs &a, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+cudaError_t launch_gqa_tile(const TileArgs &a, const CUtensorMap &tk, const CUtensorMap &tv, int n_ctas,
                             cudaStream_t st);
 
 cudaError_t launch_index_score(const IndexScoreArgs &a, int max_q, int grid_pages, int n_seq, cudaStream_t st);
