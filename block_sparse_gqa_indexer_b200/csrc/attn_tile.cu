@@ -24,11 +24,12 @@
 //                       tensor-memory buffers and warp 11 O += P V, both with
 //                       their A operand (Q, P) in tensor memory (two issuing
 //                       threads, so S of a later chunk never waits behind the
-//                       PV of an earlier one); warps 0-7 load Q into
-//                       tensor memory, run the masked online softmax (two
-//                       warps per 32 rows, one per half of the chunk's
-//                       columns), write P back to tensor memory as bf16 and
-//                       finish each item.
+//                       PV of an earlier one); warps 0-15 load Q into
+//                       tensor memory, run the masked online softmax (four
+//                       warps per 32 rows, one per quarter of the chunk's
+//                       columns, row maxima exchanged through shared memory),
+//                       write P back to tensor memory as bf16 and finish each
+//                       item.
 //
 // Each shared block is read once per tile instead of once per row; the
 // masked-out products are the price of dense tiles.
@@ -46,10 +47,15 @@ constexpr int kTChunkBlocks = 8;           // blocks per chunk
 constexpr int kTN = kTChunkBlocks * kBlk;  // 64 tokens per chunk
 constexpr int kTStages = 4;                // depth of the K ring and of the V ring
 constexpr int kTKvBytes = kTChunkBlocks * kBlockBytes;  // K (or V) of one chunk
-constexpr int kTSoftWarps = 8;
+constexpr int kTSoftWarps = 16;                // softmax / epilogue warps
 constexpr int kTSoftThreads = kTSoftWarps * 32;
-constexpr int kTWarpK = 8, kTWarpV = 9, kTWarpS = 10, kTWarpPv = 11;
-constexpr int kTThreads = 12 * 32;
+constexpr int kTSplit = kTSoftWarps / 4;        // warps per tensor-memory lane quarter
+constexpr int kTCols = kTN / kTSplit;           // S columns per softmax warp (16)
+constexpr int kTBlocksW = kTCols / kBlk;        // blocks per softmax warp and chunk (2)
+constexpr int kTOCols = kD / kTSplit;           // O columns (= Q dims) per softmax warp (48)
+constexpr int kTWarpK = kTSoftWarps, kTWarpV = kTSoftWarps + 1, kTWarpS = kTSoftWarps + 2,
+              kTWarpPv = kTSoftWarps + 3;
+constexpr int kTThreads = (kTSoftWarps + 4) * 32;
 constexpr uint32_t kTTmemCols = 512;
 constexpr uint32_t kTmemS = 0;    // 2 x 64 columns: S of chunk gc in buffer gc % 2
 constexpr uint32_t kTmemP = 128;  // 2 x 32 columns: bf16 P of chunk gc in buffer gc % 2
@@ -61,12 +67,12 @@ constexpr float kLazyRescale = 8.0f;  // log2 units
 // shared memory (offsets from a 1,024-byte aligned base)
 constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kTStages * kTKvBytes;
-constexpr int kOffXm = kOffV + kTStages * kTKvBytes;  // float [2 buffers][2 halves][128 rows]
-constexpr int kOffXl = kOffXm + 2 * 2 * kTM * 4;      // float [2 halves][128 rows]
-constexpr int kOffBar = kOffXl + 2 * kTM * 4;
+constexpr int kOffXm = kOffV + kTStages * kTKvBytes;  // float [2 buffers][kTSplit][128 rows]
+constexpr int kOffXl = kOffXm + 2 * kTSplit * kTM * 4;  // float [kTSplit][128 rows]
+constexpr int kOffBar = kOffXl + kTSplit * kTM * 4;
 constexpr int kNumBars = 44;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kOffList = kOffMisc + 64;            // int [kMaxListTiles]: shared-set tiles, ascending
+constexpr int kOffList = kOffMisc + 128;           // int [kMaxListTiles]: shared-set tiles, ascending
 constexpr int kMaxListTiles = 4096;
 constexpr int kTileSmem = kOffList + kMaxListTiles * 4 + 1024;  // + alignment slack
 
@@ -230,16 +236,6 @@ __device__ __forceinline__ TileItem decode_item(const TileArgs &a, const int *li
   return it;
 }
 
-// TMA row of a union entry in group it.g of the paged pool, or -1 (recorded).
-__device__ __forceinline__ int entry_row(const TileArgs &a, const TileItem &it, uint32_t e) {
-  const int b = (int)(e & 0xFFFFFFu);
-  const int pg = b / kBpp;
-  const int ph = (pg < a.max_pages) ? ld_cg(a.page_table + (size_t)it.s * a.max_pages + pg) : -1;
-  if (ph >= 0 && ph < a.num_pages) return ((ph * kKv + it.g) * kPage) + (b % kBpp) * kBlk;
-  record_error(a.err, S5_ERR_DEVICE_BOUNDS, it.r0);
-  return -1;
-}
-
 // Merge weights of the partitions of one (row, head): the same arithmetic as
 // the per-row kernel's merge, in partition order.
 __device__ __forceinline__ void tile_partition_weights(const float *pl, int n, float *w, float &lse_nat) {
@@ -273,7 +269,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
   int *is_last = reinterpret_cast<int *>(smem + kOffMisc + 8);
 
   int *list_s = reinterpret_cast<int *>(smem + kOffList);
-  int *wsum = reinterpret_cast<int *>(smem + kOffMisc + 16);  // [11] per-warp counts
+  int *wsum = reinterpret_cast<int *>(smem + kOffMisc + 16);  // [kTThreads / 32] per-warp counts
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -323,8 +319,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
       mbar_init(bars + kBPFree + i, 1);
     }
     mbar_init(bars + kBOEmpty, kTSoftWarps);
-    for (int i = 0; i < 8; ++i) mbar_init(bars + kBXm + i, 64);
-    for (int i = 0; i < 4; ++i) mbar_init(bars + kBXl + i, 64);
+    for (int i = 0; i < 8; ++i) mbar_init(bars + kBXm + i, 32 * kTSplit);
+    for (int i = 0; i < 4; ++i) mbar_init(bars + kBXl + i, 32 * kTSplit);
     mbar_init(bars + kBMgAll, kTSoftThreads);
     mbar_init(bars + kBMgDec, 1);
     mbar_init(bars + kBFinal, 2);  // one commit from each MMA issuer
@@ -361,7 +357,23 @@ __global__ void __launch_bounds__(kTThreads, 1)
       const TileItem it = decode_item(a, list, n_list, idx);
       if (it.n_chunks == 0) continue;
       const uint32_t *ent = a.union_ent + (size_t)it.tile * a.union_cap + it.e0;
+      const int32_t *pt = a.page_table + (size_t)it.s * a.max_pages;
+      // lookups run two chunks ahead of the copies: the entry of chunk c + 2
+      // and the page of chunk c + 1 are in flight while chunk c is issued
+      auto load_block = [&](int c) -> int {  // this lane's block of chunk c, or -1
+        const int i = c * kTChunkBlocks + lane;
+        return (lane < kTChunkBlocks && c < it.n_chunks && i < it.ne) ? (int)(ld_cg(ent + i) & 0xFFFFFFu) : -1;
+      };
+      auto load_page = [&](int b) -> int {  // physical page of block b (-1: none or unmapped)
+        const int pg = b / kBpp;
+        return (b >= 0 && pg < a.max_pages) ? ld_cg(pt + pg) : -1;
+      };
+      int b0 = load_block(0);
+      int ph0 = load_page(b0);
+      int b1 = load_block(1);
       for (int c = 0; c < it.n_chunks; ++c, ++gc) {
+        const int b2 = load_block(c + 2);
+        const int ph1 = load_page(b1);
         const int st = gc % kTStages;
         int go = 1;
         if (lane == 0 && gc >= kTStages) go = wait(empty + st, ((gc / kTStages) - 1) & 1) ? 1 : 0;
@@ -369,8 +381,14 @@ __global__ void __launch_bounds__(kTThreads, 1)
           ok = false;
           break;
         }
-        const int i = c * kTChunkBlocks + lane;
-        const int row = (lane < kTChunkBlocks && i < it.ne) ? entry_row(a, it, ld_cg(ent + i)) : -1;
+        int row = -1;
+        if (b0 >= 0) {
+          if (ph0 >= 0 && ph0 < a.num_pages) row = ((ph0 * kKv + it.g) * kPage) + (b0 % kBpp) * kBlk;
+          else record_error(a.err, S5_ERR_DEVICE_BOUNDS, it.r0);
+        }
+        b0 = b1;
+        ph0 = ph1;
+        b1 = b2;
         uint32_t bytes = (row >= 0) ? (uint32_t)kBlockBytes : 0u;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, off);
@@ -457,10 +475,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
       tc::commit(bars + kBFinal);
     }
   } else {
-    // ---------------- softmax / epilogue: warps 0-7 ----------------
+    // ---------------- softmax / epilogue: warps 0-15 ----------------
     // Warp w reads lanes 32 (w % 4) .. + 31 (tile rows m = lane index: query
-    // j = m / 16, head h = m % 16) and columns 32 (w / 4) .. + 31 of each S.
-    const int q4 = warp & 3, half = warp >> 2;
+    // j = m / 16, head h = m % 16) and columns 16 (w / 4) .. + 15 of each S
+    // (blocks 2 (w / 4), + 1 of the chunk); it owns Q dims and O columns
+    // 48 (w / 4) .. + 47 of its rows.
+    const int q4 = warp & 3, qq = warp >> 2;
     const int m = q4 * 32 + lane;
     const int j = m >> 4, h = m & 15;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
@@ -478,44 +498,35 @@ __global__ void __launch_bounds__(kTThreads, 1)
       float m_ref = -INFINITY, l = 0.f;
       if (it.n_chunks > 0) {
         // Q of the item into tensor memory: this thread's row (query j, head
-        // 16g + h), dims 96 half .. + 95 (zeros past the tile's rows); the
-        // previous item's last S must be done with the old Q
+        // 16g + h), its 48 dims (zeros past the tile's rows); the previous
+        // item's last S must be done with the old Q
         if (qi > 0 && !wait(bars + kBQEmpty, (qi - 1) & 1)) {
           ok = false;
           break;
         }
-        uint32_t qv[48];
         const uint4 *qs = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.q) +
                                                           ((size_t)(it.r0 + j) * kHeads + it.g * kHpg + h) * kD +
-                                                          half * 96);
+                                                          qq * kTOCols);
 #pragma unroll
-        for (int x = 0; x < 12; ++x) {
-          const uint4 u = row_ok ? ld_cg(qs + x) : make_uint4(0, 0, 0, 0);
-          qv[4 * x] = u.x;
-          qv[4 * x + 1] = u.y;
-          qv[4 * x + 2] = u.z;
-          qv[4 * x + 3] = u.w;
-        }
-#pragma unroll
-        for (int x = 0; x < 3; ++x) {
-          uint32_t w16[16];
-#pragma unroll
-          for (int y = 0; y < 16; ++y) w16[y] = qv[16 * x + y];
-          tc::st_16cols(tmem + lane_base + kTmemQ + half * 48 + x * 16, w16);
+        for (int x = 0; x < kTOCols / 16; ++x) {  // 16 dims = 8 columns per store
+          const uint4 u0 = row_ok ? ld_cg(qs + 2 * x) : make_uint4(0, 0, 0, 0);
+          const uint4 u1 = row_ok ? ld_cg(qs + 2 * x + 1) : make_uint4(0, 0, 0, 0);
+          const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+          tc::st_8cols(tmem + lane_base + kTmemQ + qq * (kTOCols / 2) + x * 8, w8);
         }
         tc::wait_st();
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + kBQFull);
       }
-      // lanes 0..3 hold the entries of this half's 4 blocks of the next chunk
+      // lanes 0..1 hold the entries of this warp's 2 blocks of the next chunk
       uint32_t e_next = 0u;
-      if (lane < 4 && half * 4 + lane < it.ne) e_next = ld_cg(ent + half * 4 + lane);
+      if (lane < kTBlocksW && qq * kTBlocksW + lane < it.ne) e_next = ld_cg(ent + qq * kTBlocksW + lane);
       for (int c = 0; c < it.n_chunks; ++c, ++gc) {
         const uint32_t e_cur = e_next;
         {
-          const int i = (c + 1) * kTChunkBlocks + half * 4 + lane;
-          e_next = (lane < 4 && c + 1 < it.n_chunks && i < it.ne) ? ld_cg(ent + i) : 0u;
+          const int i = (c + 1) * kTChunkBlocks + qq * kTBlocksW + lane;
+          e_next = (lane < kTBlocksW && c + 1 < it.n_chunks && i < it.ne) ? ld_cg(ent + i) : 0u;
         }
         const int sb = gc & 1;
         if (!wait(bars + kBSFull + sb, (gc >> 1) & 1)) {
@@ -523,19 +534,19 @@ __global__ void __launch_bounds__(kTThreads, 1)
           break;
         }
         tc::fence_after_sync();
-        uint32_t v[32];
-        tc::ld_32cols(tmem + lane_base + kTmemS + sb * kTN + half * 32, v);
+        uint32_t v[kTCols];
+        tc::ld_16cols(tmem + lane_base + kTmemS + sb * kTN + qq * kTCols, v);
         tc::wait_ld();
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + kBSEmpty + sb);
-        // mask: column x = 8 ib + tok is token tok of block (4 half + ib) of the chunk
-        float sc[32];  // scaled, masked scores
+        // mask: column x = 8 ib + tok is token tok of block (2 qq + ib) of the chunk
+        float sc[kTCols];  // scaled, masked scores
         float mx = -INFINITY;
 #pragma unroll
-        for (int ib = 0; ib < 4; ++ib) {
+        for (int ib = 0; ib < kTBlocksW; ++ib) {
           const uint32_t e = __shfl_sync(0xffffffffu, e_cur, ib);
-          const bool valid = row_ok && (c * kTChunkBlocks + half * 4 + ib < it.ne);
+          const bool valid = row_ok && (c * kTChunkBlocks + qq * kTBlocksW + ib < it.ne);
           const int blk = (int)(e & 0xFFFFFFu);
           const bool sel = valid && ((e >> (24 + j)) & 1u);
           const int lim = sel ? kBlk - 1 : ((valid && blk == cj) ? t - blk * kBlk : -1);  // tokens 0..lim visible
@@ -546,15 +557,17 @@ __global__ void __launch_bounds__(kTThreads, 1)
             mx = fmaxf(mx, s);
           }
         }
-        // row max over both halves
-        float *xmb = xm + sb * 2 * kTM;
-        xmb[half * kTM + m] = mx;
+        // row max over the four column quarters
+        float *xmb = xm + sb * kTSplit * kTM;
+        xmb[qq * kTM + m] = mx;
         mbar_arrive(bars + kBXm + q4 * 2 + sb);
         if (!wait(bars + kBXm + q4 * 2 + sb, (gc >> 1) & 1)) {
           ok = false;
           break;
         }
-        const float rmax = fmaxf(mx, xmb[(1 - half) * kTM + m]);
+        float rmax = mx;
+#pragma unroll
+        for (int o = 1; o < kTSplit; ++o) rmax = fmaxf(rmax, xmb[((qq + o) % kTSplit) * kTM + m]);
         // lazy rescale: keep the reference max unless the row max grows by more than 2^8
         const bool grow = rmax > m_ref + kLazyRescale;
         const bool resc = grow && m_ref != -INFINITY;
@@ -568,14 +581,14 @@ __global__ void __launch_bounds__(kTThreads, 1)
           }
           tc::fence_after_sync();
 #pragma unroll 1
-          for (int cb = 0; cb < 3; ++cb) {
-            uint32_t o[32];
-            const uint32_t ta = tmem + lane_base + kTmemO + half * 96 + cb * 32;
-            tc::ld_32cols(ta, o);
+          for (int cb = 0; cb < kTOCols / 16; ++cb) {
+            uint32_t o[16];
+            const uint32_t ta = tmem + lane_base + kTmemO + qq * kTOCols + cb * 16;
+            tc::ld_16cols(ta, o);
             tc::wait_ld();
 #pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * corr);
-            tc::st_32cols(ta, o);
+            for (int x = 0; x < 16; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * corr);
+            tc::st_16cols(ta, o);
           }
           tc::wait_st();
         }
@@ -586,21 +599,21 @@ __global__ void __launch_bounds__(kTThreads, 1)
           break;
         }
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-        uint32_t pk[16];
+        uint32_t pk[kTCols / 2];
         float ps = 0.f;
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
+        for (int x = 0; x < kTCols / 2; ++x) {
           const float p0 = hw_exp2(sc[2 * x] - mu);
           const float p1 = hw_exp2(sc[2 * x + 1] - mu);
           ps += p0 + p1;
           pk[x] = pack_bf16(p0, p1);
         }
         l += ps;
-        tc::st_16cols(tmem + lane_base + kTmemP + sb * 32 + half * 16, pk);
+        tc::st_8cols(tmem + lane_base + kTmemP + sb * 32 + qq * (kTCols / 2), pk);
         // V rows no row may read (padding slots, tokens past the tile's last
         // position, all in the item's last chunk) must be finite: zero them
-        // (P is 0 there, but 0 * NaN is NaN).  Warp w checks block w.
-        if (c == it.n_chunks - 1) {
+        // (P is 0 there, but 0 * NaN is NaN).  Warp w < 8 checks block w.
+        if (c == it.n_chunks - 1 && warp < kTChunkBlocks) {
           const int ir = c * kTChunkBlocks + warp;
           const int blk = (ir < it.ne) ? (int)(ld_cg(ent + ir) & 0xFFFFFFu) : -1;
           const int first_bad = (blk < 0) ? 0 : t_max - blk * kBlk + 1;  // tokens >= first_bad are zeroed
@@ -628,13 +641,14 @@ __global__ void __launch_bounds__(kTThreads, 1)
       float lt = 0.f;
       const bool have = it.n_chunks > 0;
       if (have) {
-        xl[half * kTM + m] = l;
+        xl[qq * kTM + m] = l;
         mbar_arrive(bars + kBXl + q4);
         if (!wait(bars + kBXl + q4, qi & 1)) {
           ok = false;
           break;
         }
-        lt = l + xl[(1 - half) * kTM + m];
+#pragma unroll
+        for (int o = 0; o < kTSplit; ++o) lt += xl[o * kTM + m];
         if (!wait(bars + kBPFree + ((gc - 1) & 1), ((gc - 1) >> 1) & 1)) {
           ok = false;
           break;
@@ -645,21 +659,21 @@ __global__ void __launch_bounds__(kTThreads, 1)
       const float lse2 = (lt > 0.f) ? m_ref + hw_log2(lt) : -INFINITY;
       const size_t rh = (size_t)(it.r0 + j) * kHeads + it.g * kHpg + h;
 #pragma unroll 1
-      for (int cb = 0; cb < 3; ++cb) {
-        uint32_t o[32];
+      for (int cb = 0; cb < kTOCols / 16; ++cb) {
+        uint32_t o[16];
         if (have) {
-          tc::ld_32cols(tmem + lane_base + kTmemO + half * 96 + cb * 32, o);
+          tc::ld_16cols(tmem + lane_base + kTmemO + qq * kTOCols + cb * 16, o);
           tc::wait_ld();
         } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] = 0u;
+          for (int x = 0; x < 16; ++x) o[x] = 0u;
         }
         if (row_ok) {
-          const int d0 = half * 96 + cb * 32;
+          const int d0 = qq * kTOCols + cb * 16;
           if (a.n_split == 1) {
             uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(a.out) + rh * kD + d0);
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
+            for (int x = 0; x < 2; ++x)
               dst[x] = make_uint4(pack_bf16(__uint_as_float(o[8 * x]) * inv, __uint_as_float(o[8 * x + 1]) * inv),
                                   pack_bf16(__uint_as_float(o[8 * x + 2]) * inv, __uint_as_float(o[8 * x + 3]) * inv),
                                   pack_bf16(__uint_as_float(o[8 * x + 4]) * inv, __uint_as_float(o[8 * x + 5]) * inv),
@@ -667,7 +681,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
           } else {
             float4 *dst = reinterpret_cast<float4 *>(a.part_o + (rh * a.n_split + it.p) * kD + d0);
 #pragma unroll
-            for (int x = 0; x < 8; ++x)
+            for (int x = 0; x < 4; ++x)
               dst[x] = make_float4(__uint_as_float(o[4 * x]) * inv, __uint_as_float(o[4 * x + 1]) * inv,
                                    __uint_as_float(o[4 * x + 2]) * inv, __uint_as_float(o[4 * x + 3]) * inv);
           }
@@ -679,7 +693,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
         if (lane == 0) mbar_arrive(bars + kBOEmpty);
         ++qi;
       }
-      if (row_ok && half == 0) {
+      if (row_ok && qq == 0) {
         if (a.n_split == 1) {
           if (a.lse != nullptr) a.lse[rh] = lse2 * 0.69314718055994531f;
         } else {
@@ -708,7 +722,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
       ++mi;
       if (*is_last) {
         __threadfence();
-        const int mm = tid >> 1, dh = (tid & 1) * 96;
+        const int mm = tid / kTSplit, dh = (tid % kTSplit) * kTOCols;
         const int jj = mm >> 4, hh = mm & 15;
         if (jj < it.nr) {
           const size_t rh2 = (size_t)(it.r0 + jj) * kHeads + it.g * kHpg + hh;
@@ -716,7 +730,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
           float lse;
           tile_partition_weights(a.part_lse + rh2 * a.n_split, a.n_split, w, lse);
           __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(a.out) + rh2 * kD + dh;
-          for (int x = 0; x < 96; x += 4) {
+          for (int x = 0; x < kTOCols; x += 4) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int q = 0; q < a.n_split; ++q) {
               const float4 pv = ld_cg(reinterpret_cast<const float4 *>(a.part_o + (rh2 * a.n_split + q) * kD + dh + x));
@@ -730,7 +744,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
             w2.y = pack_bf16(acc.z, acc.w);
             *reinterpret_cast<uint2 *>(out + x) = w2;
           }
-          if ((tid & 1) == 0 && a.lse != nullptr) a.lse[rh2] = lse;
+          if ((tid % kTSplit) == 0 && a.lse != nullptr) a.lse[rh2] = lse;
         }
       }
     }
