@@ -93,11 +93,11 @@ static_assert(kBFinal < kNumBars, "barrier slots");
 // Entry: block (bits 0..23) | rows that selected it << 24 (bit j = row j).
 __global__ void __launch_bounds__(256) tile_union_kernel(const TileArgs a) {
   extern __shared__ uint32_t bmap[];  // byte b: rows that selected block b
-  __shared__ int cur_blk[kTRows];
   __shared__ int scan[8];
   const int s = blockIdx.y, k = blockIdx.x;
   const int tile = s * a.tiles_per_seq + k;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();  // (programmatic launch) the selection is read after this point
   const int q_beg = ld_cg(a.cu_q + s);
   const int nq = ld_cg(a.cu_q + s + 1) - q_beg;
   const int ctx = ld_cg(a.ctx_lens + s);
@@ -128,7 +128,6 @@ __global__ void __launch_bounds__(256) tile_union_kernel(const TileArgs a) {
     return;
   }
   for (int i = tid; i < words; i += 256) bmap[i] = 0;
-  if (tid < kTRows) cur_blk[tid] = (tid < nr) ? (ctx + k * kTRows + tid) / kBlk : -1;
   __syncthreads();
   int row_blocks = 0;  // sum over the tile's rows of (selected blocks + current block)
   for (int j = 0; j < nr; ++j) {
@@ -147,13 +146,11 @@ __global__ void __launch_bounds__(256) tile_union_kernel(const TileArgs a) {
     }
   }
   __syncthreads();
-  // ascending compaction of the selected blocks and the current blocks
-  auto in_union = [&](int b, uint32_t byte) {
-    if (byte != 0) return true;
-    for (int j = 0; j < nr; ++j)
-      if (cur_blk[j] == b) return true;
-    return false;
-  };
+  // ascending compaction of the selected blocks and the current blocks (the
+  // rows' positions are consecutive, so their current blocks are exactly
+  // c_first .. c_last)
+  const int c_first = (ctx + k * kTRows) / kBlk;
+  auto in_union = [&](int b, uint32_t byte) { return byte != 0 || (b >= c_first && b <= c_last); };
   const int per = (words + 255) / 256;  // words per thread, in order
   const int w_lo = min(words, tid * per), w_hi = min(words, tid * per + per);
   int cnt = 0;
@@ -272,6 +269,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
   int *wsum = reinterpret_cast<int *>(smem + kOffMisc + 16);  // [kTThreads / 32] per-warp counts
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_wait();  // (programmatic launch) the union kernel's outputs are read after this point
 
   // ---- the shared-set tiles, in order (most batches of independent queries have none) ----
   const int *list = nullptr;
@@ -760,12 +758,28 @@ __global__ void __launch_bounds__(kTThreads, 1)
   }
 }
 
+// Programmatic stream serialization: a kernel's launch overlaps the end of the
+// previous one; every global read of these kernels follows pdl_wait().
+template <typename K>
+cudaError_t launch_after(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, const TileArgs &a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
 cudaError_t launch_tile_union(const TileArgs &a, int batch, cudaStream_t st) {
   const size_t smem = (size_t)a.map_words * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(tile_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  tile_union_kernel<<<dim3(a.tiles_per_seq, batch), 256, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_after(tile_union_kernel, dim3(a.tiles_per_seq, batch), dim3(256), smem, st, a);
 }
 
 cudaError_t launch_gqa_tile(const TileArgs &a, const CUtensorMap &tk, const CUtensorMap &tv, int n_ctas,
@@ -776,8 +790,17 @@ cudaError_t launch_gqa_tile(const TileArgs &a, const CUtensorMap &tk, const CUte
   if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;
   const int grid = (int)(n_items < n_ctas ? n_items : n_ctas);
   if (grid < 1) return cudaSuccess;
-  gqa_tile_kernel<<<grid, kTThreads, kTileSmem, st>>>(a, tk, tv);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kTThreads);
+  cfg.dynamicSmemBytes = kTileSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gqa_tile_kernel, a, tk, tv);
 }
 
 }  // namespace s5

@@ -324,39 +324,10 @@ __device__ __forceinline__ void write_all(int32_t *out, int n, int topk, int nt)
   for (int i = threadIdx.x; i < topk; i += nt) out[i] = (i < n) ? i : -1;
 }
 
-// Single stage: one CTA per query row (rows of up to NT * EMAX blocks).
-template <int NT, int EMAX>
-__global__ void __launch_bounds__(NT) topk_select_kernel(SelectArgs a) {
-  __shared__ SelectSmem<NT> sm;
-  const int r = blockIdx.x;
-  int32_t *out = a.sel + (size_t)r * a.topk;
-  pdl_trigger();
-  pdl_wait();
-  int c = 0;
-  const bool row_ok = row_history(a, r, c) && c <= NT * EMAX;
-  if (!row_ok) {
-    if (threadIdx.x == 0) {
-      record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
-      a.sel_count[r] = 0;
-    }
-    write_all(out, 0, a.topk, NT);
-    return;
-  }
-  if (c <= a.topk) {
-    write_all(out, c, a.topk, NT);
-    if (threadIdx.x == 0) a.sel_count[r] = c;
-    return;
-  }
-  const int E = owned_per_thread<NT>(c);
-  uint32_t key[EMAX];
-  load_keys<NT, EMAX>(a.scores + (size_t)r * a.score_stride, c, E, key);
-  cta_select<NT, EMAX>(key, c, E, a.topk, sm, [&](int pos, int i, uint32_t) { out[pos] = i; });
-  if (threadIdx.x == 0) a.sel_count[r] = a.topk;
-}
-
 constexpr int kWarpRefine = 2048;  // threshold bins up to this size are refined by one warp
 
 struct HistSmem {
+  uint32_t h1[kHistBins];       // row histogram of the top 12 key bits, when not given
   uint32_t h2[1024];            // block-wide refinement of a large threshold bin
   uint32_t cand[kWarpRefine];   // keys of the threshold bin (any order)
   int scan_a[32];
@@ -396,7 +367,8 @@ __device__ __forceinline__ void find_bin_desc(const uint32_t (&c)[NB], int top, 
 }
 
 // Single stage from a row histogram of the top 12 key bits (built while the
-// scores were produced).  The histogram gives the threshold bin; its keys are
+// scores were produced, or here in shared memory from the keys when a.hist is
+// null).  The histogram gives the threshold bin; its keys are
 // then resolved either by one warp (a bit-by-bit search over the remaining 20
 // bits, when the bin holds at most kWarpRefine keys and WARP_REFINE is set) or
 // by two more block-wide radix passes of 10 bits.
@@ -416,7 +388,7 @@ __global__ void __launch_bounds__(NT) topk_select_hist_kernel(SelectArgs a) {
   const bool row_ok = row_history(a, r, c) && c <= NT * EMAX;
   // this thread's row-histogram bins, top first: 4095 - NB1*t .. (loaded with the keys)
   uint32_t cc1[NB1];
-  {
+  if (a.hist != nullptr) {
     const uint4 *h4 = reinterpret_cast<const uint4 *>(a.hist + (size_t)r * kHistBins);
 #pragma unroll
     for (int q = 0; q < NB1 / 4; ++q) {
@@ -445,6 +417,17 @@ __global__ void __launch_bounds__(NT) topk_select_hist_kernel(SelectArgs a) {
   const int mine = max(0, min(E, c - first));
   uint32_t key[EMAX];
   load_keys<NT, EMAX>(a.scores + (size_t)r * a.score_stride, c, E, key);
+  if (a.hist == nullptr) {
+#pragma unroll
+    for (int i = 0; i < kHistBins / NT; ++i) sm.h1[tid + i * NT] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < EMAX; ++j)
+      if (j < mine) atomicAdd(&sm.h1[key[j] >> 20], 1u);
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < NB1; ++i) cc1[i] = sm.h1[kHistBins - 1 - NB1 * tid - i];
+  }
   if (tid == 0) sm.ncand = 0;
   find_bin_desc<NT, NB1>(cc1, kHistBins - 1, a.topk, sm);
   int kk = a.topk - (int)sm.above;
@@ -628,11 +611,8 @@ cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, cudaStrea
 }
 
 cudaError_t launch_topk_select(const SelectArgs &a, int total_q, bool two_stage, cudaStream_t st) {
-  if (!two_stage) {
-    if (a.hist != nullptr)
-      return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false>, dim3(total_q), dim3(kSelThreads), st, a);
-    return launch_pdl(topk_select_kernel<kSelThreads, 16>, dim3(total_q), dim3(kSelThreads), st, a);
-  }
+  if (!two_stage)  // with a row histogram from the scoring kernel, or one built in shared memory
+    return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false>, dim3(total_q), dim3(kSelThreads), st, a);
   cudaError_t e = launch_pdl(topk_segment_kernel<kSegThreads, 32>, dim3(a.n_seg, total_q), dim3(kSegThreads), st, a);
   if (e != cudaSuccess) return e;
   if (a.n_seg * a.topk <= 512 * 16) return launch_pdl(topk_merge_kernel<512, 16>, dim3(total_q), dim3(512), st, a);
