@@ -94,3 +94,26 @@ def test_bad_descriptors_rejected_before_launch(s5):
                                        None) == s5.S5_ERR_INVALID_ARG
     assert s5._lib.s5_index_score_topk(ctypes.byref(ix), ctypes.byref(b), fake, 512, fake, fake, None, 1 << 30,
                                        None) == s5.S5_ERR_WORKSPACE
+
+
+def test_workspace_covers_shared_set_tiles(s5):
+    # multi-token batches also hold the tile kernel's union lists (8 rows per
+    # tile, 8 x topk + 8 entries each), per-tile path flags and per-row skip
+    # flags above the per-row partials; single-token batches do not
+    n1, n4 = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    one = _batch(batch=64, total_q=64, max_q=1, max_pages=2049, max_len=131073)
+    four = _batch(batch=64, total_q=256, max_q=4, max_pages=2049, max_len=131076)
+    assert s5._lib.s5_workspace_size(ctypes.byref(one), 0, ctypes.byref(n1)) == 0
+    assert s5._lib.s5_workspace_size(ctypes.byref(four), 0, ctypes.byref(n4)) == 0
+    union = 64 * (8 * 512 + 8) * 4
+    flags = 64 * 4 + 256 * 4
+    assert n4.value >= 256 + 16384 + union + flags
+    assert n4.value > n1.value
+    # more rows per sequence never need less
+    prev = 0
+    for max_q in (2, 8, 9, 64, 65, 1000):
+        b = _batch(batch=4, total_q=4 * max_q, max_q=max_q, max_pages=300, max_len=19000)
+        n = ctypes.c_size_t(0)
+        assert s5._lib.s5_workspace_size(ctypes.byref(b), 512, ctypes.byref(n)) == 0
+        assert n.value >= prev
+        prev = n.value

@@ -366,3 +366,18 @@ def test_prefill_both_paths(lib, ctx, nq, coherent, need_per_row):
 @pytest.mark.slow
 def test_config6_block_coherent_prefill_16k(lib):
     _config_sparse(lib, 6, 6)
+
+
+def test_tile_batches_beyond_the_compacted_list(lib):
+    # more than 4,096 tiles (520 sequences x 8 tiles of 8 rows): the tile
+    # kernel walks every tile instead of a compacted list of shared-set tiles
+    ctx = [int(x) for x in S.uniform_lengths(25, 520, 0, 300)]
+    w = S.Workload(ctx=ctx, nq=[64] * 520, seed=25)
+    d = DeviceInputs(w, lib)
+    lib.s5_reset_device_error(d.ws)
+    _run_index(lib, d)
+    _run_sparse(lib, d)
+    rows = sample_rows(w.total_q, 12, 6)
+    want_sel = _check_selection(lib, d, rows)
+    _check_sparse_out(d, rows, want_sel, "4,160 tiles")
+    _check_no_device_error(lib, d)
