@@ -171,13 +171,13 @@ TileWs tile_ws(const s5_batch_desc *b, int topk, int slots_1cta, bool sizing, si
   const long long words = (long long)(b->max_len / kBlk) / 4 + 2;
   w.map_words = (int)(words < kUnionMapWords ? words : kUnionMapWords);
   // partitions: fewest waves of the persistent CTAs per unit of work
-  // (ceil(n * units / slots) / n), n <= 8, ties to fewer partitions; merge
+  // (ceil(n * units / slots) / n), n <= kMaxTileSplit, ties to fewer partitions; merge
   // counters cover 1,024 tiles
   const long long units = (long long)w.n_tiles * kKv;
   int best = 1;
   if (w.n_tiles <= kMaxMergeRows && units > 0 && slots_1cta > 0) {
     double best_cost = 1e30;
-    for (int n = 1; n <= 8; ++n) {
+    for (int n = 1; n <= kMaxTileSplit; ++n) {
       const double cost = (double)((n * units + slots_1cta - 1) / slots_1cta) / n;
       if (cost < best_cost - 1e-9) {
         best_cost = cost;
@@ -196,7 +196,7 @@ TileWs tile_ws(const s5_batch_desc *b, int topk, int slots_1cta, bool sizing, si
   w.ent = off;
   off = align_up(off + (size_t)w.n_tiles * w.union_cap * sizeof(uint32_t), 256);
   w.part_o = w.part_lse = off;
-  const int n_res = (sizing && w.n_tiles <= kMaxMergeRows) ? 8 : w.n_split;
+  const int n_res = (sizing && w.n_tiles <= kMaxMergeRows) ? kMaxTileSplit : w.n_split;
   if (n_res > 1) {
     off = align_up(off + (size_t)b->total_q * kHeads * n_res * kD * sizeof(float), 256);
     w.part_lse = off;

@@ -53,19 +53,20 @@ __device__ __forceinline__ uint32_t swz(int r, int d) {
 // wherever the merge runs, so results do not depend on which partition
 // finished last.
 __device__ __forceinline__ void partition_weights(const float *pl, int n, float *w, float &lse_nat) {
+  float lv[kMaxSplitMerge];  // all loads in flight together (n <= kMaxSplitMerge)
+#pragma unroll
+  for (int p = 0; p < kMaxSplitMerge; ++p) lv[p] = (p < n) ? ld_cg(pl + p) : -INFINITY;
   float M = -INFINITY;
-  for (int p = 0; p < n; ++p) M = fmaxf(M, ld_cg(pl + p));
+#pragma unroll
+  for (int p = 0; p < kMaxSplitMerge; ++p) M = fmaxf(M, lv[p]);
   const float Mu = (M == -INFINITY) ? 0.f : M;
   float L = 0.f;
-  for (int p = 0; p < n; ++p) {
-    const float lp = ld_cg(pl + p);
-    L += (lp == -INFINITY) ? 0.f : hw_exp2(lp - Mu);
-  }
+#pragma unroll
+  for (int p = 0; p < kMaxSplitMerge; ++p) L += (lv[p] == -INFINITY) ? 0.f : hw_exp2(lv[p] - Mu);
   const float inv = (L > 0.f) ? 1.f / L : 0.f;
-  for (int p = 0; p < n; ++p) {
-    const float lp = ld_cg(pl + p);
-    w[p] = (lp == -INFINITY) ? 0.f : hw_exp2(lp - Mu) * inv;
-  }
+#pragma unroll
+  for (int p = 0; p < kMaxSplitMerge; ++p)
+    if (p < n) w[p] = (lv[p] == -INFINITY) ? 0.f : hw_exp2(lv[p] - Mu) * inv;
   lse_nat = (L > 0.f) ? (M + hw_log2(L)) * 0.69314718055994531f : -INFINITY;
 }
 
@@ -87,12 +88,20 @@ __global__ void __launch_bounds__(kD / 4) s5_combine_kernel(const AttnArgs a) {
   partition_weights(a.part_lse + rh * n, n, w, lse);
   const int d = threadIdx.x * 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int p = 0; p < n; ++p) {
-    const float4 v = ld_cg(reinterpret_cast<const float4 *>(a.part_o + (rh * n + p) * kD + d));
-    acc.x = fmaf(w[p], v.x, acc.x);
-    acc.y = fmaf(w[p], v.y, acc.y);
-    acc.z = fmaf(w[p], v.z, acc.z);
-    acc.w = fmaf(w[p], v.w, acc.w);
+  for (int p0 = 0; p0 < n; p0 += 8) {  // eight partitions' loads in flight at a time
+    float4 v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (p0 + q < n) v[q] = ld_cg(reinterpret_cast<const float4 *>(a.part_o + (rh * n + p0 + q) * kD + d));
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (p0 + q < n) {
+        acc.x = fmaf(w[p0 + q], v[q].x, acc.x);
+        acc.y = fmaf(w[p0 + q], v[q].y, acc.y);
+        acc.z = fmaf(w[p0 + q], v[q].z, acc.z);
+        acc.w = fmaf(w[p0 + q], v[q].w, acc.w);
+      }
+    }
   }
   store_bf16x4(reinterpret_cast<__nv_bfloat16 *>(a.out) + rh * kD + d, acc);
   if (threadIdx.x == 0 && a.lse != nullptr) a.lse[rh] = lse;

@@ -236,19 +236,21 @@ __device__ __forceinline__ TileItem decode_item(const TileArgs &a, const int *li
 // Merge weights of the partitions of one (row, head): the same arithmetic as
 // the per-row kernel's merge, in partition order.
 __device__ __forceinline__ void tile_partition_weights(const float *pl, int n, float *w, float &lse_nat) {
+  constexpr int kMaxN = kMaxTileSplit;
+  float lv[kMaxN];  // all loads in flight together
+#pragma unroll
+  for (int p = 0; p < kMaxN; ++p) lv[p] = (p < n) ? ld_cg(pl + p) : -INFINITY;
   float M = -INFINITY;
-  for (int p = 0; p < n; ++p) M = fmaxf(M, ld_cg(pl + p));
+#pragma unroll
+  for (int p = 0; p < kMaxN; ++p) M = fmaxf(M, lv[p]);
   const float Mu = (M == -INFINITY) ? 0.f : M;
   float L = 0.f;
-  for (int p = 0; p < n; ++p) {
-    const float lp = ld_cg(pl + p);
-    L += (lp == -INFINITY) ? 0.f : hw_exp2(lp - Mu);
-  }
+#pragma unroll
+  for (int p = 0; p < kMaxN; ++p) L += (lv[p] == -INFINITY) ? 0.f : hw_exp2(lv[p] - Mu);
   const float inv = (L > 0.f) ? 1.f / L : 0.f;
-  for (int p = 0; p < n; ++p) {
-    const float lp = ld_cg(pl + p);
-    w[p] = (lp == -INFINITY) ? 0.f : hw_exp2(lp - Mu) * inv;
-  }
+#pragma unroll
+  for (int p = 0; p < kMaxN; ++p)
+    if (p < n) w[p] = (lv[p] == -INFINITY) ? 0.f : hw_exp2(lv[p] - Mu) * inv;
   lse_nat = (L > 0.f) ? (M + hw_log2(L)) * 0.69314718055994531f : -INFINITY;
 }
 

@@ -100,7 +100,7 @@ struct GemmArgs {
 
 // Multi-row tiles (verify / prefill): shared-set attention on the tensor cores.
 constexpr int kTileRows = 8;           // query rows per shared-set tile (8 rows x 16 heads = M 128)
-constexpr int kMaxTileSplit = 32;
+constexpr int kMaxTileSplit = 8;      // partitions of one tile's block list
 constexpr int kUnionMapWords = 49152;  // shared byte map of the union kernel: blocks < 196,608
 
 struct TileArgs {

@@ -381,3 +381,20 @@ def test_tile_batches_beyond_the_compacted_list(lib):
     want_sel = _check_selection(lib, d, rows)
     _check_sparse_out(d, rows, want_sel, "4,160 tiles")
     _check_no_device_error(lib, d)
+
+
+@pytest.mark.parametrize("sm_scale", [0.0, -0.04, 0.3])
+def test_softmax_scale_sign_and_zero_both_paths(lib, sm_scale):
+    # a zero or negative scale turns the row maximum into the scores' minimum
+    # (or makes every weight equal): shared-set tiles (8 rows at a short
+    # history) and per-row decode rows in one batch
+    w = S.Workload(ctx=[2000, 7000, 150], nq=[8, 1, 3], seed=26)
+    d = DeviceInputs(w, lib)
+    _run_index(lib, d)
+    _run_sparse(lib, d, sm_scale=sm_scale)
+    rows = list(range(w.total_q))
+    want_sel = _check_selection(lib, d, rows)
+    want, want_lse = oracle_sparse(w, rows, want_sel, sm_scale)
+    assert_attn_close(d.out.float().cpu().numpy(), want, f"sm_scale={sm_scale}")
+    assert np.abs(d.lse.cpu().numpy() - want_lse).max() <= LSE_ABS
+    _check_no_device_error(lib, d)
