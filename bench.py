@@ -392,7 +392,9 @@ def run_ours(args) -> None:
 def run_config(args) -> None:
     """Time one step of numbered configuration `args.config` (1..6) on this GPU and
     print a JSON line with its own bytes / FLOPs (a measurement aid; the bench
-    line is the default mode)."""
+    line is the default mode).  The step and each call are captured in CUDA
+    graphs and replayed, so small batches are timed on the device rather than
+    by the host's launch rate."""
     from block_sparse_gqa_indexer_b200 import s5
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -409,9 +411,10 @@ def run_config(args) -> None:
         q, qx = w.queries(dev)
         out = torch.empty((w.total_q, 64, 192), dtype=torch.bfloat16, device=dev)
         lse = torch.empty((w.total_q, 64), dtype=torch.float32, device=dev)
+        # calls take the current stream, so the same lambdas run eagerly or under capture
         if swa:
             calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, o=out, l=lse, ws=ws:
-                         s5.s5_swa_gqa_attn(k, v, b, q, S.WINDOW, scale, o, l, ws, stream))
+                         s5.s5_swa_gqa_attn(k, v, b, q, S.WINDOW, scale, o, l, ws))
             kinds.append("swa")
             bytes_total += R.swa_decode_bytes(w.ctx, w.nq)["total"]
             flops_total += sum(R.attn_flops(R.swa_tokens(c + j)) for c, n in zip(w.ctx, w.nq) for j in range(n))
@@ -420,10 +423,10 @@ def run_config(args) -> None:
             sel = torch.empty((w.total_q, S.TOPK), dtype=torch.int32, device=dev)
             cnt = torch.empty((w.total_q,), dtype=torch.int32, device=dev)
             calls.append(lambda kp=key_pool, b=batch, qx=qx, sel=sel, cnt=cnt, ws=ws:
-                         s5.s5_index_score_topk(kp, b, qx, S.TOPK, sel, cnt, ws, stream))
+                         s5.s5_index_score_topk(kp, b, qx, S.TOPK, sel, cnt, ws))
             kinds.append("index")
             calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, sel=sel, cnt=cnt, o=out, l=lse, ws=ws:
-                         s5.s5_sparse_gqa_attn(k, v, b, q, sel, cnt, S.TOPK, scale, o, l, ws, stream))
+                         s5.s5_sparse_gqa_attn(k, v, b, q, sel, cnt, S.TOPK, scale, o, l, ws))
             kinds.append("sparse")
             bytes_total += R.sparse_decode_bytes(w.ctx, w.nq)["total"]
             flops_total += R.sparse_flops(w.ctx, w.nq)["total"]
@@ -431,26 +434,34 @@ def run_config(args) -> None:
         for c in calls:
             c()
     torch.cuda.synchronize(dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(args.steps):
-        for c in calls:
-            c()
-    t1.record(stream)
+
+    def capture(fns):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for f in fns:
+                f()
+        return g
+
+    step_graph = capture(calls)
+    call_graphs = [capture([c]) for c in calls]
     torch.cuda.synchronize(dev)
-    ms = t0.elapsed_time(t1) / args.steps
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        for j, c in enumerate(calls):
-            c()
-            ev[i][j + 1].record(stream)
-    torch.cuda.synchronize(dev)
-    per_call = [statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps))
-                for j in range(len(calls))]
+
+    def replay_ms(g, n):
+        g.replay()  # warm
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(n):
+            g.replay()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        return t0.elapsed_time(t1) / n
+
+    ms = replay_ms(step_graph, args.steps)
+    per_call = [replay_ms(g, args.steps) for g in call_graphs]
     peak, kind = _peaks()
     line = {"config": args.config, "ms_per_step": ms, "calls_ms": dict(zip([f"{k}{i}" for i, k in enumerate(kinds)],
                                                                            per_call)),
+            "timing": "CUDA-graph replay of the step (and of each call), CUDA events",
             "algorithmic_bytes": bytes_total, "useful_flops": flops_total,
             "gbs": bytes_total / (ms * 1e-3) / 1e9, "pct_hbm_peak": 100 * bytes_total / (ms * 1e-3) / 1e9 / peak,
             "useful_tflops": flops_total / (ms * 1e-3) / 1e12, "steps": args.steps, "warmup": args.warmup}

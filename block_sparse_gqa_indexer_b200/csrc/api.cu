@@ -131,6 +131,38 @@ int device_slots() {
   return cache[dev];
 }
 
+}  // namespace
+
+namespace s5 {
+cudaError_t ensure_dynamic_smem(const void *kernel, int bytes) {
+  struct Entry {
+    int dev;
+    const void *fn;
+    int bytes;
+  };
+  static std::mutex mu;
+  static Entry set[64];
+  static int n_set = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_set; ++i)
+    if (set[i].dev == dev && set[i].fn == kernel && set[i].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  for (int i = 0; i < n_set; ++i)
+    if (set[i].dev == dev && set[i].fn == kernel) {
+      set[i].bytes = bytes;
+      return cudaSuccess;
+    }
+  if (n_set < 64) set[n_set++] = Entry{dev, kernel, bytes};
+  return cudaSuccess;
+}
+}  // namespace s5
+
+namespace {
+
 struct AttnWs {
   size_t part_o, part_lse, end;
   int n_split;

@@ -521,7 +521,7 @@ cudaError_t launch_gqa_decode(int mode, const AttnArgs &a, const CUtensorMap &tk
   dim3 grid((unsigned)n_cta);
   cudaError_t e;
   auto kernel = (mode == kModeSparse) ? gqa_decode_kernel<kModeSparse> : gqa_decode_kernel<kModeSwa>;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+  e = ensure_dynamic_smem(reinterpret_cast<const void *>(kernel), kAttnSmem);
   if (e != cudaSuccess) return e;
   // programmatic stream serialization: launch and barrier setup overlap the
   // previous kernel; the kernel reads no global memory before pdl_wait()

@@ -779,14 +779,14 @@ cudaError_t launch_after(K kernel, dim3 grid, dim3 block, size_t smem, cudaStrea
 
 cudaError_t launch_tile_union(const TileArgs &a, int batch, cudaStream_t st) {
   const size_t smem = (size_t)a.map_words * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(tile_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(tile_union_kernel), (int)smem);
   if (e != cudaSuccess) return e;
   return launch_after(tile_union_kernel, dim3(a.tiles_per_seq, batch), dim3(256), smem, st, a);
 }
 
 cudaError_t launch_gqa_tile(const TileArgs &a, const CUtensorMap &tk, const CUtensorMap &tv, int n_ctas,
                             cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(gqa_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileSmem);
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(gqa_tile_kernel), kTileSmem);
   if (e != cudaSuccess) return e;
   const long long n_items = (long long)a.n_split * a.n_tiles * kKv;  // upper bound: every tile shared-set
   if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;

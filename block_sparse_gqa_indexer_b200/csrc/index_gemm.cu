@@ -226,7 +226,7 @@ cudaError_t launch_gather_keys(const GatherArgs &a, int batch, cudaStream_t st) 
 
 cudaError_t launch_index_gemm(const GemmArgs &a, const CUtensorMap &tq, const CUtensorMap &tk, int batch, int max_q,
                               cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(index_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem);
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(index_gemm_kernel), kGSmem);
   if (e != cudaSuccess) return e;
   const int n_tiles = (a.max_blocks + kGN - 1) / kGN;
   dim3 grid((n_tiles + a.tiles_per_cta - 1) / a.tiles_per_cta, (max_q + kGM - 1) / kGM, batch);

@@ -134,6 +134,11 @@ struct TileArgs {
   int32_t *err;
 };
 
+// cudaFuncSetAttribute(kernel, MaxDynamicSharedMemorySize, bytes) on the
+// current device, skipped when an equal or larger value is already set there
+// (the host cost of a call stays off the launch path of small batches).
+cudaError_t ensure_dynamic_smem(const void *kernel, int bytes);
+
 cudaError_t launch_tile_union(const TileArgs &a, int batch, cudaStream_t st);
 cudaError_t launch_gqa_tile(const TileArgs &a, const CUtensorMap &tk, const CUtensorMap &tv, int n_ctas,
                             cudaStream_t st);

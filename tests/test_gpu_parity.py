@@ -398,3 +398,34 @@ def test_softmax_scale_sign_and_zero_both_paths(lib, sm_scale):
     assert_attn_close(d.out.float().cpu().numpy(), want, f"sm_scale={sm_scale}")
     assert np.abs(d.lse.cpu().numpy() - want_lse).max() <= LSE_ABS
     _check_no_device_error(lib, d)
+
+
+def test_cuda_graph_replay_matches_eager(lib):
+    # the entry points allocate nothing and never synchronise, so a whole
+    # layer step (indexer, sparse attention with both tile paths, and a
+    # sliding-window call) captures into a CUDA graph and replays to the same
+    # bits as eager calls
+    w = S.Workload(ctx=[5003, 9000, 300, 3000], nq=[1, 2, 1, 8], seed=27)
+    d = DeviceInputs(w, lib)
+    out_swa, lse_swa = torch.empty_like(d.out), torch.empty_like(d.lse)
+
+    def step():
+        _run_index(lib, d)
+        _run_sparse(lib, d)
+        lib.s5_swa_gqa_attn(d.k_pool, d.v_pool, d.batch, d.q, S.WINDOW, O.DEFAULT_SM_SCALE, out_swa, lse_swa, d.ws)
+
+    results = (d.sel, d.sel_count, d.out, d.lse, out_swa, lse_swa)
+    step()
+    torch.cuda.synchronize()
+    eager = [t.clone() for t in results]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for t in results:
+        t.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(eager, results):
+        assert torch.equal(a, b)
+    _check_no_device_error(lib, d)
