@@ -21,7 +21,7 @@ constexpr int kSelCap = 16384;      // rows up to this many blocks: one CTA sele
 constexpr int kSegShort = 4096;     // longer rows: top-k per segment of this many blocks, then a merge
 constexpr int kSeg = 8192;          // ... segments of rows longer than 16,384 blocks
 constexpr int kMaxSeg = 32;         // (kSeg * kMaxSeg >= S5_MAX_LEN / 8)
-constexpr int kMaxSplit = 32;
+constexpr int kMaxSplit = 8;        // partitions per (row, group) beyond what kMaxList forces
 constexpr int kScorePagesPerCta = 64;  // indexer CTA: 64 pages = 512 block keys = 256 KB
 
 static_assert((long long)kSeg * kMaxSeg >= S5_MAX_LEN / S5_BLOCK_SIZE, "segments must cover the longest row");
@@ -100,7 +100,10 @@ IndexWs index_ws(const s5_batch_desc *b) {
 // Partitions per (row, group).  The kernel is HBM-bound, so the aim is one
 // wave of equal CTAs (2 resident per SM): as many partitions as fit in that
 // wave, none when the batch alone fills it, each warp keeping at least two
-// block pairs, and no CTA owning more than kMaxList blocks.
+// block pairs, and no CTA owning more than kMaxList blocks.  At most
+// kMaxSplit partitions otherwise: for the smallest batches the last CTA's
+// merge of every partition outweighs the shorter partitions (B=1 at 16K
+// tokens: 39 us of attention with 32 partitions, 25 us with 8).
 int choose_split(int total_q, int blocks_per_row, int slots) {
   const int units = total_q * kKv;
   int n = units > 0 ? slots / units : 1;
