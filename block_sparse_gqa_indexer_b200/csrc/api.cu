@@ -194,7 +194,7 @@ struct TileWs {
   int tiles_per_seq, n_tiles, union_cap, map_words, n_split;
 };
 
-// Tile CTAs hold 213 KB of shared memory: one per SM.  With `sizing`, the
+// Tile CTAs hold 215 KB of shared memory: one per SM.  With `sizing`, the
 // partials are reserved for the largest partition count any device may pick.
 // The region starts at `base`: below it lie the per-row kernel's partials,
 // which that kernel writes while other CTAs still read the tile flags.

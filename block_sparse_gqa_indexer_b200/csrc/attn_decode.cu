@@ -17,8 +17,11 @@
 // conflict-free).  The 16 query heads of the group are the M=16 rows of
 // mma.sync m16n8k16 tiles: S = Q K^T over one block is a 16x8 tile, P V over
 // two blocks a 16x192 accumulation.  Softmax is online (base 2, running max
-// per head).  The warps of a CTA merge through shared memory; partitions of a
-// row merge in s5_combine in a fixed order, so results are deterministic.
+// per head).  The warps of a CTA merge through shared memory; the partitions
+// of a (row, group) are merged in a fixed order by the last of their CTAs to
+// finish (or, beyond 1,024 rows, by s5_combine_kernel), so results are
+// deterministic.  In multi-token batches the kernel skips the rows whose tile
+// the shared-set tile kernel computes.
 //
 // This path is HBM-bound (16 FLOPs per gathered byte); its QK^T / PV run on
 // the tensor pipe only because the FP32 CUDA cores could not keep up with the

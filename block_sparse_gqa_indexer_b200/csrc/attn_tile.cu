@@ -17,14 +17,14 @@
 //   gqa_tile_kernel     a persistent kernel, one CTA per SM, walking work items
 //                       (tile, KV group, partition of the tile's list).  The
 //                       8 rows x 16 heads of a group are the M = 128 rows of
-//                       the MMAs.  Warp 8 streams 8-block chunks of K and warp
-//                       9 of V by TMA (one 3 KB copy per block, plane-major,
-//                       128-byte swizzled) through 4-stage rings; warp 10
-//                       issues S = Q K^T (N = 64 tokens, K = 192) into two
-//                       tensor-memory buffers and warp 11 O += P V, both with
-//                       their A operand (Q, P) in tensor memory (two issuing
-//                       threads, so S of a later chunk never waits behind the
-//                       PV of an earlier one); warps 0-15 load Q into
+//                       the MMAs.  Warp 16 streams 8-block chunks of K and
+//                       warp 17 of V by TMA (one 3 KB copy per block,
+//                       plane-major, 128-byte swizzled) through 4-stage rings;
+//                       warp 18 issues S = Q K^T (N = 64 tokens, K = 192) into
+//                       two tensor-memory buffers and warp 19 O += P V, both
+//                       with their A operand (Q, P) in tensor memory (two
+//                       issuing threads, so S of a later chunk never waits
+//                       behind the PV of an earlier one); warps 0-15 load Q into
 //                       tensor memory, run the masked online softmax (four
 //                       warps per 32 rows, one per quarter of the chunk's
 //                       columns, row maxima exchanged through shared memory),
@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
   };
 
   if (warp == kTWarpK || warp == kTWarpV) {
-    // ---------------- TMA producers: warp 8 K, warp 9 V ----------------
+    // ---------------- TMA producers: warp 16 K, warp 17 V ----------------
     // Lane b < 8 copies block b of each chunk (one 3 KB box: 3 planes x 8
     // tokens x 64 dims); lane 0 keeps the barrier bookkeeping.
     const bool is_k = warp == kTWarpK;
