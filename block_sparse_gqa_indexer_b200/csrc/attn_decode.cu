@@ -143,14 +143,6 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   const int sel_cnt = (MODE == kModeSparse) ? ld_cg(a.sel_count + r) : 0;
   bool bad = !locate_row(a.cu_q, a.ctx_lens, a.batch, r, row_guess(r, a.batch, a.total_q), s, t);
   if (!bad) bad = (t < 0) || (t >= a.max_pages * kPage) || (t >= a.max_len);
-  // ---- query tile of the group: 16 heads x 192, padded rows ----
-  {
-    const uint4 *qg = reinterpret_cast<const uint4 *>(a.q) + ((size_t)r * kHeads + g * kHpg) * (kD / 8);
-    for (int i = tid; i < kHpg * (kD / 8); i += kWarps * 32) {
-      const int h = i / (kD / 8), cc = i % (kD / 8);
-      *reinterpret_cast<uint4 *>(q_s + h * kQStride + cc * 16) = ld_cg(qg + i);
-    }
-  }
   const int c = bad ? 0 : t / kBlk;
   if (!bad) {
     if (MODE == kModeSparse) {
@@ -243,8 +235,24 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   if (lane == 0) {
     for (int j = 0; j < kStages && j < n_pairs; ++j) issue(j);
   }
+  // the query tile of the group (16 heads x 192, padded rows) is read while
+  // the first blocks are in flight: every thread's loads issued together
+  {
+    constexpr int kQv = kHpg * (kD / 8) / (kWarps * 32);  // 16-byte pieces per thread
+    static_assert(kHpg * (kD / 8) % (kWarps * 32) == 0, "query tile split evenly over the CTA");
+    const uint4 *qg = reinterpret_cast<const uint4 *>(a.q) + ((size_t)r * kHeads + g * kHpg) * (kD / 8);
+    uint4 qv[kQv];
+#pragma unroll
+    for (int x = 0; x < kQv; ++x) qv[x] = ld_cg(qg + tid + x * kWarps * 32);
+#pragma unroll
+    for (int x = 0; x < kQv; ++x) {
+      const int i = tid + x * kWarps * 32;
+      const int h = i / (kD / 8), cc = i % (kD / 8);
+      *reinterpret_cast<uint4 *>(q_s + h * kQStride + cc * 16) = qv[x];
+    }
+  }
   for (int k = lane + 32; k < w_n; k += 32) resolve(k);
-  __syncwarp();
+  __syncthreads();  // the query tile is complete
 
   // Q fragments (A operand) for the 12 k-steps of 16 dims
   uint32_t qa[kD / 16][4];
