@@ -371,9 +371,12 @@ __device__ __forceinline__ void find_bin_desc(const uint32_t (&c)[NB], int top, 
 // null).  The histogram gives the threshold bin; its keys are
 // then resolved either by one warp (a bit-by-bit search over the remaining 20
 // bits, when the bin holds at most kWarpRefine keys and WARP_REFINE is set) or
-// by two more block-wide radix passes of 10 bits.
-template <int NT, int EMAX, bool WARP_REFINE>
-__global__ void __launch_bounds__(NT) topk_select_hist_kernel(SelectArgs a) {
+// by two more block-wide radix passes of 10 bits.  MINB CTAs per SM: 1 keeps
+// every key in registers (short launches: one CTA per row of a decode batch),
+// 2 caps registers at 32 per thread so that batches of many rows (prefill)
+// run twice as many rows at a time.
+template <int NT, int EMAX, bool WARP_REFINE, int MINB>
+__global__ void __launch_bounds__(NT, MINB) topk_select_hist_kernel(SelectArgs a) {
   static_assert(NT == 512 || NT == 1024, "row-histogram and refinement bins are split evenly over threads");
   constexpr int NB1 = kHistBins / NT;  // row-histogram bins per thread
   constexpr int NB2 = 1024 / NT;       // refinement bins per thread
@@ -611,8 +614,11 @@ cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, cudaStrea
 }
 
 cudaError_t launch_topk_select(const SelectArgs &a, int total_q, bool two_stage, cudaStream_t st) {
-  if (!two_stage)  // with a row histogram from the scoring kernel, or one built in shared memory
-    return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false>, dim3(total_q), dim3(kSelThreads), st, a);
+  if (!two_stage) {  // with a row histogram from the scoring kernel, or one built in shared memory
+    if (total_q > 1024)
+      return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 2>, dim3(total_q), dim3(kSelThreads), st, a);
+    return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 1>, dim3(total_q), dim3(kSelThreads), st, a);
+  }
   cudaError_t e = launch_pdl(topk_segment_kernel<kSegThreads, 32>, dim3(a.n_seg, total_q), dim3(kSegThreads), st, a);
   if (e != cudaSuccess) return e;
   if (a.n_seg * a.topk <= 512 * 16) return launch_pdl(topk_merge_kernel<512, 16>, dim3(total_q), dim3(512), st, a);
