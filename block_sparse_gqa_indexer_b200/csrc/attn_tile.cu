@@ -35,6 +35,8 @@
 // masked-out products are the price of dense tiles.
 #include <cuda.h>
 
+#include <climits>
+
 #include "s5_common.cuh"
 #include "s5_kernels.h"
 #include "s5_tcgen05.cuh"
@@ -94,6 +96,7 @@ static_assert(kBFinal < kNumBars, "barrier slots");
 __global__ void __launch_bounds__(256) tile_union_kernel(const TileArgs a) {
   extern __shared__ uint32_t bmap[];  // byte b: rows that selected block b
   __shared__ int scan[8];
+  __shared__ int n_sel[kTRows];
   const int s = blockIdx.y, k = blockIdx.x;
   const int tile = s * a.tiles_per_seq + k;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -129,20 +132,40 @@ __global__ void __launch_bounds__(256) tile_union_kernel(const TileArgs a) {
   }
   for (int i = tid; i < words; i += 256) bmap[i] = 0;
   __syncthreads();
-  int row_blocks = 0;  // sum over the tile's rows of (selected blocks + current block)
-  for (int j = 0; j < nr; ++j) {
-    const int r = r0 + j;
-    const int c = (ctx + k * kTRows + j) / kBlk;
-    int n = ld_cg(a.sel_count + r);
-    if (n < 0 || n > a.topk || n > c) {
-      if (tid == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
-      n = 0;
+  // the rows' selection counts first, then every (row, entry) pair with eight
+  // loads per thread in flight at a time
+  if (tid < kTRows) {
+    int n = 0;
+    if (tid < nr) {
+      const int c = (ctx + k * kTRows + tid) / kBlk;
+      n = ld_cg(a.sel_count + r0 + tid);
+      if (n < 0 || n > a.topk || n > c) {
+        record_error(a.err, S5_ERR_DEVICE_BOUNDS, r0 + tid);
+        n = 0;
+      }
     }
-    row_blocks += n + 1;
-    for (int i = tid; i < n; i += 256) {
-      const int b = ld_cg(a.sel + (size_t)r * a.topk + i);
+    n_sel[tid] = n;
+  }
+  __syncthreads();
+  int row_blocks = 0;  // sum over the tile's rows of (selected blocks + current block)
+  for (int j = 0; j < nr; ++j) row_blocks += n_sel[j] + 1;
+  const int pairs = nr * a.topk;
+  for (int x0 = 0; x0 < pairs; x0 += 256 * 8) {
+    int bv[8], jv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int x = x0 + u * 256 + tid;
+      const int j = min(x / a.topk, kTRows - 1), i = x - j * a.topk;  // j is only used when x < pairs
+      jv[u] = j;
+      bv[u] = (x < pairs && i < n_sel[j]) ? ld_cg(a.sel + (size_t)(r0 + j) * a.topk + i) : INT_MIN;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (bv[u] == INT_MIN) continue;
+      const int j = jv[u], b = bv[u];
+      const int c = (ctx + k * kTRows + j) / kBlk;
       if (b >= 0 && b < c) atomicOr(bmap + (b >> 2), (1u << j) << ((b & 3) * 8));
-      else record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
+      else record_error(a.err, S5_ERR_DEVICE_BOUNDS, r0 + j);
     }
   }
   __syncthreads();
