@@ -82,3 +82,35 @@ def test_config_shapes():
     assert len(w5) == 4 and w5[0].ctx == [1 << 20] * 4
     # different layers draw different values
     assert not torch.equal(w5[0].k_tokens(0, torch.arange(4)), w5[1].k_tokens(0, torch.arange(4)))
+
+
+def test_block_coherent_indexer_queries():
+    # tokens of one 64-token window share a base query and differ from it by
+    # +-1 in about 1/16 of the dimensions; windows draw independent bases
+    w = S.Workload(ctx=[1000, 130], nq=[200, 64], seed=9, qx_coherent=64)
+    rows = torch.arange(w.total_q)
+    qx = w.qx_rows(rows).float()
+    seq, pos = w.row_seq_pos(rows)
+    assert torch.equal(seq[:200], torch.zeros(200, dtype=torch.int64))
+    assert torch.equal(pos[:200], torch.arange(1000, 1200))
+    assert torch.equal(pos[200:], torch.arange(130, 194))
+    assert qx.abs().max() <= 5 and torch.equal(qx, qx.round())
+    same = pos[:200] // 64 == 1000 // 64  # rows of the window holding position 1000
+    a, b = qx[:200][same][0], qx[:200][same][1]
+    frac = (a != b).float().mean().item()  # two tokens differ where either was perturbed
+    assert 0.0 < frac < 0.3
+    far = qx[0] != qx[150]  # positions 1000 and 1150: different windows
+    assert far.float().mean().item() > 0.5
+    # deterministic, a pure function of (seed, sequence, position): the second
+    # sequence drawn alone gives the same values
+    w2 = S.Workload(ctx=[130], nq=[64], seed=9, qx_coherent=64, seq_base=1, row_base=200)
+    assert torch.equal(w2.qx_rows(torch.arange(64)), w.qx_rows(torch.arange(200, 264)))
+    assert torch.equal(S.shard(w, 1, 2).qx_rows(torch.arange(64)), w.qx_rows(torch.arange(200, 264)))
+    # independent queries are unchanged by the option's existence
+    w0 = S.Workload(ctx=[1000, 130], nq=[200, 64], seed=9)
+    assert not torch.equal(w0.qx_rows(rows), w.qx_rows(rows))
+
+
+def test_config6_is_config4_with_coherent_queries():
+    (w4,), (w6,) = S.config_workloads(4), S.config_workloads(6)
+    assert w6.ctx == w4.ctx and w6.nq == w4.nq and w6.qx_coherent == 64 and w4.qx_coherent == 0
