@@ -1,8 +1,9 @@
 """Benchmark of one sparse-layer decode step (indexer + top-512 + gathered GQA).
 
 Workload: batch 64, 131,072 cached tokens per sequence, one query token each
-(64 query heads, 4 KV groups, head dim 192, bf16 KV in 64-token pages, one
-256-dim integer-valued bf16 block key per 8 tokens), seeded synthetic data.
+(64 query heads sharing 4 KV groups of dimension 192, bf16 KV in 64-token
+pages, an integer-valued 256-wide bf16 key for each 8-token block), seeded
+synthetic data.
 A step is s5_index_score_topk followed by s5_sparse_gqa_attn on resident
 inputs.  Metric: algorithmic bytes of the step (selected KV + scored block
 keys + queries / outputs) per second, with queries/s beside it.

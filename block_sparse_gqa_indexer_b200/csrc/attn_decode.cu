@@ -3,12 +3,12 @@
 // layer (the last `window` tokens).
 //
 // SGLang day-0 blog ("Step 5 Preview: Day-0 Inference and RL Support with
-// SGLang and Miles"), "Hybrid Attention": the sparse layer reads the tokens of
-// up to 512 selected 8-token blocks and of the current block; three of four
-// layers read the most recent 512 tokens.  "Kernels from StepFun": sparse
-// decode splits long KV histories into partitions and merges the partial
-// results.  StepFun open-weights blog, "What the config says": 64 query
-// heads, 4 KV groups, head dim 192.
+// SGLang and Miles"), "Hybrid Attention": a sparse-layer query attends to the
+// tokens of at most 512 chosen 8-token blocks and of its own block; the
+// sliding-window layers attend to a 512-token window.  "Kernels from
+// StepFun": decode cuts long selections into partitions and combines their
+// partial results.  StepFun open-weights blog, "What the config says": the
+// head geometry (64 query heads over 4 KV groups of dimension 192).
 //
 // Work unit: (query row r, KV group g, partition p).  One CTA of 4 warps owns
 // a unit; each warp streams its share of the unit's 8-token blocks through a

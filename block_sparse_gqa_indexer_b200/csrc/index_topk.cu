@@ -2,9 +2,10 @@
 //
 // SGLang day-0 blog ("Step 5 Preview: Day-0 Inference and RL Support with
 // SGLang and Miles"), sections "Hybrid Attention" and "Kernels from StepFun":
-// each query scores the 8-token block summaries kept in the paged cache and
-// keeps up to 512 historical blocks.  StepFun open-weights blog, "What the
-// config says": one 256-dim key per 8-token block, top 512 blocks.
+// every query rates the per-block summaries held in the paged cache and keeps
+// the best 512 blocks of its history.  StepFun open-weights blog, "What the
+// config says": the key of each 8-token block is 256 wide; the selection
+// size is 512.
 //
 // Decode / verify (a few query tokens per sequence) is an HBM-bound GEMV over
 // the block keys: every key is read once per sequence and scored against all

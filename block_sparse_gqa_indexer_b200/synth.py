@@ -28,10 +28,10 @@ arithmetic runs in int64 with every intermediate below 2**49 (32-bit
 multiplies are split into 16-bit halves), so nothing overflows.
 
 Workload shapes follow the Step 5 Preview attention configuration (the
-StepFun open-weights blog, "What the config says": 64 query heads, 4 KV
-groups, head dim 192, one 256-dim index key per 8-token block) and the SGLang
-launch flags (the SGLang day-0 blog, "Get Started": ``--page-size 64``,
-``--kv-cache-dtype bfloat16``).
+StepFun open-weights blog, "What the config says": 64 query heads sharing 4
+KV groups of dimension 192, and a 256-wide index key for each 8-token block)
+and the serving setup of the SGLang day-0 blog ("Get Started": 64-token pages
+and a bf16 KV cache).
 """
 from __future__ import annotations
 

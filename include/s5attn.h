@@ -7,12 +7,12 @@
  *   sparse full-attention layer  (SGLang day-0 blog "Step 5 Preview: Day-0
  *     Inference and RL Support with SGLang and Miles", section "Hybrid
  *     Attention"; StepFun open-weights blog, section "What the config says"):
- *     an indexer scores one 256-dim key per 8-token block of history, each
- *     query token keeps its 512 best blocks plus its current block, and
- *     grouped-query attention (64 query heads, 4 KV groups, head dim 192)
- *     runs over the tokens of those blocks only;
- *   sliding-window layer (same sections): causal GQA over the most recent
- *     512 tokens.
+ *     every block of 8 history tokens carries a 256-wide key that an
+ *     indexer rates against the query; the 512 best-rated blocks and the
+ *     block holding the query are the only tokens its grouped-query
+ *     attention (64 query heads over 4 KV groups, dimension 192) reads;
+ *   sliding-window layer (same sections): causal GQA limited to a window of
+ *     512 positions ending at the query.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -157,8 +157,8 @@ s5_status s5_sparse_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch,
                              int32_t topk, float sm_scale, void *out, float *lse,
                              void *workspace, size_t workspace_bytes, s5_stream_t stream);
 
-/* Sliding-window GQA (SGLang day-0 blog, "Hybrid Attention": three of four
- * layers read the most recent 512 tokens).  T = positions
+/* Sliding-window GQA (SGLang day-0 blog, "Hybrid Attention": the layers
+ * between sparse layers see a 512-token window).  T = positions
  * max(0, t - window + 1) .. t; otherwise as s5_sparse_gqa_attn.  Pages that
  * hold no position of any window are never read, so a sliding-window pool
  * may leave them unmapped (-1). */

@@ -18,19 +18,23 @@ Everything here is the plain definition, evaluated in float64:
 Sources (the pages give prose and a configuration table, no formulas or code):
 
 [HA]  SGLang day-0 blog "Step 5 Preview: Day-0 Inference and RL Support with
-      SGLang and Miles", section "Hybrid Attention": three of every four layers
-      read the most recent 512 tokens; the fourth scores summaries of 8-token
-      blocks, selects up to 512 historical blocks, and reads the individual
-      tokens of those blocks and of the current block.
-[KS]  same page, section "Kernels from StepFun": indexer scoring of each query
-      against the compressed history in the paged cache; sparse decode splits
-      long histories into partitions and merges partial results.
-[CFG] StepFun open-weights blog, section "What the config says": 64 query
-      heads, 4 KV groups, head dim 192; one 256-dim key per 8-token block; top
-      512 blocks (k = 4,096 tokens); 512-token sliding windows.
-[SAV] same blog, section "What sparse attention does and doesn't save": the
-      indexer scores every block; up to 512 historical blocks plus the current
-      one are read.
+      SGLang and Miles", section "Hybrid Attention": a sliding-window layer
+      attends to a 512-token window and is followed (after two more such
+      layers) by a sparse layer; the sparse layer rates each 8-token block of
+      history through a per-block summary, keeps at most 512 of them, and
+      attends to their tokens together with the tokens of the block the query
+      itself sits in.
+[KS]  same page, section "Kernels from StepFun": the indexer rates each query
+      against the compressed (per-block) history held in the paged cache;
+      decode cuts a long selection into partitions and combines their partial
+      results.
+[CFG] StepFun open-weights blog, section "What the config says": the head
+      geometry (64 query heads over 4 KV groups of dimension 192), the 256-wide
+      block key for each block of 8 tokens, the selection size (512 blocks,
+      4,096 tokens) and the window width (512).
+[SAV] same blog, section "What sparse attention does and doesn't save": every
+      history block is scored; the attention side reads at most 512 selected
+      blocks and the query's own block.
 
 Readings taken where the pages are silent (each the plainest one):
 
