@@ -180,6 +180,16 @@ def cpu_baseline(w: S.Workload, n_rows: int = 16) -> dict:
             "queries_per_s": len(rows) / dt}
 
 
+def bench_config(batch: int, n: int) -> dict:
+    """The workload description both arms report."""
+    return {"workload": f"sparse-layer decode: B={batch} per GPU, 131,072 cached tokens each, 1 query "
+                        "token; 64 q heads / 4 KV groups / head dim 192; top-512 of 16,384 blocks + current "
+                        "block",
+            "batch": batch, "ctx": 131072, "topk": 512, "page": 64, "parallelism": f"replicas x{n}",
+            "l2": "inputs larger than L2: each step reads 1.35 GB (806 MB selected KV + 537 MB block "
+                  "keys) and rotates 4 query sets so consecutive steps select different blocks"}
+
+
 def run_reference(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -200,11 +210,11 @@ def run_reference(args) -> None:
     line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "sparse decode B=64 ctx=131072 (oracle: 4 query rows per step)",
-                       "batch": 64, "ctx": 131072, "topk": 512},
+            "config": bench_config(w.batch, args.gpus),
             "queries_per_s": per_step * args.steps / total,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads(), "kind": "oracle",
-                             "sample": f"{per_step} query rows per step, {args.steps} steps"},
+                             "sample": f"{per_step} of the 64 query rows per step (float64 numpy oracle: full-sort "
+                                       f"top-512 over 16,384 block scores + sparse attention), {args.steps} steps"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -365,12 +375,7 @@ def run_ours(args) -> None:
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"sparse-layer decode: B={w.batch} per GPU, 131,072 cached tokens each, 1 query "
-                               "token; 64 q heads / 4 KV groups / head dim 192; top-512 of 16,384 blocks + current "
-                               "block",
-                   "batch": w.batch, "ctx": 131072, "topk": 512, "page": 64, "parallelism": f"replicas x{n}",
-                   "l2": "inputs larger than L2: each step reads 1.35 GB (806 MB selected KV + 537 MB block "
-                         "keys) and rotates 4 query sets so consecutive steps select different blocks"},
+        "config": bench_config(w.batch, n),
         "queries_per_s": n * w.total_q * args.steps / (ms * 1e-3),
         "pct_hbm_peak": 100.0 * (by["total"] / (step_ms * 1e-3) / 1e9) / peak,
         "kernels_ms": {"s5_index_score_topk": idx_ms, "s5_sparse_gqa_attn": attn_ms,
