@@ -303,19 +303,22 @@ class Workload:
         return own_s, own_p
 
     def kv_pools(self, device, pt: Optional[torch.Tensor] = None, pages_per_chunk: int = 2048,
-                 window_only: Optional[int] = None):
+                 window_only: Optional[int] = None, upto: Optional[Sequence[int]] = None):
         """K and V pools, bf16 [num_pages][4][64][192] each, filled through the page table.
 
         With ``window_only = W`` only pages that can hold one of the last W
         tokens before any query of the sequence are filled (the rest stay
-        zero): a sliding-window layer never reads older pages."""
+        zero): a sliding-window layer never reads older pages.  With ``upto``
+        only positions below ``upto[s]`` of sequence s are filled (e.g.
+        ``upto = ctx``: the cache before the new tokens are appended); the
+        page table and pool size stay those of the whole batch."""
         if pt is None:
             pt = self.page_table()
         own_s, own_p = self._page_owner(pt)
         n = self.num_pages
         k_pool = torch.zeros((n, N_KV, PAGE, HEAD_DIM), dtype=torch.bfloat16, device=device)
         v_pool = torch.zeros_like(k_pool)
-        lens = torch.tensor(self.lens, dtype=torch.int64)
+        lens = torch.tensor(self.lens if upto is None else list(upto), dtype=torch.int64)
         keep = own_s >= 0
         if window_only is not None:
             ctx = torch.tensor(self.ctx, dtype=torch.int64)
@@ -343,15 +346,17 @@ class Workload:
             del kv, idx, valid
         return k_pool, v_pool
 
-    def index_pool(self, device, pt: Optional[torch.Tensor] = None, pages_per_chunk: int = 16384):
+    def index_pool(self, device, pt: Optional[torch.Tensor] = None, pages_per_chunk: int = 16384,
+                   upto: Optional[Sequence[int]] = None):
         """Block-key pool, bf16 [num_pages][8][256]; slot j of page p holds the key
-        of block 8 * (logical page) + j.  Only complete blocks carry a key."""
+        of block 8 * (logical page) + j.  Only complete blocks carry a key: those
+        that end at or below ``upto[s]`` tokens (default: the whole sequence)."""
         if pt is None:
             pt = self.page_table()
         own_s, own_p = self._page_owner(pt)
         n = self.num_pages
         pool = torch.zeros((n, BLOCKS_PER_PAGE, INDEX_DIM), dtype=torch.bfloat16, device=device)
-        nblk = torch.tensor([L // BLOCK for L in self.lens], dtype=torch.int64)
+        nblk = torch.tensor([L // BLOCK for L in (self.lens if upto is None else list(upto))], dtype=torch.int64)
         ar_j = torch.arange(BLOCKS_PER_PAGE, device=device).view(1, -1, 1)
         ar_d = torch.arange(INDEX_DIM, device=device).view(1, 1, -1)
         tid = self.tid(TID_KX)
@@ -371,6 +376,24 @@ class Workload:
                 vals = normal_bf16(self.seed, tid, idx)
             pool[p0:p1] = torch.where(valid, vals, torch.zeros((), dtype=torch.bfloat16, device=device))
         return pool
+
+    def new_tokens(self, device="cpu") -> tuple:
+        """Inputs of a cache append of every query row (sequence s, position t):
+        ``(k_new, v_new)`` bf16 [total_q][4][192], the values the pools hold at
+        t, and ``key_new`` bf16 [total_q][256], the key of block t // 8 (an
+        append stores it only for a token that completes its block)."""
+        ks, vs, xs = [], [], []
+        for s in range(self.batch):
+            if self.nq[s] == 0:
+                continue
+            pos = torch.arange(self.ctx[s], self.lens[s], dtype=torch.int64)
+            ks.append(self.k_tokens(s, pos, device))
+            vs.append(self.v_tokens(s, pos, device))
+            xs.append(self.kx_blocks(s, pos // BLOCK, device))
+        if not ks:
+            e = torch.zeros((0, N_KV, HEAD_DIM), dtype=torch.bfloat16, device=device)
+            return e, e.clone(), torch.zeros((0, INDEX_DIM), dtype=torch.bfloat16, device=device)
+        return torch.cat(ks), torch.cat(vs), torch.cat(xs)
 
     def queries(self, device) -> tuple:
         """(q bf16 [total_q][64][192], qx bf16 [total_q][256]) for every query row."""

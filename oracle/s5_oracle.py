@@ -35,6 +35,8 @@ Sources (the pages give prose and a configuration table, no formulas or code):
 [SAV] same blog, section "What sparse attention does and doesn't save": every
       history block is scored; the attention side reads at most 512 selected
       blocks and the query's own block.
+[GS]  SGLang day-0 blog, section "Get Started": the cache is paged, 64 tokens
+      per page, and stored in bf16.
 
 Readings taken where the pages are silent (each the plainest one):
 
@@ -47,9 +49,15 @@ Readings taken where the pages are silent (each the plainest one):
 * softmax scale ``sm_scale`` (1/sqrt(192) by default), natural exponent;
 * the sliding window covers positions max(0, t - W + 1) .. t (the query
   included);
-* outputs rounded to bf16 with round-to-nearest-even directly from float64.
+* outputs rounded to bf16 with round-to-nearest-even directly from float64;
+* cache append: token t of a sequence lives in slot t % 64 of the page that
+  holds its logical page t // 64; a block's key is stored, in slot
+  (t % 64) // 8 of the same page, when its last token t (t % 8 == 7) arrives,
+  since only complete blocks are ever scored.
 
-Parity status: block selection is pinned by brute force, tie cases and the
+Parity status: the cache append is pinned by rebuilding the seeded pools of
+a whole batch from the pools of its cached prefix;
+block selection is pinned by brute force, tie cases and the
 subset characterisation of top-k; the attention functions are pinned by closed
 forms (one token, identical keys, two tokens), the reduction of sparse and
 sliding-window attention to full causal attention, weight normalisation and
@@ -67,6 +75,7 @@ N_HEADS = 64
 N_KV = 4
 HEADS_PER_GROUP = N_HEADS // N_KV
 HEAD_DIM = 192
+PAGE = 64
 BLOCK = 8
 INDEX_DIM = 256
 TOPK = 512
@@ -265,3 +274,44 @@ def swa_attention_batch(q, ctx, nq, kv_of_seq, window: int = WINDOW, sm_scale: f
         outs.append(o)
         lses.append(l)
     return np.array(outs), np.array(lses)
+
+
+# ----------------------------------------------------------------------------
+# cache append: new tokens and completed block keys into the paged cache
+# [KS], [GS], [CFG]
+# ----------------------------------------------------------------------------
+
+def append_to_paged_cache(k_pool, v_pool, key_pool, page_table, ctx, nq, k_new, v_new, key_new):
+    """The paged pools after appending the new tokens of a varlen batch (copies).
+
+    k_pool, v_pool  [num_pages][4][64][192]   K / V of page p, group g, slot i
+    key_pool        [num_pages][8][256] or None (a cache without block keys)
+    page_table      [batch][max_pages]        logical page -> physical page
+    k_new, v_new    [total_q][4][192]         row r = token t = ctx[s] + j
+    key_new         [total_q][256]            key of the block row r completes
+
+    Token t goes to slot t % 64 of physical page page_table[s][t // 64], for
+    all four groups.  If t is the last token of its block (t % 8 == 7),
+    key_new[r] becomes the key of block t // 8: slot (t % 64) // 8 of that
+    page.  Other rows of key_new are not read.  An unmapped page (-1) or a
+    page id outside the pool raises ValueError."""
+    k_out = np.array(k_pool, copy=True)
+    v_out = np.array(v_pool, copy=True)
+    key_out = None if key_pool is None else np.array(key_pool, copy=True)
+    page_table = np.asarray(page_table)
+    for r, (s, t) in enumerate(query_positions(ctx, nq)):
+        logical = t // PAGE
+        if logical >= page_table.shape[1]:
+            raise ValueError(f"row {r}: position {t} beyond the page table")
+        p = int(page_table[s, logical])
+        if p < 0 or p >= k_out.shape[0]:
+            raise ValueError(f"row {r}: page {p} not in the pool")
+        slot = t % PAGE
+        for g in range(N_KV):
+            k_out[p, g, slot, :] = k_new[r][g]
+            v_out[p, g, slot, :] = v_new[r][g]
+        if key_out is not None and t % BLOCK == BLOCK - 1:
+            if p >= key_out.shape[0]:
+                raise ValueError(f"row {r}: page {p} not in the key pool")
+            key_out[p, slot // BLOCK, :] = key_new[r]
+    return k_out, v_out, key_out

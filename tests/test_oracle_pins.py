@@ -401,3 +401,67 @@ def test_sparse_tokens_bounds():
     assert {R.sparse_tokens(8 * 5000 + j) for j in range(8)} == set(range(4097, 4105))
     assert R.sparse_tokens(0) == 1
     assert R.scored_blocks(8 * 512 + 7) == 0 and R.scored_blocks(8 * 513) == 513
+
+
+# ---------------------------------------------------------------- cache append
+
+def _bits(t):
+    """bf16 tensor -> int16 numpy bit patterns (exact comparisons)."""
+    return t.contiguous().view(torch.int16).numpy()
+
+
+def _append_case():
+    from block_sparse_gqa_indexer_b200 import synth as S
+    # page and block boundaries on both sides of the new tokens, an empty
+    # sequence, a fresh sequence, several pages of new tokens
+    return S.Workload(ctx=[0, 5, 63, 64, 130, 1000, 7, 40], nq=[3, 9, 1, 64, 70, 17, 0, 200], seed=11)
+
+
+def test_append_rebuilds_the_seeded_cache_from_its_prefix():
+    # The generator's pool builder fills positions below `upto` through the
+    # page table on its own; appending the new tokens (and the keys of the
+    # blocks they complete) to the prefix pools must give the whole batch's
+    # pools bit for bit.
+    w = _append_case()
+    pt = w.page_table()
+    k0, v0 = w.kv_pools("cpu", pt, upto=w.ctx)
+    x0 = w.index_pool("cpu", pt, upto=w.ctx)
+    k1, v1 = w.kv_pools("cpu", pt)
+    x1 = w.index_pool("cpu", pt)
+    kn, vn, xn = w.new_tokens("cpu")
+    # rows that complete no block carry junk: the append must not read them
+    _, pos = w.query_seq_pos()
+    junk = torch.tensor([p % 8 != 7 for p in pos])
+    xn = xn.clone()
+    xn[junk] = torch.tensor(-3.5, dtype=torch.bfloat16)
+    ko, vo, xo = O.append_to_paged_cache(_bits(k0), _bits(v0), _bits(x0), pt.numpy(), w.ctx, w.nq, _bits(kn),
+                                         _bits(vn), _bits(xn))
+    assert np.array_equal(ko, _bits(k1)) and np.array_equal(vo, _bits(v1)) and np.array_equal(xo, _bits(x1))
+    # the prefix really differed (the append did the work)
+    assert not np.array_equal(_bits(k0), _bits(k1)) and not np.array_equal(_bits(x0), _bits(x1))
+
+
+def test_append_without_block_keys_and_empty_batch():
+    w = _append_case()
+    pt = w.page_table()
+    k0, v0 = w.kv_pools("cpu", pt, upto=w.ctx)
+    k1, v1 = w.kv_pools("cpu", pt)
+    kn, vn, _ = w.new_tokens("cpu")
+    ko, vo, xo = O.append_to_paged_cache(_bits(k0), _bits(v0), None, pt.numpy(), w.ctx, w.nq, _bits(kn),
+                                         _bits(vn), None)
+    assert xo is None and np.array_equal(ko, _bits(k1)) and np.array_equal(vo, _bits(v1))
+    # no new tokens: nothing changes
+    z = np.zeros((0, 4, 192), dtype=np.int16)
+    ke, ve, xe = O.append_to_paged_cache(_bits(k0), _bits(v0), None, pt.numpy(), w.ctx, [0] * w.batch, z, z, None)
+    assert np.array_equal(ke, _bits(k0)) and np.array_equal(ve, _bits(v0))
+
+
+def test_append_rejects_unmapped_pages():
+    w = _append_case()
+    pt = w.page_table()
+    k0, v0 = w.kv_pools("cpu", pt, upto=w.ctx)
+    kn, vn, xn = w.new_tokens("cpu")
+    bad = pt.numpy().copy()
+    bad[4, 2] = -1  # sequence 4 appends positions 130..199: logical pages 2 and 3
+    with pytest.raises(ValueError):
+        O.append_to_paged_cache(_bits(k0), _bits(v0), None, bad, w.ctx, w.nq, _bits(kn), _bits(vn), None)
