@@ -417,6 +417,16 @@ def run_config(args) -> None:
         q, qx = w.queries(dev)
         out = torch.empty((w.total_q, 64, 192), dtype=torch.bfloat16, device=dev)
         lse = torch.empty((w.total_q, 64), dtype=torch.float32, device=dev)
+        key_pool = None if swa else w.index_pool(dev, pt)
+        if args.append:
+            # the step starts by storing its new tokens (and completed block
+            # keys); the pools already hold these values, so every replay
+            # writes the same bytes
+            kn, vn, xn = w.new_tokens(dev)
+            calls.append(lambda k=k_pool, v=v_pool, kp=key_pool, b=batch, kn=kn, vn=vn, xn=xn, ws=ws:
+                         s5.s5_append_kv(k, v, kp, b, kn, vn, None if kp is None else xn, ws))
+            kinds.append("append")
+            bytes_total += R.append_bytes(w.ctx, w.nq, with_keys=not swa)["total"]
         # calls take the current stream, so the same lambdas run eagerly or under capture
         if swa:
             calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, o=out, l=lse, ws=ws:
@@ -425,7 +435,6 @@ def run_config(args) -> None:
             bytes_total += R.swa_decode_bytes(w.ctx, w.nq)["total"]
             flops_total += sum(R.attn_flops(R.swa_tokens(c + j)) for c, n in zip(w.ctx, w.nq) for j in range(n))
         else:
-            key_pool = w.index_pool(dev, pt)
             sel = torch.empty((w.total_q, S.TOPK), dtype=torch.int32, device=dev)
             cnt = torch.empty((w.total_q,), dtype=torch.int32, device=dev)
             calls.append(lambda kp=key_pool, b=batch, qx=qx, sel=sel, cnt=cnt, ws=ws:
@@ -470,7 +479,8 @@ def run_config(args) -> None:
             "timing": "CUDA-graph replay of the step (and of each call), CUDA events",
             "algorithmic_bytes": bytes_total, "useful_flops": flops_total,
             "gbs": bytes_total / (ms * 1e-3) / 1e9, "pct_hbm_peak": 100 * bytes_total / (ms * 1e-3) / 1e9 / peak,
-            "useful_tflops": flops_total / (ms * 1e-3) / 1e12, "steps": args.steps, "warmup": args.warmup}
+            "useful_tflops": flops_total / (ms * 1e-3) / 1e12, "steps": args.steps, "warmup": args.warmup,
+            "append": bool(args.append)}
     print(json.dumps(line), flush=True)
 
 
@@ -484,6 +494,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--config", type=int, default=0, help="time numbered configuration 1..6 instead")
     ap.add_argument("--shard", type=int, default=1, help="with --config: run the first of this many batch shards")
+    ap.add_argument("--append", action="store_true",
+                    help="with --config: each layer step first appends its new tokens to the cache")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

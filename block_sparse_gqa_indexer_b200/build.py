@@ -15,7 +15,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libs5attn.so")
-SOURCES = ["api.cu", "index_topk.cu", "index_gemm.cu", "attn_decode.cu", "attn_tile.cu", "index_noalloc.cu"]
+SOURCES = ["api.cu", "index_topk.cu", "index_gemm.cu", "attn_decode.cu", "attn_tile.cu", "index_noalloc.cu",
+           "kv_append.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

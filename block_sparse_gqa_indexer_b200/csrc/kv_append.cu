@@ -1,0 +1,133 @@
+// s5_append_kv: the cache-append step on either side of the attention path.
+// Every new token's K and V rows go into their slot of the paged pools, and a
+// token that completes its 8-token block stores that block's 256-wide key in
+// the index-key pool, so the next indexer call scores it (SGLang day-0 blog,
+// "Kernels from StepFun": the indexer reads the per-block history from the
+// paged cache; "Get Started": 64-token pages, bf16 cache).
+//
+// Layout of one row's work: K and V of one token are 4 groups x 384 bytes
+// each, scattered to 4 slots 24 KB apart in one physical page; the block key is
+// 512 bytes.  The CTA has 7 warps, one 16-byte chunk per thread: warps 0-2
+// copy K (96 chunks), warps 3-5 copy V, warp 6 the key.  Each warp covers 512
+// contiguous source bytes, and each group's 384-byte destination row is
+// contiguous.  The kernel is a pure copy (about 3.6 KB read and written per
+// token), so it is bound by latency at decode sizes and by HBM in prefill.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "s5_common.cuh"
+
+using namespace s5;
+
+namespace {
+
+constexpr int kAppendThreads = 224;                    // 7 warps
+constexpr int kRowChunks = kD * 2 / 16;                // 24 chunks of 16 B per (token, group) row
+constexpr int kKvChunks = kKv * kRowChunks;            // 96 per token, K or V
+constexpr int kKeyChunks = kDx * 2 / 16;               // 32 per block key
+constexpr int kAppendCtasPerSm = 8;
+constexpr int kAppendMaxCtas = 148 * kAppendCtasPerSm;
+
+static_assert(2 * kKvChunks + kKeyChunks == kAppendThreads, "one chunk per thread");
+
+struct AppendArgs {
+  uint8_t *k_pool;
+  uint8_t *v_pool;
+  uint8_t *key_pool;  // null: no block keys
+  int32_t kv_pages;
+  int32_t key_pages;
+  const int32_t *page_table;
+  int32_t max_pages;
+  const int32_t *ctx_lens;
+  const int32_t *cu_q;
+  int32_t batch;
+  int32_t total_q;
+  const uint8_t *k_new;
+  const uint8_t *v_new;
+  const uint8_t *key_new;
+  int32_t *err;
+};
+
+__global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(const AppendArgs a) {
+  const int tid = threadIdx.x;
+  for (int r = blockIdx.x; r < a.total_q; r += gridDim.x) {
+    int s = 0, t = 0;
+    if (!locate_row(a.cu_q, a.ctx_lens, a.batch, r, row_guess(r, a.batch, a.total_q), s, t) || t < 0) {
+      if (tid == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
+      continue;
+    }
+    const int logical = t / kPage;
+    const int page = logical < a.max_pages ? ld_cg(a.page_table + (size_t)s * a.max_pages + logical) : -1;
+    const int slot = t % kPage;
+    if (tid < 2 * kKvChunks) {
+      if (page < 0 || page >= a.kv_pages) {
+        if (tid == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
+        continue;
+      }
+      const bool is_v = tid >= kKvChunks;
+      const int c = is_v ? tid - kKvChunks : tid;
+      const int g = c / kRowChunks, w = c % kRowChunks;
+      const uint8_t *src = (is_v ? a.v_new : a.k_new) + ((size_t)r * kKvChunks + c) * 16;
+      uint8_t *dst = (is_v ? a.v_pool : a.k_pool) +
+                     ((((size_t)page * kKv + g) * kPage + slot) * kRowChunks + w) * 16;
+      *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
+    } else if (a.key_pool != nullptr && t % kBlk == kBlk - 1) {
+      // the key of block t / 8 lives in slot (t % 64) / 8 of the same page
+      const int c = tid - 2 * kKvChunks;
+      if (page < 0 || page >= a.key_pages) {
+        if (c == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
+        continue;
+      }
+      const uint8_t *src = a.key_new + ((size_t)r * kKeyChunks + c) * 16;
+      uint8_t *dst = a.key_pool + (((size_t)page * kBpp + slot / kBlk) * kKeyChunks + c) * 16;
+      *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
+    }
+  }
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" s5_status s5_append_kv(const s5_kv_desc *kv, const s5_index_desc *index, const s5_batch_desc *batch,
+                                  const void *k_new, const void *v_new, const void *key_new, void *workspace,
+                                  size_t workspace_bytes, s5_stream_t stream) {
+  if (batch == nullptr || kv == nullptr) return S5_ERR_INVALID_ARG;
+  if (batch->batch < 1 || batch->max_pages < 1 || batch->total_q < 0) return S5_ERR_INVALID_ARG;
+  if (batch->page_table == nullptr || batch->ctx_lens == nullptr || batch->cu_q == nullptr)
+    return S5_ERR_INVALID_ARG;
+  if (kv->k_pool == nullptr || kv->v_pool == nullptr || kv->num_pages < 1) return S5_ERR_INVALID_ARG;
+  if (kv->page_size != kPage || kv->n_kv_heads != kKv || kv->head_dim != kD) return S5_ERR_UNSUPPORTED;
+  if (!aligned16(kv->k_pool) || !aligned16(kv->v_pool)) return S5_ERR_INVALID_ARG;
+  if (index != nullptr) {
+    if (index->key_pool == nullptr || index->num_pages < 1 || !aligned16(index->key_pool))
+      return S5_ERR_INVALID_ARG;
+    if (index->index_dim != kDx) return S5_ERR_UNSUPPORTED;
+  }
+  if (workspace == nullptr || workspace_bytes < S5_WS_FIXED_BYTES) return S5_ERR_WORKSPACE;
+  if (batch->total_q == 0) return S5_OK;
+  if (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new)) return S5_ERR_INVALID_ARG;
+  if (index != nullptr && (key_new == nullptr || !aligned16(key_new))) return S5_ERR_INVALID_ARG;
+
+  AppendArgs a{};
+  // the pools are written: the descriptors' const covers the read-only calls
+  a.k_pool = static_cast<uint8_t *>(const_cast<void *>(kv->k_pool));
+  a.v_pool = static_cast<uint8_t *>(const_cast<void *>(kv->v_pool));
+  a.key_pool = index != nullptr ? static_cast<uint8_t *>(const_cast<void *>(index->key_pool)) : nullptr;
+  a.kv_pages = kv->num_pages;
+  a.key_pages = index != nullptr ? index->num_pages : 0;
+  a.page_table = batch->page_table;
+  a.max_pages = batch->max_pages;
+  a.ctx_lens = batch->ctx_lens;
+  a.cu_q = batch->cu_q;
+  a.batch = batch->batch;
+  a.total_q = batch->total_q;
+  a.k_new = static_cast<const uint8_t *>(k_new);
+  a.v_new = static_cast<const uint8_t *>(v_new);
+  a.key_new = index != nullptr ? static_cast<const uint8_t *>(key_new) : nullptr;
+  a.err = static_cast<int32_t *>(workspace);
+  const int grid = batch->total_q < kAppendMaxCtas ? batch->total_q : kAppendMaxCtas;
+  kv_append_kernel<<<grid, kAppendThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return cudaGetLastError() == cudaSuccess ? S5_OK : S5_ERR_CUDA;
+}

@@ -109,6 +109,18 @@ def swa_decode_bytes(ctx, nq, window: int = WINDOW) -> dict:
     return {"kv": kv, "keys": 0, "qio": qio, "total": kv + qio}
 
 
+def append_bytes(ctx, nq, with_keys: bool = True) -> dict:
+    """Algorithmic bytes of one cache append: each new token's K/V read once
+    and written once; with block keys, each key of a block the batch
+    completes read once and written once."""
+    kv = keys = 0
+    for c0, n in zip(ctx, nq):
+        kv += 2 * n * kv_bytes_per_token()
+        if with_keys:
+            keys += 2 * ((c0 + n) // BLOCK - c0 // BLOCK) * index_key_bytes()
+    return {"kv": kv, "keys": keys, "total": kv + keys}
+
+
 def sparse_flops(ctx, nq, topk: int = TOPK) -> dict:
     attn = index = 0
     for c0, n in zip(ctx, nq):

@@ -30,8 +30,8 @@ S5_OK, S5_ERR_INVALID_ARG, S5_ERR_UNSUPPORTED, S5_ERR_CUDA, S5_ERR_DEVICE_BOUNDS
 
 # exported symbols (every declaration of include/s5attn.h)
 SYMBOLS = ("s5_workspace_size", "s5_index_score_topk", "s5_sparse_gqa_attn", "s5_swa_gqa_attn",
-           "s5_index_score_topk_noalloc", "s5_reset_device_error", "s5_get_device_error", "s5_status_string",
-           "s5_abi_version")
+           "s5_index_score_topk_noalloc", "s5_append_kv", "s5_reset_device_error", "s5_get_device_error",
+           "s5_status_string", "s5_abi_version")
 
 
 class KvDesc(ctypes.Structure):
@@ -60,6 +60,8 @@ _lib.s5_swa_gqa_attn.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(BatchDes
                                  _P, _P, ctypes.c_size_t, _P]
 _lib.s5_index_score_topk_noalloc.argtypes = [ctypes.POINTER(IndexDesc), ctypes.POINTER(BatchDesc), _P, _I, _P,
                                              _P, _P]
+_lib.s5_append_kv.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(IndexDesc), ctypes.POINTER(BatchDesc), _P, _P,
+                              _P, _P, ctypes.c_size_t, _P]
 _lib.s5_reset_device_error.argtypes = [_P, _P]
 _lib.s5_get_device_error.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
 _lib.s5_status_string.argtypes = [ctypes.c_int]
@@ -208,6 +210,24 @@ def s5_swa_gqa_attn(k_pool, v_pool, batch: Batch, q, window: int, sm_scale: floa
     _check(_lib.s5_swa_gqa_attn(ctypes.byref(kv), ctypes.byref(batch.desc), _ptr(q), int(window),
                                 float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
            "s5_swa_gqa_attn")
+
+
+def s5_append_kv(k_pool, v_pool, key_pool, batch: Batch, k_new, v_new, key_new, ws, stream=None):
+    """Write the new tokens' K/V (and, with a key pool, the keys of the blocks
+    they complete) into the paged cache; ``key_pool`` and ``key_new`` may be
+    None for a cache without block keys."""
+    kv = _kv(k_pool, v_pool)
+    _need(k_new, torch.bfloat16, "k_new", (batch.total_q, N_KV, HEAD_DIM))
+    _need(v_new, torch.bfloat16, "v_new", (batch.total_q, N_KV, HEAD_DIM))
+    idx = None
+    if key_pool is not None:
+        _need(key_pool, torch.bfloat16, "key_pool")
+        _need(key_new, torch.bfloat16, "key_new", (batch.total_q, INDEX_DIM))
+        idx = IndexDesc(key_pool.data_ptr(), key_pool.shape[0], key_pool.shape[-1])
+    _need(ws, torch.uint8, "ws")
+    _check(_lib.s5_append_kv(ctypes.byref(kv), None if idx is None else ctypes.byref(idx), ctypes.byref(batch.desc),
+                             _ptr(k_new), _ptr(v_new), None if idx is None else _ptr(key_new), _ptr(ws),
+                             ws.numel(), _stream(stream)), "s5_append_kv")
 
 
 def s5_reset_device_error(ws: torch.Tensor, stream=None):

@@ -192,6 +192,33 @@ s5_status s5_index_score_topk_noalloc(const s5_index_desc *index, const s5_batch
                                       const void *q_index, int32_t topk, int32_t *sel, int32_t *sel_count,
                                       s5_stream_t stream);
 
+/* Cache append: store the batch's new tokens, and the keys of the blocks
+ * they complete, in the paged cache before the layer's attention reads them
+ * (SGLang day-0 blog, "Kernels from StepFun": the indexer scores the
+ * per-block history kept in the paged cache; "Get Started": 64-token pages,
+ * bf16 cache).  For row r of sequence s at position t = ctx_lens[s] + j:
+ *   K/V   k_new[r][g] / v_new[r][g] -> slot t % 64 of group g of physical page
+ *         page_table[s][t / 64], for g = 0..3;
+ *   key   if t % 8 == 7 (t completes block t / 8): key_new[r] -> slot
+ *         (t % 64) / 8 of the same physical page of the index-key pool.
+ * Only complete blocks are ever scored, so a block's key is stored once, with
+ * its last token; key_new rows of other tokens are not read.
+ *   kv       the pools to WRITE (the descriptor's const applies to the
+ *            attention calls, which only read them)
+ *   index    the block-key pool to write, or NULL for a cache without block
+ *            keys (a sliding-window layer); key_new is then ignored
+ *   k_new, v_new  device bf16 [total_q][4][192], 16-byte aligned
+ *   key_new  device bf16 [total_q][256], 16-byte aligned (when index != NULL)
+ *   workspace  at least S5_WS_FIXED_BYTES; only its error record is used
+ * The pages of every new position must be mapped before the call.  An
+ * unmapped page (-1), a page id outside its pool or a position past the page
+ * table records S5_ERR_DEVICE_BOUNDS (info = the row) and that row's write is
+ * skipped.  batch->max_q and batch->max_len are not used.  Rows are
+ * independent: positions written by one call must be distinct. */
+s5_status s5_append_kv(const s5_kv_desc *kv, const s5_index_desc *index, const s5_batch_desc *batch,
+                       const void *k_new, const void *v_new, const void *key_new, void *workspace,
+                       size_t workspace_bytes, s5_stream_t stream);
+
 /* Zero the first S5_WS_FIXED_BYTES of a workspace: the device error record
  * and the partition counters (asynchronous, on `stream`). */
 s5_status s5_reset_device_error(void *workspace, s5_stream_t stream);

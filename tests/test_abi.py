@@ -117,3 +117,33 @@ def test_workspace_covers_shared_set_tiles(s5):
         assert s5._lib.s5_workspace_size(ctypes.byref(b), 512, ctypes.byref(n)) == 0
         assert n.value >= prev
         prev = n.value
+
+
+def test_append_rejects_bad_arguments_before_launch(s5):
+    fake = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1008)
+    b = _batch()
+    kv = s5.KvDesc(0x1000, 0x1000, 8, 64, 4, 192)
+    ix = s5.IndexDesc(0x1000, 8, 256)
+    big = 1 << 20
+    ap = s5._lib.s5_append_kv
+    # unsupported geometry
+    bad_kv = s5.KvDesc(0x1000, 0x1000, 8, 64, 4, 128)
+    assert ap(ctypes.byref(bad_kv), None, ctypes.byref(b), fake, fake, None, fake, big, None) == s5.S5_ERR_UNSUPPORTED
+    bad_ix = s5.IndexDesc(0x1000, 8, 128)
+    assert ap(ctypes.byref(kv), ctypes.byref(bad_ix), ctypes.byref(b), fake, fake, fake, fake, big,
+              None) == s5.S5_ERR_UNSUPPORTED
+    # missing or misaligned new rows, missing keys with a key pool
+    assert ap(ctypes.byref(kv), None, ctypes.byref(b), None, fake, None, fake, big, None) == s5.S5_ERR_INVALID_ARG
+    assert ap(ctypes.byref(kv), None, ctypes.byref(b), fake, odd, None, fake, big, None) == s5.S5_ERR_INVALID_ARG
+    assert ap(ctypes.byref(kv), ctypes.byref(ix), ctypes.byref(b), fake, fake, None, fake, big,
+              None) == s5.S5_ERR_INVALID_ARG
+    # workspace: the error record and counters at least
+    assert ap(ctypes.byref(kv), None, ctypes.byref(b), fake, fake, None, fake, 256, None) == s5.S5_ERR_WORKSPACE
+    assert ap(ctypes.byref(kv), None, ctypes.byref(b), fake, fake, None, None, big, None) == s5.S5_ERR_WORKSPACE
+    # bad batch
+    assert ap(ctypes.byref(kv), None, ctypes.byref(_batch(batch=0)), fake, fake, None, fake, big,
+              None) == s5.S5_ERR_INVALID_ARG
+    # nothing to append: OK with nothing enqueued (null rows allowed)
+    assert ap(ctypes.byref(kv), ctypes.byref(ix), ctypes.byref(_batch(total_q=0)), None, None, None, fake, big,
+              None) == s5.S5_OK

@@ -403,6 +403,22 @@ def test_sparse_tokens_bounds():
     assert R.scored_blocks(8 * 512 + 7) == 0 and R.scored_blocks(8 * 513) == 513
 
 
+def test_append_bytes_count_written_keys():
+    from block_sparse_gqa_indexer_b200 import roofline as R
+    # a token is 3,072 bytes of K and V, read once and written once; a key is
+    # moved only for blocks the batch completes: 7 -> 8 completes block 0,
+    # 8 -> 9 completes none, 5 -> 22 completes blocks 0 and 1
+    assert R.append_bytes([7], [1]) == {"kv": 6144, "keys": 1024, "total": 7168}
+    assert R.append_bytes([8], [1])["keys"] == 0
+    assert R.append_bytes([5], [17])["keys"] == 2 * 1024
+    assert R.append_bytes([7], [1], with_keys=False)["total"] == 6144
+    # the prefix-to-whole check of the oracle counts the same blocks
+    w = _append_case()
+    _, pos = w.query_seq_pos()
+    completing = sum(1 for t in pos if t % 8 == 7)
+    assert R.append_bytes(w.ctx, w.nq)["keys"] == completing * 1024
+
+
 # ---------------------------------------------------------------- cache append
 
 def _bits(t):
