@@ -7,11 +7,12 @@
 //
 // Layout of one row's work: K and V of one token are 4 groups x 384 bytes
 // each, scattered to 4 slots 24 KB apart in one physical page; the block key is
-// 512 bytes.  The CTA has 7 warps, one 16-byte chunk per thread: warps 0-2
-// copy K (96 chunks), warps 3-5 copy V, warp 6 the key.  Each warp covers 512
-// contiguous source bytes, and each group's 384-byte destination row is
-// contiguous.  The kernel is a pure copy (about 3.6 KB read and written per
-// token), so it is bound by latency at decode sizes and by HBM in prefill.
+// 512 bytes.  The CTA has 7 warps, one 16-byte chunk of each row per thread:
+// warps 0-2 copy K (96 chunks), warps 3-5 copy V, warp 6 the key.  Each warp
+// covers 512 contiguous source bytes, and each group's 384-byte destination
+// row is contiguous.  The kernel is a pure copy (about 3.6 KB read and
+// written per token), so it is bound by latency at decode sizes and by HBM in
+// prefill.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -26,8 +27,8 @@ constexpr int kAppendThreads = 224;                    // 7 warps
 constexpr int kRowChunks = kD * 2 / 16;                // 24 chunks of 16 B per (token, group) row
 constexpr int kKvChunks = kKv * kRowChunks;            // 96 per token, K or V
 constexpr int kKeyChunks = kDx * 2 / 16;               // 32 per block key
-constexpr int kAppendCtasPerSm = 8;
-constexpr int kAppendMaxCtas = 148 * kAppendCtasPerSm;
+constexpr int kAppendRows = 4;                         // rows per CTA pass
+constexpr int kAppendMaxCtas = 148 * 32;
 
 static_assert(2 * kKvChunks + kKeyChunks == kAppendThreads, "one chunk per thread");
 
@@ -49,40 +50,61 @@ struct AppendArgs {
   int32_t *err;
 };
 
+// One pass of a CTA covers kAppendRows rows: first one thread per row finds
+// its sequence, position and physical page (dependent lookups, all rows at
+// once), then every thread issues its 16-byte loads for all rows before any
+// store, so each thread keeps kAppendRows independent loads in flight.
 __global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(const AppendArgs a) {
+  __shared__ int s_page[kAppendRows];
+  __shared__ int s_pos[kAppendRows];
   const int tid = threadIdx.x;
-  for (int r = blockIdx.x; r < a.total_q; r += gridDim.x) {
-    int s = 0, t = 0;
-    if (!locate_row(a.cu_q, a.ctx_lens, a.batch, r, row_guess(r, a.batch, a.total_q), s, t) || t < 0) {
-      if (tid == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
-      continue;
-    }
-    const int logical = t / kPage;
-    const int page = logical < a.max_pages ? ld_cg(a.page_table + (size_t)s * a.max_pages + logical) : -1;
-    const int slot = t % kPage;
-    if (tid < 2 * kKvChunks) {
-      if (page < 0 || page >= a.kv_pages) {
-        if (tid == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
-        continue;
+  const bool is_key = tid >= 2 * kKvChunks;
+  const bool is_v = tid >= kKvChunks && !is_key;
+  const int c = is_key ? tid - 2 * kKvChunks : (is_v ? tid - kKvChunks : tid);
+  const int g = c / kRowChunks, w = c % kRowChunks;
+  for (int r0 = blockIdx.x * kAppendRows; r0 < a.total_q; r0 += gridDim.x * kAppendRows) {
+    if (tid < kAppendRows) {
+      const int r = r0 + tid;
+      int page = -1, t = -1;
+      if (r < a.total_q) {
+        int s = 0;
+        if (locate_row(a.cu_q, a.ctx_lens, a.batch, r, row_guess(r, a.batch, a.total_q), s, t) && t >= 0) {
+          const int logical = t / kPage;
+          page = logical < a.max_pages ? ld_cg(a.page_table + (size_t)s * a.max_pages + logical) : -1;
+        }
+        if (page < 0 || page >= a.kv_pages || (a.key_pool != nullptr && page >= a.key_pages)) {
+          record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
+          page = -1;
+        }
       }
-      const bool is_v = tid >= kKvChunks;
-      const int c = is_v ? tid - kKvChunks : tid;
-      const int g = c / kRowChunks, w = c % kRowChunks;
-      const uint8_t *src = (is_v ? a.v_new : a.k_new) + ((size_t)r * kKvChunks + c) * 16;
-      uint8_t *dst = (is_v ? a.v_pool : a.k_pool) +
-                     ((((size_t)page * kKv + g) * kPage + slot) * kRowChunks + w) * 16;
-      *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
-    } else if (a.key_pool != nullptr && t % kBlk == kBlk - 1) {
-      // the key of block t / 8 lives in slot (t % 64) / 8 of the same page
-      const int c = tid - 2 * kKvChunks;
-      if (page < 0 || page >= a.key_pages) {
-        if (c == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
-        continue;
-      }
-      const uint8_t *src = a.key_new + ((size_t)r * kKeyChunks + c) * 16;
-      uint8_t *dst = a.key_pool + (((size_t)page * kBpp + slot / kBlk) * kKeyChunks + c) * 16;
-      *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
+      s_page[tid] = page;
+      s_pos[tid] = t;
     }
+    __syncthreads();
+    uint4 v[kAppendRows];
+    bool on[kAppendRows];
+#pragma unroll
+    for (int i = 0; i < kAppendRows; ++i) {
+      const int t = s_pos[i];
+      // a key moves only for the token that completes its block
+      on[i] = s_page[i] >= 0 && (!is_key || (a.key_pool != nullptr && t % kBlk == kBlk - 1));
+      if (on[i]) {
+        const size_t r = (size_t)(r0 + i);
+        const uint8_t *src = is_key ? a.key_new + (r * kKeyChunks + c) * 16
+                                    : (is_v ? a.v_new : a.k_new) + (r * kKvChunks + c) * 16;
+        v[i] = *reinterpret_cast<const uint4 *>(src);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kAppendRows; ++i) {
+      if (!on[i]) continue;
+      const size_t page = (size_t)s_page[i];
+      const int slot = s_pos[i] % kPage;
+      uint8_t *dst = is_key ? a.key_pool + ((page * kBpp + slot / kBlk) * kKeyChunks + c) * 16
+                            : (is_v ? a.v_pool : a.k_pool) + (((page * kKv + g) * kPage + slot) * kRowChunks + w) * 16;
+      *reinterpret_cast<uint4 *>(dst) = v[i];
+    }
+    __syncthreads();  // s_page / s_pos are rewritten by the next pass
   }
 }
 
@@ -127,7 +149,8 @@ extern "C" s5_status s5_append_kv(const s5_kv_desc *kv, const s5_index_desc *ind
   a.v_new = static_cast<const uint8_t *>(v_new);
   a.key_new = index != nullptr ? static_cast<const uint8_t *>(key_new) : nullptr;
   a.err = static_cast<int32_t *>(workspace);
-  const int grid = batch->total_q < kAppendMaxCtas ? batch->total_q : kAppendMaxCtas;
+  const int passes = (batch->total_q + kAppendRows - 1) / kAppendRows;
+  const int grid = passes < kAppendMaxCtas ? passes : kAppendMaxCtas;
   kv_append_kernel<<<grid, kAppendThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return cudaGetLastError() == cudaSuccess ? S5_OK : S5_ERR_CUDA;
 }

@@ -211,9 +211,9 @@ s5_status s5_index_score_topk_noalloc(const s5_index_desc *index, const s5_batch
  *   key_new  device bf16 [total_q][256], 16-byte aligned (when index != NULL)
  *   workspace  at least S5_WS_FIXED_BYTES; only its error record is used
  * The pages of every new position must be mapped before the call.  An
- * unmapped page (-1), a page id outside its pool or a position past the page
- * table records S5_ERR_DEVICE_BOUNDS (info = the row) and that row's write is
- * skipped.  batch->max_q and batch->max_len are not used.  Rows are
+ * unmapped page (-1), a page id outside the KV pool (or, with a key pool,
+ * outside the key pool) or a position past the page table records
+ * S5_ERR_DEVICE_BOUNDS (info = the first such row) and that row is skipped.  batch->max_q and batch->max_len are not used.  Rows are
  * independent: positions written by one call must be distinct. */
 s5_status s5_append_kv(const s5_kv_desc *kv, const s5_index_desc *index, const s5_batch_desc *batch,
                        const void *k_new, const void *v_new, const void *key_new, void *workspace,
