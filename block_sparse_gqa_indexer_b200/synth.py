@@ -57,7 +57,7 @@ MAX_TOKENS = 1 << 21
 MAX_BLOCKS = MAX_TOKENS // BLOCK
 
 # tensor ids (one stream per tensor kind, per layer: id + 16 * layer)
-TID_Q, TID_QX, TID_K, TID_V, TID_KX, TID_LEN, TID_PERM, TID_QXN = 1, 2, 3, 4, 5, 6, 7, 8
+TID_Q, TID_QX, TID_K, TID_V, TID_KX, TID_LEN, TID_PERM, TID_QXN, TID_QXG = 1, 2, 3, 4, 5, 6, 7, 8, 9
 
 _M32 = 0xFFFFFFFF
 _M64 = (1 << 64) - 1
@@ -266,6 +266,16 @@ class Workload:
         u = uniform_int(self.seed, self.tid(TID_QXN), idx, 0, 31)
         noise = (u == 0).to(torch.int64) - (u == 1).to(torch.int64)
         return (base + noise).to(torch.bfloat16)
+
+    def qx_group_rows(self, rows: torch.Tensor, device="cpu") -> torch.Tensor:
+        """Per-KV-group indexer queries, bf16 [len(rows)][4][256]: one query per
+        token and KV group, for a selection made separately by each group."""
+        rows = rows.to(device=device, dtype=torch.int64) + self.row_base
+        idx = (rows.view(-1, 1, 1) * N_KV + torch.arange(N_KV, device=device).view(1, -1, 1)) * INDEX_DIM \
+            + torch.arange(INDEX_DIM, device=device).view(1, 1, -1)
+        if self.index_int:
+            return small_int_bf16(self.seed, self.tid(TID_QXG), idx)
+        return normal_bf16(self.seed, self.tid(TID_QXG), idx)
 
     def kx_blocks(self, s: int, blocks: torch.Tensor, device="cpu") -> torch.Tensor:
         """Block keys of sequence s, bf16 [len(blocks)][256]."""

@@ -55,6 +55,14 @@ Readings taken where the pages are silent (each the plainest one):
   (t % 64) // 8 of the same page, when its last token t (t % 8 == 7) arrives,
   since only complete blocks are ever scored.
 
+Per-KV-group selection (the StepFun open-weights blog, section "What sparse
+attention does and doesn't save", has each KV group pick its own blocks):
+reading taken here, since the configuration gives a single 256-wide key per
+block, the block keys are shared and the indexer query differs per group;
+group g's selection is made exactly as the shared one, from group g's query,
+and heads 16g .. 16g+15 attend over group g's selected blocks and the current
+block.
+
 Parity status: the cache append is pinned by rebuilding the seeded pools of
 a whole batch from the pools of its cached prefix;
 block selection is pinned by brute force, tie cases and the
@@ -223,6 +231,28 @@ def swa_attention_query(q, t: int, k_seq, v_seq, window: int = WINDOW, sm_scale:
 # ----------------------------------------------------------------------------
 # batched drivers (varlen batches: per sequence, ctx cached tokens, then nq queries)
 # ----------------------------------------------------------------------------
+
+def index_topk_query_grouped(qx_groups, kx_seq, t: int, topk: int = TOPK) -> np.ndarray:
+    """Per-KV-group selections of one query at t: ``qx_groups`` [4][256] holds
+    one indexer query per KV group; returns [4][topk] (each row as
+    index_topk_query)."""
+    return np.stack([index_topk_query(qx_groups[g], kx_seq, t, topk) for g in range(N_KV)])
+
+
+def sparse_attention_query_grouped(q, sel_groups, t: int, k_seq, v_seq, sm_scale: float = DEFAULT_SM_SCALE):
+    """Sparse-layer attention with a selection per KV group: head h (group
+    g = h // 16) reads the tokens of sel_groups[g] plus the current block.
+    Returns (out [64][192], lse [64])."""
+    out = np.zeros((N_HEADS, HEAD_DIM))
+    lse = np.zeros(N_HEADS)
+    for g in range(N_KV):
+        T = sparse_token_set(sel_groups[g], t)
+        o, l = gqa_attention(q, k_seq[T], v_seq[T], sm_scale)
+        heads = slice(g * HEADS_PER_GROUP, (g + 1) * HEADS_PER_GROUP)
+        out[heads] = o[heads]
+        lse[heads] = l[heads]
+    return out, lse
+
 
 def query_positions(ctx, nq):
     """(sequence, position) of every query row, rows ordered by sequence."""

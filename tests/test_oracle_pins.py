@@ -481,3 +481,60 @@ def test_append_rejects_unmapped_pages():
     bad[4, 2] = -1  # sequence 4 appends positions 130..199: logical pages 2 and 3
     with pytest.raises(ValueError):
         O.append_to_paged_cache(_bits(k0), _bits(v0), None, bad, w.ctx, w.nq, _bits(kn), _bits(vn), None)
+
+
+# ---------------------------------------------------------------- per-KV-group selection
+
+def test_grouped_selection_follows_each_groups_query():
+    # Group g's query is a unit vector on dimension d_g, and exactly the 512
+    # blocks of a known set S_g have a 1 there (0 elsewhere): each group must
+    # select its own S_g, whatever the other dimensions hold.
+    rng = np.random.default_rng(7)
+    c = 700
+    dims = [3, 77, 140, 255]
+    kx = rng.integers(-4, 5, size=(c, 256)).astype(np.float64)
+    qx = np.zeros((4, 256))
+    sets = []
+    for g, d in enumerate(dims):
+        qx[g, d] = 1.0
+        S_g = np.sort(rng.choice(c, 512, replace=False))
+        kx[:, d] = 0.0
+        kx[S_g, d] = 1.0
+        sets.append(S_g)
+    sel = O.index_topk_query_grouped(qx, kx, 8 * c + 5)
+    assert sel.shape == (4, 512)
+    for g in range(4):
+        assert np.array_equal(sel[g], sets[g]), g
+
+
+def test_grouped_attention_routes_heads_to_their_groups_selection():
+    # Zero keys give uniform weights, so head h returns the mean of its
+    # group's values over that group's token set; values encode (position,
+    # group), which pins the token set of each group and the head-to-group map.
+    t = 8 * 40 + 3
+    rng = np.random.default_rng(8)
+    sels = [np.sort(rng.choice(40, 5 + 3 * g, replace=False)) for g in range(4)]
+    k_seq = np.zeros((t + 1, 4, 192))
+    pos = np.arange(t + 1, dtype=np.float64)
+    v_seq = np.zeros((t + 1, 4, 192))
+    for g in range(4):
+        v_seq[:, g, :] = (pos + 1000.0 * g)[:, None]
+    q = rng.standard_normal((64, 192))
+    out, lse = O.sparse_attention_query_grouped(q, sels, t, k_seq, v_seq)
+    for h in range(64):
+        g = h // 16
+        toks = np.concatenate([(sels[g][:, None] * 8 + np.arange(8)).ravel(), np.arange(8 * 40, t + 1)])
+        assert np.allclose(out[h], toks.mean() + 1000.0 * g, rtol=0, atol=1e-9), h
+        assert abs(lse[h] - math.log(len(toks))) < 1e-12
+
+
+def test_grouped_attention_with_equal_selections_is_the_shared_layer():
+    rng = np.random.default_rng(9)
+    t = 8 * 600 + 2
+    k_seq = rng.standard_normal((t + 1, 4, 192))
+    v_seq = rng.standard_normal((t + 1, 4, 192))
+    q = rng.standard_normal((64, 192))
+    sel = np.sort(rng.choice(600, 512, replace=False))
+    o1, l1 = O.sparse_attention_query(q, sel, t, k_seq, v_seq)
+    o4, l4 = O.sparse_attention_query_grouped(q, [sel] * 4, t, k_seq, v_seq)
+    assert np.array_equal(o1, o4) and np.array_equal(l1, l4)

@@ -114,3 +114,18 @@ def test_block_coherent_indexer_queries():
 def test_config6_is_config4_with_coherent_queries():
     (w4,), (w6,) = S.config_workloads(4), S.config_workloads(6)
     assert w6.ctx == w4.ctx and w6.nq == w4.nq and w6.qx_coherent == 64 and w4.qx_coherent == 0
+
+
+def test_grouped_indexer_queries():
+    w = S.Workload(ctx=[100, 9000], nq=[3, 2], seed=5)
+    rows = torch.arange(w.total_q)
+    qg = w.qx_group_rows(rows)
+    assert qg.shape == (5, 4, 256) and qg.dtype == torch.bfloat16
+    v = qg.float()
+    assert torch.equal(v, v.round()) and v.abs().max() <= 4
+    # four different queries per token, and a stream of their own
+    assert not torch.equal(qg[:, 0], qg[:, 1])
+    assert not torch.equal(qg[:, 0], w.qx_rows(rows))
+    # a shard draws the same values for its rows
+    sh = S.shard(w, 1, 2)
+    assert torch.equal(sh.qx_group_rows(torch.arange(sh.total_q)), qg[3:])
