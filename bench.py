@@ -396,7 +396,7 @@ def run_ours(args) -> None:
 
 
 def run_config(args) -> None:
-    """Time one step of numbered configuration `args.config` (1..6) on this GPU and
+    """Time one step of numbered configuration `args.config` (0..6) on this GPU and
     print a JSON line with its own bytes / FLOPs (a measurement aid; the bench
     line is the default mode).  The step and each call are captured in CUDA
     graphs and replayed, so small batches are timed on the device rather than
@@ -434,6 +434,22 @@ def run_config(args) -> None:
             kinds.append("swa")
             bytes_total += R.swa_decode_bytes(w.ctx, w.nq)["total"]
             flops_total += sum(R.attn_flops(R.swa_tokens(c + j)) for c, n in zip(w.ctx, w.nq) for j in range(n))
+        elif args.grouped:
+            # one indexer query and one selection per KV group
+            ws = s5.new_workspace(batch, window=S.WINDOW, device=dev, grouped=True)
+            qxg = w.qx_group_rows(torch.arange(w.total_q), dev).contiguous()
+            sel = torch.empty((w.total_q, S.N_KV, S.TOPK), dtype=torch.int32, device=dev)
+            cnt = torch.empty((w.total_q, S.N_KV), dtype=torch.int32, device=dev)
+            calls.append(lambda kp=key_pool, b=batch, qx=qxg, sel=sel, cnt=cnt, ws=ws:
+                         s5.s5_index_score_topk_grouped(kp, b, qx, S.TOPK, sel, cnt, ws))
+            kinds.append("index_grouped")
+            calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, sel=sel, cnt=cnt, o=out, l=lse, ws=ws:
+                         s5.s5_sparse_gqa_attn_grouped(k, v, b, q, sel, cnt, S.TOPK, scale, o, l, ws))
+            kinds.append("sparse_grouped")
+            # the same KV and key bytes; 4 indexer queries and selections per token
+            extra = w.total_q * (S.N_KV - 1) * (R.index_key_bytes() + 4 * (S.TOPK + 1))
+            bytes_total += R.sparse_decode_bytes(w.ctx, w.nq)["total"] + extra
+            flops_total += R.sparse_flops(w.ctx, w.nq)["attn"] + S.N_KV * R.sparse_flops(w.ctx, w.nq)["index"]
         else:
             sel = torch.empty((w.total_q, S.TOPK), dtype=torch.int32, device=dev)
             cnt = torch.empty((w.total_q,), dtype=torch.int32, device=dev)
@@ -480,7 +496,7 @@ def run_config(args) -> None:
             "algorithmic_bytes": bytes_total, "useful_flops": flops_total,
             "gbs": bytes_total / (ms * 1e-3) / 1e9, "pct_hbm_peak": 100 * bytes_total / (ms * 1e-3) / 1e9 / peak,
             "useful_tflops": flops_total / (ms * 1e-3) / 1e12, "steps": args.steps, "warmup": args.warmup,
-            "append": bool(args.append)}
+            "append": bool(args.append), "grouped": bool(args.grouped)}
     print(json.dumps(line), flush=True)
 
 
@@ -492,17 +508,20 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--batch", type=int, default=64, help="sequences per GPU (64 = the stated workload)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg")
-    ap.add_argument("--config", type=int, default=0, help="time numbered configuration 1..6 instead")
+    ap.add_argument("--config", type=int, default=None,
+                    help="time numbered configuration 0..6 (0: the bench workload) per call instead")
     ap.add_argument("--shard", type=int, default=1, help="with --config: run the first of this many batch shards")
     ap.add_argument("--append", action="store_true",
                     help="with --config: each layer step first appends its new tokens to the cache")
+    ap.add_argument("--grouped", action="store_true",
+                    help="with --config: sparse layers select per KV group (4 indexer queries per token)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         args.steps = min(args.steps, 20)
         run_reference(args)
-    elif args.config:
+    elif args.config is not None:
         run_config(args)
     else:
         run_ours(args)

@@ -71,24 +71,27 @@ struct IndexWs {
   bool two_stage;
 };
 
-IndexWs index_ws(const s5_batch_desc *b) {
+// Indexer scratch for `groups` indexer queries per token (1, or one per KV
+// group): every row below is one (token, group) pair.
+IndexWs index_ws(const s5_batch_desc *b, int groups) {
   IndexWs w{};
+  const size_t rows = (size_t)b->total_q * groups;
   w.stride = (max_blocks(b) + 3) & ~3;  // rows start 16-byte aligned
   w.two_stage = w.stride > kSelCap;
   w.seg = (w.stride <= 16384) ? kSegShort : kSeg;
   w.n_seg = w.two_stage ? (w.stride + w.seg - 1) / w.seg : 0;
   size_t off = kWsFixed;
   w.scores = off;
-  off = align_up(off + (size_t)b->total_q * w.stride * sizeof(float), 256);
+  off = align_up(off + rows * w.stride * sizeof(float), 256);
   w.cand_key = off;
-  off = align_up(off + (size_t)b->total_q * w.n_seg * kMaxTopk * sizeof(uint32_t), 256);
+  off = align_up(off + rows * w.n_seg * kMaxTopk * sizeof(uint32_t), 256);
   w.cand_idx = off;
-  off = align_up(off + (size_t)b->total_q * w.n_seg * kMaxTopk * sizeof(int32_t), 256);
+  off = align_up(off + rows * w.n_seg * kMaxTopk * sizeof(int32_t), 256);
   w.hist = off;
   // the histograms are built by the CUDA-core scoring kernel (not by the tensor-core GEMM)
-  const bool gemm = b->max_q > kGemmMinRows;
-  w.hist_bytes = (!gemm && !w.two_stage && b->total_q <= kMaxHistRows)
-                     ? (size_t)b->total_q * kHistBins * sizeof(uint32_t) : 0;
+  const bool gemm = (long long)b->max_q * groups > kGemmMinRows;
+  w.hist_bytes = (!gemm && !w.two_stage && rows <= (size_t)kMaxHistRows)
+                     ? rows * kHistBins * sizeof(uint32_t) : 0;
   off = align_up(off + w.hist_bytes, 256);
   w.kxs = off;
   w.kxs_bytes = gemm ? (size_t)b->batch * w.stride * kDx * 2 : 0;
@@ -328,7 +331,7 @@ s5_status cuda_status(cudaError_t e) { return e == cudaSuccess ? S5_OK : S5_ERR_
 
 s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, const void *q, const int32_t *sel,
                       const int32_t *sel_count, int32_t topk, int32_t window, float sm_scale, void *out,
-                      float *lse, void *ws, size_t ws_bytes, cudaStream_t stream) {
+                      float *lse, void *ws, size_t ws_bytes, cudaStream_t stream, int sel_groups = 1) {
   s5_status st = check_batch(b);
   if (st != S5_OK) return st;
   if ((st = check_kv(kv)) != S5_OK) return st;
@@ -350,6 +353,7 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   a.q = q;
   a.sel = sel;
   a.sel_count = sel_count;
+  a.sel_groups = sel_groups;
   a.topk = topk;
   a.window = window;
   a.page_table = b->page_table;
@@ -370,7 +374,8 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   a.row_skip = nullptr;
   a.err = reinterpret_cast<int32_t *>(ws);
 
-  if (mode == kModeSparse && use_tiles(b)) {
+  // (one selection per KV group: every row takes the per-row kernel)
+  if (mode == kModeSparse && sel_groups == 1 && use_tiles(b)) {
     // union lists and per-tile choice, then the shared-set tiles; the per-row
     // kernel below skips the rows those tiles computed
     const TileWs tw = tile_ws(b, topk, device_slots() / kCtasPerSm, false, w.end);
@@ -414,16 +419,18 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   return cuda_status(launch_gqa_decode(mode, a, tk, tv, b->total_q, stream));
 }
 
-}  // namespace
-
-extern "C" {
-
-s5_status s5_workspace_size(const s5_batch_desc *batch, int32_t window, size_t *bytes) {
+// Workspace of every call for this batch, with `groups` indexer queries and
+// selections per token (1: shared; 4: one per KV group).
+s5_status workspace_need(const s5_batch_desc *batch, int32_t window, int groups, size_t *bytes) {
   if (bytes == nullptr) return S5_ERR_INVALID_ARG;
   s5_status st = check_batch(batch);
   if (st != S5_OK) return st;
   if (window < 0) return S5_ERR_INVALID_ARG;
-  size_t need = index_ws(batch).end;
+  size_t need = index_ws(batch, 1).end;
+  if (groups > 1) {
+    const size_t ng = index_ws(batch, groups).end;
+    if (ng > need) need = ng;
+  }
   const int slots = kCtasPerSm * kSizingSms;  // an upper bound: no device query here
   size_t sp = attn_ws(batch, sparse_blocks_per_row(kMaxTopk), slots).end;
   if (use_tiles(batch)) sp = tile_ws(batch, kMaxTopk, kSizingSms, true, sp).end;
@@ -436,9 +443,11 @@ s5_status s5_workspace_size(const s5_batch_desc *batch, int32_t window, size_t *
   return S5_OK;
 }
 
-s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *batch, const void *q_index,
-                              int32_t topk, int32_t *sel, int32_t *sel_count, void *workspace,
-                              size_t workspace_bytes, s5_stream_t stream) {
+// Block scores and top-k for `groups` indexer queries per token: q_index
+// [total_q][groups][256], one selection per (token, group) row.
+s5_status index_common(const s5_index_desc *index, const s5_batch_desc *batch, const void *q_index, int32_t topk,
+                       int32_t *sel, int32_t *sel_count, void *workspace, size_t workspace_bytes,
+                       s5_stream_t stream, int groups) {
   s5_status st = check_batch(batch);
   if (st != S5_OK) return st;
   if (index == nullptr || index->key_pool == nullptr || index->num_pages < 1) return S5_ERR_INVALID_ARG;
@@ -449,7 +458,9 @@ s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *b
   if (batch->total_q == 0) return S5_OK;
   if (q_index == nullptr || sel == nullptr || sel_count == nullptr || !aligned16(q_index))
     return S5_ERR_INVALID_ARG;
-  const IndexWs w = index_ws(batch);
+  const long long rows = (long long)batch->total_q * groups;
+  const IndexWs w = index_ws(batch, groups);
+  if (w.two_stage && rows > 65535) return S5_ERR_UNSUPPORTED;  // stage 1 has one grid row per selection
   if (workspace_bytes < w.end) return S5_ERR_WORKSPACE;
   uint8_t *wsb = static_cast<uint8_t *>(workspace);
   int32_t *err = reinterpret_cast<int32_t *>(workspace);
@@ -465,6 +476,7 @@ s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *b
   ia.batch = batch->batch;
   ia.total_q = batch->total_q;
   ia.q_index = q_index;
+  ia.q_groups = groups;
   ia.scores = reinterpret_cast<float *>(wsb + w.scores);
   ia.score_stride = w.stride;
   ia.pages_per_cta = kScorePagesPerCta;
@@ -483,24 +495,25 @@ s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *b
     ga.max_blocks = w.stride;
     if (launch_gather_keys(ga, batch->batch, cs) != cudaSuccess) return S5_ERR_CUDA;
     CUtensorMap tq, tk;
-    if (!make_k256_map(&tq, q_index, batch->total_q) ||
-        !make_k256_map(&tk, ga.kxs, (long long)batch->batch * w.stride))
+    if (!make_k256_map(&tq, q_index, rows) || !make_k256_map(&tk, ga.kxs, (long long)batch->batch * w.stride))
       return S5_ERR_CUDA;
     GemmArgs gm{};
     gm.ctx_lens = batch->ctx_lens;
     gm.cu_q = batch->cu_q;
     gm.batch = batch->batch;
     gm.total_q = batch->total_q;
+    gm.q_groups = groups;
     gm.scores = ia.scores;
     gm.score_stride = w.stride;
     gm.max_blocks = w.stride;
     gm.tiles_per_cta = kGemmTilesPerCta;
     gm.err = err;
-    if (launch_index_gemm(gm, tq, tk, batch->batch, batch->max_q, cs) != cudaSuccess) return S5_ERR_CUDA;
+    if (launch_index_gemm(gm, tq, tk, batch->batch, batch->max_q * groups, cs) != cudaSuccess) return S5_ERR_CUDA;
   } else {
     const int pages = (w.stride + kBpp - 1) / kBpp;
     const int grid_pages = (pages + kScorePagesPerCta - 1) / kScorePagesPerCta;
-    if (launch_index_score(ia, batch->max_q, grid_pages, batch->batch, cs) != cudaSuccess) return S5_ERR_CUDA;
+    if (launch_index_score(ia, batch->max_q * groups, grid_pages, batch->batch, cs) != cudaSuccess)
+      return S5_ERR_CUDA;
   }
 
   SelectArgs sa{};
@@ -510,6 +523,7 @@ s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *b
   sa.cu_q = batch->cu_q;
   sa.batch = batch->batch;
   sa.total_q = batch->total_q;
+  sa.q_groups = groups;
   sa.topk = topk;
   sa.sel = sel;
   sa.sel_count = sel_count;
@@ -519,7 +533,31 @@ s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *b
   sa.cand_idx = reinterpret_cast<int32_t *>(wsb + w.cand_idx);
   sa.hist = ia.hist;
   sa.err = err;
-  return cuda_status(launch_topk_select(sa, batch->total_q, w.two_stage, cs));
+  return cuda_status(launch_topk_select(sa, (int)rows, w.two_stage, cs));
+}
+
+}  // namespace
+
+extern "C" {
+
+s5_status s5_workspace_size(const s5_batch_desc *batch, int32_t window, size_t *bytes) {
+  return workspace_need(batch, window, 1, bytes);
+}
+
+s5_status s5_workspace_size_grouped(const s5_batch_desc *batch, int32_t window, size_t *bytes) {
+  return workspace_need(batch, window, kKv, bytes);
+}
+
+s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *batch, const void *q_index,
+                              int32_t topk, int32_t *sel, int32_t *sel_count, void *workspace,
+                              size_t workspace_bytes, s5_stream_t stream) {
+  return index_common(index, batch, q_index, topk, sel, sel_count, workspace, workspace_bytes, stream, 1);
+}
+
+s5_status s5_index_score_topk_grouped(const s5_index_desc *index, const s5_batch_desc *batch, const void *q_index,
+                                      int32_t topk, int32_t *sel, int32_t *sel_count, void *workspace,
+                                      size_t workspace_bytes, s5_stream_t stream) {
+  return index_common(index, batch, q_index, topk, sel, sel_count, workspace, workspace_bytes, stream, kKv);
 }
 
 s5_status s5_sparse_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, const void *q, const int32_t *sel,
@@ -527,6 +565,14 @@ s5_status s5_sparse_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, c
                              void *workspace, size_t workspace_bytes, s5_stream_t stream) {
   return attn_common(kModeSparse, kv, batch, q, sel, sel_count, topk, 0, sm_scale, out, lse, workspace,
                      workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+s5_status s5_sparse_gqa_attn_grouped(const s5_kv_desc *kv, const s5_batch_desc *batch, const void *q,
+                                     const int32_t *sel, const int32_t *sel_count, int32_t topk, float sm_scale,
+                                     void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                     s5_stream_t stream) {
+  return attn_common(kModeSparse, kv, batch, q, sel, sel_count, topk, 0, sm_scale, out, lse, workspace,
+                     workspace_bytes, reinterpret_cast<cudaStream_t>(stream), kKv);
 }
 
 s5_status s5_swa_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, const void *q, int32_t window,

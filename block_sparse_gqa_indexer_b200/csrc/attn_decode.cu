@@ -140,7 +140,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   pdl_wait();
   if (a.row_skip != nullptr && ld_cg(a.row_skip + r) != 0) return;  // row computed by the tile kernel
   int s = -1, t = -1, lo_tok = 0, n_list = 0, b_first = 0, n_sel = 0;
-  const int sel_cnt = (MODE == kModeSparse) ? ld_cg(a.sel_count + r) : 0;
+  // the selection this unit reads: the row's, or its KV group's (sel_groups = 4)
+  const int srow = a.sel_groups > 1 ? r * a.sel_groups + g : r;
+  const int sel_cnt = (MODE == kModeSparse) ? ld_cg(a.sel_count + srow) : 0;
   bool bad = !locate_row(a.cu_q, a.ctx_lens, a.batch, r, row_guess(r, a.batch, a.total_q), s, t);
   if (!bad) bad = (t < 0) || (t >= a.max_pages * kPage) || (t >= a.max_len);
   const int c = bad ? 0 : t / kBlk;
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     }
   }
   if (bad) {
-    if (tid == 0 && p == 0 && g == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
+    if (tid == 0 && p == 0 && (g == 0 || a.sel_groups > 1)) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
     n_list = 0;
   }
   int chunk = (n_list + a.n_split - 1) / a.n_split;
@@ -212,7 +214,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     bool ok = true;
     if (MODE == kModeSparse) {
       if (li < n_sel) {
-        b = ld_cg(a.sel + (size_t)r * a.topk + li);
+        b = ld_cg(a.sel + (size_t)srow * a.topk + li);
         ok = (b >= 0) && (b < c);
       } else {
         b = c;

@@ -85,14 +85,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
   const int q_beg = ld_cg(a.cu_q + s);
   const int nq = ld_cg(a.cu_q + s + 1) - q_beg;
   const int ctx = ld_cg(a.ctx_lens + s);
+  // indexer rows of the sequence: token-major, G queries per token (G = 1, or
+  // one per KV group); row m of the sequence belongs to its token m / G
+  const int G = a.q_groups > 1 ? a.q_groups : 1;
   const int m0 = blockIdx.y * kGM;
-  if (nq <= 0 || m0 >= nq) return;
-  const int rows = min(kGM, nq - m0);
-  const int c_last = (ctx + m0 + rows - 1) / kBlk;  // history blocks of the tile's last row
+  if (nq <= 0 || m0 >= nq * G) return;
+  const int rows = min(kGM, nq * G - m0);
+  const int c_last = (ctx + (m0 + rows - 1) / G) / kBlk;  // history blocks of the tile's last row
   if (q_beg < 0 || q_beg + nq > a.total_q || ctx < 0 || c_last > a.score_stride || c_last > a.max_blocks) {
-    if (tid == 0 && blockIdx.x == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, max(q_beg, 0) + m0);
+    if (tid == 0 && blockIdx.x == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, max(q_beg, 0) + m0 / G);
     return;
   }
+  const int row0 = q_beg * G + m0;  // first indexer row of the tile
   const int j_beg = blockIdx.x * a.tiles_per_cta;
   const int j_end = min(j_beg + a.tiles_per_cta, (c_last + kGN - 1) / kGN);
   const int nt = j_end - j_beg;
@@ -120,7 +124,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
     if (mbar_wait_bounded(bar, parity, kGWaitNs)) return true;
     *reinterpret_cast<volatile int *>(abort_flag) = 1;
-    record_error(a.err, S5_ERR_TIMEOUT, q_beg + m0);
+    record_error(a.err, S5_ERR_TIMEOUT, q_beg + m0 / G);
     return false;
   };
 
@@ -128,7 +132,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_a, kGOperand);
-      for (int kb = 0; kb < kGKb; ++kb) tma_load_2d(sa + kb * kGTileBytes, &tm_q, kb * 64, q_beg + m0, bar_a);
+      for (int kb = 0; kb < kGKb; ++kb) tma_load_2d(sa + kb * kGTileBytes, &tm_q, kb * 64, row0, bar_a);
       int issued = 0;
       for (int jj = 0; jj < nt; ++jj) {
         const int st = jj % kGStages;
@@ -175,8 +179,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
   } else {
     // ---------------- epilogue: warps 0-3, TMEM lanes 32w .. 32w+31 ----------------
     const int row = warp * 32 + lane;
-    const int grow = q_beg + m0 + row;
-    const int c_row = (row < rows) ? (ctx + m0 + row) / kBlk : 0;
+    const int grow = row0 + row;
+    const int c_row = (row < rows) ? (ctx + (m0 + row) / G) / kBlk : 0;
     float *dst_row = a.scores + (size_t)grow * a.score_stride;
     for (int jj = 0; jj < nt; ++jj) {
       const int db = jj % 2;

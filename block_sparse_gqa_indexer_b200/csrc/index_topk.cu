@@ -43,7 +43,9 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&vals)[1 << LOGV], in
   for (int off = 16 >> LOGV; off >= 1; off >>= 1) vals[0] += __shfl_xor_sync(0xffffffffu, vals[0], off);
 }
 
-template <int QT, int UNROLL>
+// GROUPED: a.q_groups indexer queries per token (one per KV group), rows
+// token-major; otherwise one query per token.
+template <int QT, int UNROLL, bool GROUPED>
 __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
   constexpr int LOGV = (QT == 1) ? 3 : (QT == 2) ? 4 : 5;
   constexpr int V = 1 << LOGV;  // 8 blocks x QT queries
@@ -58,13 +60,16 @@ __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
     if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, s);
     return;
   }
-  if (tile0 >= nq_s) return;
-  const int nq = min(QT, nq_s - tile0);
+  // indexer rows of the sequence: token-major, G queries per token (G = 1, or
+  // one per KV group); row q of the sequence belongs to its token q / G
+  const int G = GROUPED ? a.q_groups : 1;
+  if (tile0 >= nq_s * G) return;
+  const int nq = min(QT, nq_s * G - tile0);
   const int ctx = __ldg(a.ctx_lens + s);
-  const int t_last = ctx + tile0 + nq - 1;
+  const int t_last = GROUPED ? ctx + (tile0 + nq - 1) / G : ctx + tile0 + nq - 1;
   const int c_hi = t_last / kBlk;  // history blocks of the last query in the tile
   if (ctx < 0 || t_last >= a.max_pages * kPage || c_hi > a.score_stride) {
-    if (threadIdx.x == 0 && blockIdx.x == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, q_beg + tile0);
+    if (threadIdx.x == 0 && blockIdx.x == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, q_beg + tile0 / G);
     return;
   }
   if (c_hi <= a.topk) return;  // every row of the tile keeps all its history blocks
@@ -77,7 +82,7 @@ __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
 #pragma unroll
   for (int qi = 0; qi < QT; ++qi) {
     uint4 w = make_uint4(0, 0, 0, 0);
-    if (qi < nq) w = __ldg(reinterpret_cast<const uint4 *>(a.q_index) + (size_t)(q_beg + tile0 + qi) * (kDx / 8) + lane);
+    if (qi < nq) w = __ldg(reinterpret_cast<const uint4 *>(a.q_index) + (size_t)(q_beg * G + tile0 + qi) * (kDx / 8) + lane);
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -102,7 +107,7 @@ __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
         if (ph >= 0 && ph < a.num_pages) {
           phys[u] = ph;
         } else if (lane == 0) {
-          record_error(a.err, S5_ERR_DEVICE_BOUNDS, q_beg + tile0);
+          record_error(a.err, S5_ERR_DEVICE_BOUNDS, q_beg + tile0 / G);
         }
       }
 #pragma unroll
@@ -141,8 +146,9 @@ __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
         const int qi = v / kBpp;
         const int j = v % kBpp;
         const int b = pp * kBpp + j;
-        if (qi < nq && b < (ctx + tile0 + qi) / kBlk) {
-          const size_t row = (size_t)(q_beg + tile0 + qi);
+        const int t_q = GROUPED ? ctx + (tile0 + qi) / G : ctx + tile0 + qi;  // position of the row's token
+        if (qi < nq && b < t_q / kBlk) {
+          const size_t row = (size_t)(q_beg * G + tile0 + qi);
           const float sc = (phys[u] >= 0) ? vals[0] : __int_as_float(0xff800000);  // -inf: unreadable page
           a.scores[row * a.score_stride + b] = sc;
           if (a.hist != nullptr) atomicAdd(a.hist + row * kHistBins + (score_key(sc) >> 20), 1u);
@@ -312,10 +318,15 @@ __device__ __forceinline__ void load_keys(const float *row, int n, int E, uint32
   }
 }
 
-// Query row -> (history blocks c).  Returns false on bad batch data.
+// Selection row -> (history blocks c) of its token: r, or r / 4 with one
+// selection per KV group (a.q_groups = 4; looked at only when GROUPED).
+// Returns false on bad batch data.
+template <bool GROUPED = true>
 __device__ __forceinline__ bool row_history(const SelectArgs &a, int r, int &c) {
+  static_assert(kKv == 4, "rows of per-group selections map to tokens by a shift");
   int s, t;
-  if (!locate_row(a.cu_q, a.ctx_lens, a.batch, r, row_guess(r, a.batch, a.total_q), s, t)) return false;
+  const int tok = GROUPED ? r >> (a.q_groups > 1 ? 2 : 0) : r;
+  if (!locate_row(a.cu_q, a.ctx_lens, a.batch, tok, row_guess(tok, a.batch, a.total_q), s, t)) return false;
   if (t < 0 || t / kBlk > a.score_stride) return false;
   c = t / kBlk;
   return true;
@@ -376,7 +387,7 @@ __device__ __forceinline__ void find_bin_desc(const uint32_t (&c)[NB], int top, 
 // every key in registers (short launches: one CTA per row of a decode batch),
 // 2 caps registers at 32 per thread so that batches of many rows (prefill)
 // run twice as many rows at a time.
-template <int NT, int EMAX, bool WARP_REFINE, int MINB>
+template <int NT, int EMAX, bool WARP_REFINE, int MINB, bool GROUPED>
 __global__ void __launch_bounds__(NT, MINB) topk_select_hist_kernel(SelectArgs a) {
   static_assert(NT == 512 || NT == 1024, "row-histogram and refinement bins are split evenly over threads");
   constexpr int NB1 = kHistBins / NT;  // row-histogram bins per thread
@@ -389,7 +400,7 @@ __global__ void __launch_bounds__(NT, MINB) topk_select_hist_kernel(SelectArgs a
   pdl_trigger();
   pdl_wait();  // every input (batch data, scores, histograms) is read after this point
   int c = 0;
-  const bool row_ok = row_history(a, r, c) && c <= NT * EMAX;
+  const bool row_ok = row_history<GROUPED>(a, r, c) && c <= NT * EMAX;
   // this thread's row-histogram bins, top first: 4095 - NB1*t .. (loaded with the keys)
   uint32_t cc1[NB1];
   if (a.hist != nullptr) {
@@ -584,12 +595,20 @@ __global__ void __launch_bounds__(NT) topk_merge_kernel(SelectArgs a) {
 // launchers
 // ============================================================================
 
+// max_q: indexer rows of the longest sequence (tokens x queries per token).
 cudaError_t launch_index_score(const IndexScoreArgs &a, int max_q, int grid_pages, int n_seq, cudaStream_t st) {
   const int qt = (max_q <= 1) ? 1 : (max_q <= 2) ? 2 : 4;
   dim3 grid(grid_pages, n_seq, (max_q + qt - 1) / qt);
-  if (qt == 1) index_score_kernel<1, 2><<<grid, 256, 0, st>>>(a);
-  else if (qt == 2) index_score_kernel<2, 2><<<grid, 256, 0, st>>>(a);
-  else index_score_kernel<4, 1><<<grid, 256, 0, st>>>(a);
+  if (a.q_groups > 1) {
+    if (qt != 4) return cudaErrorInvalidValue;  // >= 4 rows per token
+    index_score_kernel<4, 1, true><<<grid, 256, 0, st>>>(a);
+  } else if (qt == 1) {
+    index_score_kernel<1, 2, false><<<grid, 256, 0, st>>>(a);
+  } else if (qt == 2) {
+    index_score_kernel<2, 2, false><<<grid, 256, 0, st>>>(a);
+  } else {
+    index_score_kernel<4, 1, false><<<grid, 256, 0, st>>>(a);
+  }
   return cudaGetLastError();
 }
 
@@ -616,9 +635,14 @@ cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, cudaStrea
 
 cudaError_t launch_topk_select(const SelectArgs &a, int total_q, bool two_stage, cudaStream_t st) {
   if (!two_stage) {  // with a row histogram from the scoring kernel, or one built in shared memory
-    if (total_q > 1024)
-      return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 2>, dim3(total_q), dim3(kSelThreads), st, a);
-    return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 1>, dim3(total_q), dim3(kSelThreads), st, a);
+    const dim3 grid(total_q), block(kSelThreads);
+    if (a.q_groups > 1) {
+      if (total_q > 1024)
+        return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 2, true>, grid, block, st, a);
+      return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 1, true>, grid, block, st, a);
+    }
+    if (total_q > 1024) return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 2, false>, grid, block, st, a);
+    return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 1, false>, grid, block, st, a);
   }
   cudaError_t e = launch_pdl(topk_segment_kernel<kSegThreads, 32>, dim3(a.n_seg, total_q), dim3(kSegThreads), st, a);
   if (e != cudaSuccess) return e;

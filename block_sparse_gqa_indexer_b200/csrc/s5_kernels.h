@@ -21,13 +21,14 @@ struct IndexScoreArgs {
   const int32_t *cu_q;
   int batch;
   int total_q;
-  const void *q_index;
-  float *scores;     // [total_q][score_stride]
+  const void *q_index;  // bf16 [total_q][q_groups][256]
+  float *scores;     // [total_q * q_groups][score_stride]
   int score_stride;  // >= history blocks of any row
   int pages_per_cta;
   int topk;
-  uint32_t *hist;  // [total_q][4096] counts of score keys by their top 12 bits (zeroed before), or null
+  uint32_t *hist;  // [total_q * q_groups][4096] counts of score keys by their top 12 bits (zeroed before), or null
   int32_t *err;
+  int q_groups;  // indexer queries per token (0 or 1: one shared query; 4: one per KV group)
 };
 
 constexpr int kHistBins = 4096;  // row histogram of the top 12 bits of the score keys
@@ -40,8 +41,8 @@ struct SelectArgs {
   int batch;
   int total_q;
   int topk;
-  int32_t *sel;
-  int32_t *sel_count;
+  int32_t *sel;        // [total_q * q_groups][topk]
+  int32_t *sel_count;  // [total_q * q_groups]
   // two-stage select
   int seg;    // blocks per segment
   int n_seg;  // segments per row (stride of the candidate arrays)
@@ -49,12 +50,14 @@ struct SelectArgs {
   int32_t *cand_idx;
   const uint32_t *hist;  // row histograms built by the scoring kernel, or null
   int32_t *err;
+  int q_groups;  // selections per token: 0 or 1, or 4 (row r belongs to token r / 4)
 };
 
 struct AttnArgs {
   const void *q;
-  const int32_t *sel;
-  const int32_t *sel_count;
+  const int32_t *sel;        // [total_q][sel_groups][topk]
+  const int32_t *sel_count;  // [total_q][sel_groups]
+  int sel_groups;            // 0 or 1: one selection per token; 4: one per KV group
   int topk;
   int window;
   const int32_t *page_table;
@@ -91,7 +94,8 @@ struct GemmArgs {
   const int32_t *cu_q;
   int batch;
   int total_q;
-  float *scores;  // [total_q][score_stride]
+  int q_groups;   // indexer queries per token (0 or 1, or 4); rows token-major, group-minor
+  float *scores;  // [total_q * q_groups][score_stride]
   int score_stride;
   int max_blocks;     // rows per sequence of the gathered keys
   int tiles_per_cta;  // 128-block N tiles per CTA

@@ -30,6 +30,7 @@ S5_OK, S5_ERR_INVALID_ARG, S5_ERR_UNSUPPORTED, S5_ERR_CUDA, S5_ERR_DEVICE_BOUNDS
 
 # exported symbols (every declaration of include/s5attn.h)
 SYMBOLS = ("s5_workspace_size", "s5_index_score_topk", "s5_sparse_gqa_attn", "s5_swa_gqa_attn",
+           "s5_workspace_size_grouped", "s5_index_score_topk_grouped", "s5_sparse_gqa_attn_grouped",
            "s5_index_score_topk_noalloc", "s5_append_kv", "s5_reset_device_error", "s5_get_device_error",
            "s5_status_string", "s5_abi_version")
 
@@ -58,6 +59,9 @@ _lib.s5_sparse_gqa_attn.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(Batch
                                     ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.s5_swa_gqa_attn.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(BatchDesc), _P, _I, ctypes.c_float, _P,
                                  _P, _P, ctypes.c_size_t, _P]
+_lib.s5_workspace_size_grouped.argtypes = _lib.s5_workspace_size.argtypes
+_lib.s5_index_score_topk_grouped.argtypes = _lib.s5_index_score_topk.argtypes
+_lib.s5_sparse_gqa_attn_grouped.argtypes = _lib.s5_sparse_gqa_attn.argtypes
 _lib.s5_index_score_topk_noalloc.argtypes = [ctypes.POINTER(IndexDesc), ctypes.POINTER(BatchDesc), _P, _I, _P,
                                              _P, _P]
 _lib.s5_append_kv.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(IndexDesc), ctypes.POINTER(BatchDesc), _P, _P,
@@ -145,9 +149,18 @@ def s5_workspace_size(batch: Batch, window: int = 0) -> int:
     return int(n.value)
 
 
-def new_workspace(batch: Batch, window: int = 0, device="cuda") -> torch.Tensor:
-    """Allocate (with torch) and zero a workspace sized for ``batch``."""
-    return torch.zeros(max(256, s5_workspace_size(batch, window)), dtype=torch.uint8, device=device)
+def s5_workspace_size_grouped(batch: Batch, window: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.s5_workspace_size_grouped(ctypes.byref(batch.desc), int(window), ctypes.byref(n)),
+           "s5_workspace_size_grouped")
+    return int(n.value)
+
+
+def new_workspace(batch: Batch, window: int = 0, device="cuda", grouped: bool = False) -> torch.Tensor:
+    """Allocate (with torch) and zero a workspace sized for ``batch`` (with
+    ``grouped``, also for the per-KV-group selection calls)."""
+    n = s5_workspace_size_grouped(batch, window) if grouped else s5_workspace_size(batch, window)
+    return torch.zeros(max(256, n), dtype=torch.uint8, device=device)
 
 
 def s5_index_score_topk(key_pool: torch.Tensor, batch: Batch, q_index: torch.Tensor, topk: int,
@@ -161,6 +174,21 @@ def s5_index_score_topk(key_pool: torch.Tensor, batch: Batch, q_index: torch.Ten
     _check(_lib.s5_index_score_topk(ctypes.byref(idx), ctypes.byref(batch.desc), _ptr(q_index), int(topk),
                                     _ptr(sel), _ptr(sel_count), _ptr(ws), ws.numel(), _stream(stream)),
            "s5_index_score_topk")
+
+
+def s5_index_score_topk_grouped(key_pool: torch.Tensor, batch: Batch, q_index: torch.Tensor, topk: int,
+                                sel: torch.Tensor, sel_count: torch.Tensor, ws: torch.Tensor, stream=None):
+    """One selection per (token, KV group): q_index [total_q][4][256] ->
+    sel [total_q][4][topk], sel_count [total_q][4]."""
+    _need(key_pool, torch.bfloat16, "key_pool")
+    _need(q_index, torch.bfloat16, "q_index", (batch.total_q, N_KV, INDEX_DIM))
+    _need(sel, torch.int32, "sel", (batch.total_q, N_KV, topk))
+    _need(sel_count, torch.int32, "sel_count", (batch.total_q, N_KV))
+    _need(ws, torch.uint8, "ws")
+    idx = IndexDesc(key_pool.data_ptr(), key_pool.shape[0], key_pool.shape[-1])
+    _check(_lib.s5_index_score_topk_grouped(ctypes.byref(idx), ctypes.byref(batch.desc), _ptr(q_index), int(topk),
+                                            _ptr(sel), _ptr(sel_count), _ptr(ws), ws.numel(), _stream(stream)),
+           "s5_index_score_topk_grouped")
 
 
 def s5_index_score_topk_noalloc(key_pool: torch.Tensor, batch: Batch, q_index: torch.Tensor, topk: int,
@@ -198,6 +226,22 @@ def s5_sparse_gqa_attn(k_pool, v_pool, batch: Batch, q, sel, sel_count, topk: in
     _check(_lib.s5_sparse_gqa_attn(ctypes.byref(kv), ctypes.byref(batch.desc), _ptr(q), _ptr(sel),
                                    _ptr(sel_count), int(topk), float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws),
                                    ws.numel(), _stream(stream)), "s5_sparse_gqa_attn")
+
+
+def s5_sparse_gqa_attn_grouped(k_pool, v_pool, batch: Batch, q, sel, sel_count, topk: int, sm_scale: float,
+                               out, lse, ws, stream=None):
+    """Sparse attention with one selection per KV group (sel [total_q][4][topk])."""
+    kv = _kv(k_pool, v_pool)
+    _need(q, torch.bfloat16, "q", (batch.total_q, N_HEADS, HEAD_DIM))
+    _need(sel, torch.int32, "sel", (batch.total_q, N_KV, topk))
+    _need(sel_count, torch.int32, "sel_count", (batch.total_q, N_KV))
+    _need(out, torch.bfloat16, "out", (batch.total_q, N_HEADS, HEAD_DIM))
+    if lse is not None:
+        _need(lse, torch.float32, "lse", (batch.total_q, N_HEADS))
+    _need(ws, torch.uint8, "ws")
+    _check(_lib.s5_sparse_gqa_attn_grouped(ctypes.byref(kv), ctypes.byref(batch.desc), _ptr(q), _ptr(sel),
+                                           _ptr(sel_count), int(topk), float(sm_scale), _ptr(out), _ptr(lse),
+                                           _ptr(ws), ws.numel(), _stream(stream)), "s5_sparse_gqa_attn_grouped")
 
 
 def s5_swa_gqa_attn(k_pool, v_pool, batch: Batch, q, window: int, sm_scale: float, out, lse, ws, stream=None):

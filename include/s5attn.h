@@ -166,6 +166,33 @@ s5_status s5_swa_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, cons
                           int32_t window, float sm_scale, void *out, float *lse,
                           void *workspace, size_t workspace_bytes, s5_stream_t stream);
 
+/* Per-KV-group selection (StepFun open-weights blog, "What sparse attention
+ * does and doesn't save": each KV group picks its own blocks).  The block
+ * keys stay shared (the configuration gives one 256-wide key per block); the
+ * indexer query differs per group, so each token carries 4 queries and gets
+ * 4 selections, and the heads of group g attend over group g's blocks.
+ *
+ * s5_index_score_topk_grouped: as s5_index_score_topk for every (token,
+ * group) pair, each key read once for all four.
+ *   q_index    device bf16 [total_q][4][256]: the query of token r, group g
+ *   sel        device int32 [total_q][4][topk], sel_count [total_q][4]
+ * s5_sparse_gqa_attn_grouped: as s5_sparse_gqa_attn, with head h (group
+ * g = h / 16) reading sel[r][g][0 .. sel_count[r][g] - 1] plus the current
+ * block.  Every row takes the per-row kernel (the shared-set tiles assume one
+ * selection per token).
+ * s5_workspace_size_grouped: a workspace size that covers these two calls as
+ * well as every call s5_workspace_size covers.
+ * Limits: selections of more than 16,384 history blocks need
+ * 4 * total_q <= 65,535 (else S5_ERR_UNSUPPORTED). */
+s5_status s5_workspace_size_grouped(const s5_batch_desc *batch, int32_t window, size_t *bytes);
+s5_status s5_index_score_topk_grouped(const s5_index_desc *index, const s5_batch_desc *batch,
+                                      const void *q_index, int32_t topk, int32_t *sel, int32_t *sel_count,
+                                      void *workspace, size_t workspace_bytes, s5_stream_t stream);
+s5_status s5_sparse_gqa_attn_grouped(const s5_kv_desc *kv, const s5_batch_desc *batch, const void *q,
+                                     const int32_t *sel, const int32_t *sel_count, int32_t topk, float sm_scale,
+                                     void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                     s5_stream_t stream);
+
 /* s5_index_score_topk without a workspace.  The pages have no counterpart to
  * this entry point: it exists for callers that cannot allocate device memory
  * at all, such as code embedded in a host framework that owns every device

@@ -147,3 +147,30 @@ def test_append_rejects_bad_arguments_before_launch(s5):
     # nothing to append: OK with nothing enqueued (null rows allowed)
     assert ap(ctypes.byref(kv), ctypes.byref(ix), ctypes.byref(_batch(total_q=0)), None, None, None, fake, big,
               None) == s5.S5_OK
+
+
+def test_grouped_workspace_and_limits(s5):
+    # one selection per KV group: four score rows per token
+    n1, n4 = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    b = _batch(batch=64, total_q=64, max_q=1, max_pages=2049, max_len=131073)
+    assert s5._lib.s5_workspace_size(ctypes.byref(b), 0, ctypes.byref(n1)) == 0
+    assert s5._lib.s5_workspace_size_grouped(ctypes.byref(b), 0, ctypes.byref(n4)) == 0
+    assert n4.value >= 256 + 16384 + 4 * 64 * 16384 * 4
+    assert n4.value >= n1.value
+    # small histories with many rows: the shared call's histograms may need more
+    # than the grouped scores; the grouped size still covers every call
+    b = _batch(batch=2, total_q=512, max_q=256, max_pages=20, max_len=1200)
+    assert s5._lib.s5_workspace_size(ctypes.byref(b), 512, ctypes.byref(n1)) == 0
+    assert s5._lib.s5_workspace_size_grouped(ctypes.byref(b), 512, ctypes.byref(n4)) == 0
+    assert n4.value >= n1.value
+    fake = ctypes.c_void_p(0x1000)
+    ix = s5.IndexDesc(0x1000, 8, 256)
+    # selections over more than 16,384 blocks: at most 65,535 (token, group) rows
+    big = _batch(batch=1, total_q=20000, max_q=20000, max_pages=32768, max_len=(1 << 21))
+    assert s5._lib.s5_index_score_topk_grouped(ctypes.byref(ix), ctypes.byref(big), fake, 512, fake, fake, fake,
+                                               1 << 40, None) == s5.S5_ERR_UNSUPPORTED
+    kv = s5.KvDesc(0x1000, 0x1000, 8, 64, 4, 192)
+    assert s5._lib.s5_sparse_gqa_attn_grouped(ctypes.byref(kv), ctypes.byref(_batch()), fake, None, fake, 512, 0.1,
+                                              fake, None, fake, 1 << 30, None) == s5.S5_ERR_INVALID_ARG
+    assert s5._lib.s5_index_score_topk_grouped(ctypes.byref(ix), ctypes.byref(_batch()), fake, 512, fake, fake,
+                                               None, 1 << 30, None) == s5.S5_ERR_WORKSPACE
