@@ -130,6 +130,12 @@ def normal_bf16(seed: int, tensor_id: int, idx: torch.Tensor) -> torch.Tensor:
     return f.to(torch.bfloat16)
 
 
+def to_e4m3_codes(x: torch.Tensor) -> torch.Tensor:
+    """One-byte E4M3 codes (uint8) of the values of x, rounded by torch's
+    float8_e4m3fn conversion (exact for integers of magnitude <= 16)."""
+    return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
 def small_int_bf16(seed: int, tensor_id: int, idx: torch.Tensor, lim: int = 4) -> torch.Tensor:
     """Integer-valued bf16 in [-lim, lim] (exact in bf16)."""
     return uniform_int(seed, tensor_id, idx, -lim, lim).to(torch.bfloat16)
@@ -277,13 +283,16 @@ class Workload:
             return small_int_bf16(self.seed, self.tid(TID_QXG), idx)
         return normal_bf16(self.seed, self.tid(TID_QXG), idx)
 
-    def kx_blocks(self, s: int, blocks: torch.Tensor, device="cpu") -> torch.Tensor:
-        """Block keys of sequence s, bf16 [len(blocks)][256]."""
+    def kx_blocks(self, s: int, blocks: torch.Tensor, device="cpu", fp8: bool = False) -> torch.Tensor:
+        """Block keys of sequence s, bf16 [len(blocks)][256]; with ``fp8``, the
+        same values as one-byte E4M3 codes, uint8 [len(blocks)][256]."""
         blocks = blocks.to(device=device, dtype=torch.int64)
         idx = ((self.seq_base + s) * MAX_BLOCKS + blocks.view(-1, 1)) * INDEX_DIM + torch.arange(INDEX_DIM, device=device).view(1, -1)
         if self.index_int:
-            return small_int_bf16(self.seed, self.tid(TID_KX), idx)
-        return normal_bf16(self.seed, self.tid(TID_KX), idx)
+            vals = small_int_bf16(self.seed, self.tid(TID_KX), idx)
+        else:
+            vals = normal_bf16(self.seed, self.tid(TID_KX), idx)
+        return to_e4m3_codes(vals) if fp8 else vals
 
     def _kv_tokens(self, tid: int, s: int, pos: torch.Tensor, device) -> torch.Tensor:
         pos = pos.to(device=device, dtype=torch.int64)
@@ -357,10 +366,14 @@ class Workload:
         return k_pool, v_pool
 
     def index_pool(self, device, pt: Optional[torch.Tensor] = None, pages_per_chunk: int = 16384,
-                   upto: Optional[Sequence[int]] = None):
+                   upto: Optional[Sequence[int]] = None, fp8: bool = False):
         """Block-key pool, bf16 [num_pages][8][256]; slot j of page p holds the key
         of block 8 * (logical page) + j.  Only complete blocks carry a key: those
-        that end at or below ``upto[s]`` tokens (default: the whole sequence)."""
+        that end at or below ``upto[s]`` tokens (default: the whole sequence).
+        With ``fp8`` the pool holds the same keys as one-byte E4M3 codes (uint8;
+        exact for the integer-valued keys)."""
+        if fp8:
+            return to_e4m3_codes(self.index_pool(device, pt, pages_per_chunk, upto))
         if pt is None:
             pt = self.page_table()
         own_s, own_p = self._page_owner(pt)

@@ -63,6 +63,14 @@ group g's selection is made exactly as the shared one, from group g's query,
 and heads 16g .. 16g+15 attend over group g's selected blocks and the current
 block.
 
+One-byte block keys (the StepFun blog, section "What sparse attention does and
+doesn't save", sizes the indexer read for keys of one or two bytes per value
+without naming the one-byte format): reading taken here, the 8-bit float
+E4M3 of the OCP 8-bit floating point specification (1 sign bit, 4 exponent
+bits with bias 7, 3 mantissa bits, subnormals, no infinities, S.1111.111 is
+NaN); a key byte stands for its exact E4M3 value and scores are then formed
+as for two-byte keys.
+
 Parity status: the cache append is pinned by rebuilding the seeded pools of
 a whole batch from the pools of its cached prefix;
 block selection is pinned by brute force, tie cases and the
@@ -345,3 +353,23 @@ def append_to_paged_cache(k_pool, v_pool, key_pool, page_table, ctx, nq, k_new, 
                 raise ValueError(f"row {r}: page {p} not in the key pool")
             key_out[p, slot // BLOCK, :] = key_new[r]
     return k_out, v_out, key_out
+
+
+# ----------------------------------------------------------------------------
+# one-byte block keys: the E4M3 value of each byte   [SAV]
+# ----------------------------------------------------------------------------
+
+def decode_e4m3(b) -> np.ndarray:
+    """Exact float64 value of each E4M3 byte (uint8 array of any shape).
+
+    bits: s eeee mmm.  e = 0: (-1)^s * 2^-6 * m/8 (subnormal, zero when m = 0);
+    e = 1..15: (-1)^s * 2^(e-7) * (1 + m/8), except e = 15, m = 7: NaN.
+    Largest finite magnitude 448 (e = 15, m = 6)."""
+    b = np.asarray(b, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 0x7).astype(np.float64)
+    normal = np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64))
+    sub = np.ldexp(m / 8.0, -6)
+    v = sign * np.where(e == 0, sub, normal)
+    return np.where((e == 15) & (b & 0x7 == 7), np.nan, v)

@@ -538,3 +538,27 @@ def test_grouped_attention_with_equal_selections_is_the_shared_layer():
     o1, l1 = O.sparse_attention_query(q, sel, t, k_seq, v_seq)
     o4, l4 = O.sparse_attention_query_grouped(q, [sel] * 4, t, k_seq, v_seq)
     assert np.array_equal(o1, o4) and np.array_equal(l1, l4)
+
+
+# ---------------------------------------------------------------- one-byte (E4M3) block keys
+
+def test_e4m3_values_the_format_fixes():
+    d = lambda x: float(O.decode_e4m3(np.array([x], dtype=np.uint8))[0])
+    assert d(0x38) == 1.0 and d(0x40) == 2.0 and d(0xB8) == -1.0
+    assert d(0x7E) == 448.0                  # largest finite: e = 15, m = 6
+    assert d(0x08) == 2.0 ** -6              # smallest normal
+    assert d(0x01) == 2.0 ** -9 and d(0x07) == 7 * 2.0 ** -9   # subnormals
+    assert d(0x00) == 0.0 and d(0x80) == 0.0 and math.copysign(1, d(0x80)) == -1
+    assert math.isnan(d(0x7F)) and math.isnan(d(0xFF))
+    assert d(0x77) == 240.0                  # e = 14, m = 7: 2^7 * 1.875
+    # positive codes increase strictly up to the largest finite value
+    v = O.decode_e4m3(np.arange(0x7F, dtype=np.uint8))
+    assert np.all(np.diff(v) > 0)
+
+
+def test_e4m3_matches_the_library_type_on_every_byte():
+    b = np.arange(256, dtype=np.uint8)
+    ours = O.decode_e4m3(b)
+    lib = torch.from_numpy(b).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(lib))
+    assert np.array_equal(ours[~np.isnan(ours)], lib[~np.isnan(lib)])

@@ -129,3 +129,15 @@ def test_grouped_indexer_queries():
     # a shard draws the same values for its rows
     sh = S.shard(w, 1, 2)
     assert torch.equal(sh.qx_group_rows(torch.arange(sh.total_q)), qg[3:])
+
+
+def test_one_byte_keys_hold_the_same_integer_values():
+    from oracle import s5_oracle as O
+    w = S.Workload(ctx=[3000, 700], nq=[1, 2], seed=6)
+    pt = w.page_table()
+    codes = w.index_pool("cpu", pt, fp8=True)
+    vals = w.index_pool("cpu", pt)
+    assert codes.dtype == torch.uint8 and codes.shape == vals.shape
+    assert (O.decode_e4m3(codes.numpy()) == vals.double().numpy()).all()
+    blk = torch.arange(100)
+    assert torch.equal(w.kx_blocks(1, blk, fp8=True), S.to_e4m3_codes(w.kx_blocks(1, blk)))
