@@ -417,7 +417,7 @@ def run_config(args) -> None:
         q, qx = w.queries(dev)
         out = torch.empty((w.total_q, 64, 192), dtype=torch.bfloat16, device=dev)
         lse = torch.empty((w.total_q, 64), dtype=torch.float32, device=dev)
-        key_pool = None if swa else w.index_pool(dev, pt)
+        key_pool = None if swa else w.index_pool(dev, pt, fp8=args.fp8_keys)
         if args.append:
             # the step starts by storing its new tokens (and completed block
             # keys); the pools already hold these values, so every replay
@@ -453,13 +453,16 @@ def run_config(args) -> None:
         else:
             sel = torch.empty((w.total_q, S.TOPK), dtype=torch.int32, device=dev)
             cnt = torch.empty((w.total_q,), dtype=torch.int32, device=dev)
-            calls.append(lambda kp=key_pool, b=batch, qx=qx, sel=sel, cnt=cnt, ws=ws:
-                         s5.s5_index_score_topk(kp, b, qx, S.TOPK, sel, cnt, ws))
-            kinds.append("index")
+            index_fn = s5.s5_index_score_topk_fp8 if args.fp8_keys else s5.s5_index_score_topk
+            calls.append(lambda kp=key_pool, b=batch, qx=qx, sel=sel, cnt=cnt, ws=ws, f=index_fn:
+                         f(kp, b, qx, S.TOPK, sel, cnt, ws))
+            kinds.append("index_fp8keys" if args.fp8_keys else "index")
             calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, sel=sel, cnt=cnt, o=out, l=lse, ws=ws:
                          s5.s5_sparse_gqa_attn(k, v, b, q, sel, cnt, S.TOPK, scale, o, l, ws))
             kinds.append("sparse")
-            bytes_total += R.sparse_decode_bytes(w.ctx, w.nq)["total"]
+            sp = R.sparse_decode_bytes(w.ctx, w.nq)
+            # one-byte keys: the indexer reads half the key bytes
+            bytes_total += sp["total"] - (sp["keys"] // 2 if args.fp8_keys else 0)
             flops_total += R.sparse_flops(w.ctx, w.nq)["total"]
     for _ in range(args.warmup):
         for c in calls:
@@ -496,7 +499,7 @@ def run_config(args) -> None:
             "algorithmic_bytes": bytes_total, "useful_flops": flops_total,
             "gbs": bytes_total / (ms * 1e-3) / 1e9, "pct_hbm_peak": 100 * bytes_total / (ms * 1e-3) / 1e9 / peak,
             "useful_tflops": flops_total / (ms * 1e-3) / 1e12, "steps": args.steps, "warmup": args.warmup,
-            "append": bool(args.append), "grouped": bool(args.grouped)}
+            "append": bool(args.append), "grouped": bool(args.grouped), "fp8_keys": bool(args.fp8_keys)}
     print(json.dumps(line), flush=True)
 
 
@@ -515,9 +518,15 @@ def main():
                     help="with --config: each layer step first appends its new tokens to the cache")
     ap.add_argument("--grouped", action="store_true",
                     help="with --config: sparse layers select per KV group (4 indexer queries per token)")
+    ap.add_argument("--fp8-keys", action="store_true",
+                    help="with --config: block keys stored as one-byte E4M3 codes")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.grouped and args.fp8_keys:
+        ap.error("--grouped selection runs on bf16 block keys only")
+    if args.append and args.fp8_keys:
+        ap.error("the cache append writes bf16 block keys")
     if args.impl == "reference":
         args.steps = min(args.steps, 20)
         run_reference(args)

@@ -447,7 +447,7 @@ s5_status workspace_need(const s5_batch_desc *batch, int32_t window, int groups,
 // [total_q][groups][256], one selection per (token, group) row.
 s5_status index_common(const s5_index_desc *index, const s5_batch_desc *batch, const void *q_index, int32_t topk,
                        int32_t *sel, int32_t *sel_count, void *workspace, size_t workspace_bytes,
-                       s5_stream_t stream, int groups) {
+                       s5_stream_t stream, int groups, bool key_fp8 = false) {
   s5_status st = check_batch(batch);
   if (st != S5_OK) return st;
   if (index == nullptr || index->key_pool == nullptr || index->num_pages < 1) return S5_ERR_INVALID_ARG;
@@ -477,6 +477,7 @@ s5_status index_common(const s5_index_desc *index, const s5_batch_desc *batch, c
   ia.total_q = batch->total_q;
   ia.q_index = q_index;
   ia.q_groups = groups;
+  ia.key_fp8 = key_fp8 ? 1 : 0;
   ia.scores = reinterpret_cast<float *>(wsb + w.scores);
   ia.score_stride = w.stride;
   ia.pages_per_cta = kScorePagesPerCta;
@@ -493,6 +494,7 @@ s5_status index_common(const s5_index_desc *index, const s5_batch_desc *batch, c
     ga.max_pages = batch->max_pages;
     ga.kxs = wsb + w.kxs;
     ga.max_blocks = w.stride;
+    ga.key_fp8 = key_fp8 ? 1 : 0;
     if (launch_gather_keys(ga, batch->batch, cs) != cudaSuccess) return S5_ERR_CUDA;
     CUtensorMap tq, tk;
     if (!make_k256_map(&tq, q_index, rows) || !make_k256_map(&tk, ga.kxs, (long long)batch->batch * w.stride))
@@ -552,6 +554,12 @@ s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *b
                               int32_t topk, int32_t *sel, int32_t *sel_count, void *workspace,
                               size_t workspace_bytes, s5_stream_t stream) {
   return index_common(index, batch, q_index, topk, sel, sel_count, workspace, workspace_bytes, stream, 1);
+}
+
+s5_status s5_index_score_topk_fp8(const s5_index_desc *index, const s5_batch_desc *batch, const void *q_index,
+                                  int32_t topk, int32_t *sel, int32_t *sel_count, void *workspace,
+                                  size_t workspace_bytes, s5_stream_t stream) {
+  return index_common(index, batch, q_index, topk, sel, sel_count, workspace, workspace_bytes, stream, 1, true);
 }
 
 s5_status s5_index_score_topk_grouped(const s5_index_desc *index, const s5_batch_desc *batch, const void *q_index,

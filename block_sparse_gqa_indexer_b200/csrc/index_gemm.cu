@@ -52,11 +52,26 @@ __global__ void __launch_bounds__(256) gather_keys_kernel(GatherArgs a) {
     for (int i = lane; i < nb * (kDx / 8); i += 32) dst[i] = make_uint4(0, 0, 0, 0);
     return;
   }
-  const uint4 *src = reinterpret_cast<const uint4 *>(a.key_pool) + (size_t)ph * kBpp * (kDx / 8);
   uint4 v[8];
+  if (a.key_fp8) {
+    // one-byte E4M3 keys: 8 bytes (8 dims) per 16-byte bf16 chunk, widened exactly
+    const uint2 *src8 = reinterpret_cast<const uint2 *>(a.key_pool) + (size_t)ph * kBpp * (kDx / 8);
 #pragma unroll
-  for (int u = 0; u < 8; ++u)
-    if (lane + 32 * u < nb * (kDx / 8)) v[u] = ld_cg(src + lane + 32 * u);
+    for (int u = 0; u < 8; ++u) {
+      if (lane + 32 * u < nb * (kDx / 8)) {
+        const uint2 c = src8[lane + 32 * u];
+        float f[8];
+        e4m3x4_to_float(c.x, f[0], f[1], f[2], f[3]);
+        e4m3x4_to_float(c.y, f[4], f[5], f[6], f[7]);
+        v[u] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
+      }
+    }
+  } else {
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.key_pool) + (size_t)ph * kBpp * (kDx / 8);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (lane + 32 * u < nb * (kDx / 8)) v[u] = ld_cg(src + lane + 32 * u);
+  }
 #pragma unroll
   for (int u = 0; u < 8; ++u)
     if (lane + 32 * u < nb * (kDx / 8)) dst[lane + 32 * u] = v[u];

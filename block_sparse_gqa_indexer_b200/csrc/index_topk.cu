@@ -44,8 +44,10 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&vals)[1 << LOGV], in
 }
 
 // GROUPED: a.q_groups indexer queries per token (one per KV group), rows
-// token-major; otherwise one query per token.
-template <int QT, int UNROLL, bool GROUPED>
+// token-major; otherwise one query per token.  KEY8: block keys are one-byte
+// E4M3 codes (a lane reads 8 bytes = 8 dims of a key), decoded exactly to
+// fp32 before the same FMA chain as the bf16 keys.
+template <int QT, int UNROLL, bool GROUPED, bool KEY8>
 __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
   constexpr int LOGV = (QT == 1) ? 3 : (QT == 2) ? 4 : 5;
   constexpr int V = 1 << LOGV;  // 8 blocks x QT queries
@@ -92,11 +94,13 @@ __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
   }
 
   const uint4 *keys = reinterpret_cast<const uint4 *>(a.key_pool);
+  const uint2 *keys8 = reinterpret_cast<const uint2 *>(a.key_pool);
   const int32_t *pt = a.page_table + (size_t)s * a.max_pages;
   const int nwarps = blockDim.x >> 5;
 
   for (int p = p_beg + warp * UNROLL; p < p_end; p += nwarps * UNROLL) {
     uint4 kv[UNROLL][kBpp];
+    uint2 kv8[UNROLL][kBpp];
     int phys[UNROLL];
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
@@ -112,12 +116,22 @@ __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
       }
 #pragma unroll
       for (int j = 0; j < kBpp; ++j) {
-        kv[u][j] = make_uint4(0, 0, 0, 0);
-        if (phys[u] >= 0 && (pp * kBpp + j) < c_hi) {
-          const uint4 *src = keys + ((size_t)phys[u] * kBpp + j) * (kDx / 8) + lane;
-          asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(kv[u][j].x), "=r"(kv[u][j].y), "=r"(kv[u][j].z), "=r"(kv[u][j].w)
-                       : "l"(src));
+        if constexpr (KEY8) {
+          kv8[u][j] = make_uint2(0, 0);
+          if (phys[u] >= 0 && (pp * kBpp + j) < c_hi) {
+            const uint2 *src = keys8 + ((size_t)phys[u] * kBpp + j) * (kDx / 8) + lane;
+            asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+                         : "=r"(kv8[u][j].x), "=r"(kv8[u][j].y)
+                         : "l"(src));
+          }
+        } else {
+          kv[u][j] = make_uint4(0, 0, 0, 0);
+          if (phys[u] >= 0 && (pp * kBpp + j) < c_hi) {
+            const uint4 *src = keys + ((size_t)phys[u] * kBpp + j) * (kDx / 8) + lane;
+            asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(kv[u][j].x), "=r"(kv[u][j].y), "=r"(kv[u][j].z), "=r"(kv[u][j].w)
+                         : "l"(src));
+          }
         }
       }
     }
@@ -129,12 +143,20 @@ __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
       for (int qi = 0; qi < QT; ++qi) {
 #pragma unroll
         for (int j = 0; j < kBpp; ++j) {
-          const uint32_t ww[4] = {kv[u][j].x, kv[u][j].y, kv[u][j].z, kv[u][j].w};
           float acc = 0.f;
+          if constexpr (KEY8) {
+            float f[8];
+            e4m3x4_to_float(kv8[u][j].x, f[0], f[1], f[2], f[3]);
+            e4m3x4_to_float(kv8[u][j].y, f[4], f[5], f[6], f[7]);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            acc = fmaf(qx[qi][2 * e], bf16lo(ww[e]), acc);
-            acc = fmaf(qx[qi][2 * e + 1], bf16hi(ww[e]), acc);
+            for (int e = 0; e < 8; ++e) acc = fmaf(qx[qi][e], f[e], acc);
+          } else {
+            const uint32_t ww[4] = {kv[u][j].x, kv[u][j].y, kv[u][j].z, kv[u][j].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              acc = fmaf(qx[qi][2 * e], bf16lo(ww[e]), acc);
+              acc = fmaf(qx[qi][2 * e + 1], bf16hi(ww[e]), acc);
+            }
           }
           vals[qi * kBpp + j] = acc;
         }
@@ -601,13 +623,19 @@ cudaError_t launch_index_score(const IndexScoreArgs &a, int max_q, int grid_page
   dim3 grid(grid_pages, n_seq, (max_q + qt - 1) / qt);
   if (a.q_groups > 1) {
     if (qt != 4) return cudaErrorInvalidValue;  // >= 4 rows per token
-    index_score_kernel<4, 1, true><<<grid, 256, 0, st>>>(a);
+    if (a.key_fp8) index_score_kernel<4, 2, true, true><<<grid, 256, 0, st>>>(a);
+    else index_score_kernel<4, 1, true, false><<<grid, 256, 0, st>>>(a);
+  } else if (a.key_fp8) {
+    // one-byte keys: half the bytes per page, so twice the pages in flight
+    if (qt == 1) index_score_kernel<1, 4, false, true><<<grid, 256, 0, st>>>(a);
+    else if (qt == 2) index_score_kernel<2, 4, false, true><<<grid, 256, 0, st>>>(a);
+    else index_score_kernel<4, 2, false, true><<<grid, 256, 0, st>>>(a);
   } else if (qt == 1) {
-    index_score_kernel<1, 2, false><<<grid, 256, 0, st>>>(a);
+    index_score_kernel<1, 2, false, false><<<grid, 256, 0, st>>>(a);
   } else if (qt == 2) {
-    index_score_kernel<2, 2, false><<<grid, 256, 0, st>>>(a);
+    index_score_kernel<2, 2, false, false><<<grid, 256, 0, st>>>(a);
   } else {
-    index_score_kernel<4, 1, false><<<grid, 256, 0, st>>>(a);
+    index_score_kernel<4, 1, false, false><<<grid, 256, 0, st>>>(a);
   }
   return cudaGetLastError();
 }

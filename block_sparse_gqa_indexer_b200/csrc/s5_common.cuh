@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -237,6 +239,19 @@ __device__ __forceinline__ uint32_t score_key(float s) {
   uint32_t u = __float_as_uint(s);
   if ((u & 0x7FFFFFFFu) == 0u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Four one-byte E4M3 codes (byte i of w is element i) to their exact values:
+// every E4M3 value is a half-precision value, and every half a float.
+__device__ __forceinline__ void e4m3x4_to_float(uint32_t w, float &f0, float &f1, float &f2, float &f3) {
+  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
+  const float2 a = __half22float2(__half2(lo));
+  const float2 b = __half22float2(__half2(hi));
+  f0 = a.x;
+  f1 = a.y;
+  f2 = b.x;
+  f3 = b.y;
 }
 
 // Hardware base-2 exponential / logarithm (PTX ex2.approx / lg2.approx).

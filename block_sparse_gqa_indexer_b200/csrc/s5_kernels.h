@@ -29,6 +29,7 @@ struct IndexScoreArgs {
   uint32_t *hist;  // [total_q * q_groups][4096] counts of score keys by their top 12 bits (zeroed before), or null
   int32_t *err;
   int q_groups;  // indexer queries per token (0 or 1: one shared query; 4: one per KV group)
+  int key_fp8;   // nonzero: key_pool holds one-byte E4M3 codes [num_pages][8][256]
 };
 
 constexpr int kHistBins = 4096;  // row histogram of the top 12 bits of the score keys
@@ -87,6 +88,7 @@ struct GatherArgs {
   int max_pages;
   void *kxs;       // bf16 [batch][max_blocks][256]
   int max_blocks;  // rows per sequence in kxs
+  int key_fp8;     // nonzero: key_pool holds one-byte E4M3 codes, widened to bf16 in kxs
 };
 
 struct GemmArgs {

@@ -30,6 +30,7 @@ S5_OK, S5_ERR_INVALID_ARG, S5_ERR_UNSUPPORTED, S5_ERR_CUDA, S5_ERR_DEVICE_BOUNDS
 
 # exported symbols (every declaration of include/s5attn.h)
 SYMBOLS = ("s5_workspace_size", "s5_index_score_topk", "s5_sparse_gqa_attn", "s5_swa_gqa_attn",
+           "s5_index_score_topk_fp8",
            "s5_workspace_size_grouped", "s5_index_score_topk_grouped", "s5_sparse_gqa_attn_grouped",
            "s5_index_score_topk_noalloc", "s5_append_kv", "s5_reset_device_error", "s5_get_device_error",
            "s5_status_string", "s5_abi_version")
@@ -59,6 +60,7 @@ _lib.s5_sparse_gqa_attn.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(Batch
                                     ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.s5_swa_gqa_attn.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(BatchDesc), _P, _I, ctypes.c_float, _P,
                                  _P, _P, ctypes.c_size_t, _P]
+_lib.s5_index_score_topk_fp8.argtypes = _lib.s5_index_score_topk.argtypes
 _lib.s5_workspace_size_grouped.argtypes = _lib.s5_workspace_size.argtypes
 _lib.s5_index_score_topk_grouped.argtypes = _lib.s5_index_score_topk.argtypes
 _lib.s5_sparse_gqa_attn_grouped.argtypes = _lib.s5_sparse_gqa_attn.argtypes
@@ -174,6 +176,20 @@ def s5_index_score_topk(key_pool: torch.Tensor, batch: Batch, q_index: torch.Ten
     _check(_lib.s5_index_score_topk(ctypes.byref(idx), ctypes.byref(batch.desc), _ptr(q_index), int(topk),
                                     _ptr(sel), _ptr(sel_count), _ptr(ws), ws.numel(), _stream(stream)),
            "s5_index_score_topk")
+
+
+def s5_index_score_topk_fp8(key_pool: torch.Tensor, batch: Batch, q_index: torch.Tensor, topk: int,
+                            sel: torch.Tensor, sel_count: torch.Tensor, ws: torch.Tensor, stream=None):
+    """s5_index_score_topk with one-byte E4M3 block keys (key_pool uint8 [num_pages][8][256])."""
+    _need(key_pool, torch.uint8, "key_pool")
+    _need(q_index, torch.bfloat16, "q_index", (batch.total_q, INDEX_DIM))
+    _need(sel, torch.int32, "sel", (batch.total_q, topk))
+    _need(sel_count, torch.int32, "sel_count", (batch.total_q,))
+    _need(ws, torch.uint8, "ws")
+    idx = IndexDesc(key_pool.data_ptr(), key_pool.shape[0], key_pool.shape[-1])
+    _check(_lib.s5_index_score_topk_fp8(ctypes.byref(idx), ctypes.byref(batch.desc), _ptr(q_index), int(topk),
+                                        _ptr(sel), _ptr(sel_count), _ptr(ws), ws.numel(), _stream(stream)),
+           "s5_index_score_topk_fp8")
 
 
 def s5_index_score_topk_grouped(key_pool: torch.Tensor, batch: Batch, q_index: torch.Tensor, topk: int,

@@ -166,6 +166,19 @@ s5_status s5_swa_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, cons
                           int32_t window, float sm_scale, void *out, float *lse,
                           void *workspace, size_t workspace_bytes, s5_stream_t stream);
 
+/* s5_index_score_topk with one-byte block keys (StepFun open-weights blog,
+ * "What sparse attention does and doesn't save": the indexer read at one or
+ * two bytes per key value).  index->key_pool holds E4M3 codes, uint8
+ * [num_pages][8][256] (the 8-bit float of the OCP FP8 specification: bias 7,
+ * 3 mantissa bits, no infinities), 16-byte aligned; each code stands for its
+ * exact value, and scores, selection and results are defined as for
+ * s5_index_score_topk on those values (the same for keys that are exactly
+ * representable in E4M3).  The indexer reads half the bytes.  The workspace
+ * of s5_workspace_size covers this call. */
+s5_status s5_index_score_topk_fp8(const s5_index_desc *index, const s5_batch_desc *batch, const void *q_index,
+                                  int32_t topk, int32_t *sel, int32_t *sel_count, void *workspace,
+                                  size_t workspace_bytes, s5_stream_t stream);
+
 /* Per-KV-group selection (StepFun open-weights blog, "What sparse attention
  * does and doesn't save": each KV group picks its own blocks).  The block
  * keys stay shared (the configuration gives one 256-wide key per block); the
@@ -232,8 +245,8 @@ s5_status s5_index_score_topk_noalloc(const s5_index_desc *index, const s5_batch
  * its last token; key_new rows of other tokens are not read.
  *   kv       the pools to WRITE (the descriptor's const applies to the
  *            attention calls, which only read them)
- *   index    the block-key pool to write, or NULL for a cache without block
- *            keys (a sliding-window layer); key_new is then ignored
+ *   index    the bf16 block-key pool to write, or NULL for a cache without
+ *            block keys (a sliding-window layer); key_new is then ignored
  *   k_new, v_new  device bf16 [total_q][4][192], 16-byte aligned
  *   key_new  device bf16 [total_q][256], 16-byte aligned (when index != NULL)
  *   workspace  at least S5_WS_FIXED_BYTES; only its error record is used

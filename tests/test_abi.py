@@ -174,3 +174,13 @@ def test_grouped_workspace_and_limits(s5):
                                               fake, None, fake, 1 << 30, None) == s5.S5_ERR_INVALID_ARG
     assert s5._lib.s5_index_score_topk_grouped(ctypes.byref(ix), ctypes.byref(_batch()), fake, 512, fake, fake,
                                                None, 1 << 30, None) == s5.S5_ERR_WORKSPACE
+
+
+def test_fp8_key_entry_checks(s5):
+    fake = ctypes.c_void_p(0x1000)
+    ix = s5.IndexDesc(0x1000, 8, 128)
+    assert s5._lib.s5_index_score_topk_fp8(ctypes.byref(ix), ctypes.byref(_batch()), fake, 512, fake, fake, fake,
+                                           1 << 30, None) == s5.S5_ERR_UNSUPPORTED
+    ix = s5.IndexDesc(0x1008, 8, 256)  # not 16-byte aligned
+    assert s5._lib.s5_index_score_topk_fp8(ctypes.byref(ix), ctypes.byref(_batch()), fake, 512, fake, fake, fake,
+                                           1 << 30, None) == s5.S5_ERR_INVALID_ARG
