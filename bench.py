@@ -81,9 +81,13 @@ CLOCK_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,
 
 
 class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons during the timed
+    loop, written to S5_CLOCKS_DIR (default: _clocks/ in the repository)."""
+
     def __init__(self, gpu_index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        out_dir = os.environ.get("S5_CLOCKS_DIR") or os.path.join(ROOT, "_clocks")
+        self.path = os.path.join(out_dir, f"clocks_rank{gpu_index}.csv")
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
