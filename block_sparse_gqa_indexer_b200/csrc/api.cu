@@ -16,7 +16,7 @@ using namespace s5;
 
 namespace {
 
-constexpr int kAbiVersion = 100;
+constexpr int kAbiVersion = S5_ABI_VERSION;
 constexpr int kSelCap = 16384;      // rows up to this many blocks: one CTA selects the whole row
 constexpr int kSegShort = 4096;     // longer rows: top-k per segment of this many blocks, then a merge
 constexpr int kSeg = 8192;          // ... segments of rows longer than 16,384 blocks

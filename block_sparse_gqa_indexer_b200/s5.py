@@ -21,6 +21,7 @@ if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m block_sparse_gqa_indexer_b200.build`")
 _lib = ctypes.CDLL(LIB_PATH)
 
+ABI_VERSION = 101  # S5_ABI_VERSION of the header this binding follows
 N_HEADS, N_KV, HEAD_DIM, PAGE, BLOCK, INDEX_DIM, MAX_TOPK = 64, 4, 192, 64, 8, 256, 512
 MAX_LEN = 1 << 21
 DEFAULT_SM_SCALE = 1.0 / math.sqrt(HEAD_DIM)
@@ -76,6 +77,8 @@ _lib.s5_abi_version.restype = ctypes.c_int32
 for _name in SYMBOLS:
     if _name not in ("s5_status_string", "s5_abi_version"):
         getattr(_lib, _name).restype = ctypes.c_int
+if _lib.s5_abi_version() != ABI_VERSION:
+    raise ImportError(f"{LIB_PATH} implements ABI {_lib.s5_abi_version()}, this binding {ABI_VERSION}: rebuild it")
 
 
 class S5Error(RuntimeError):

@@ -86,6 +86,10 @@ typedef enum {
 #define S5_MAX_TOPK 512
 #define S5_MAX_LEN (1 << 21) /* longest sequence (cached + new tokens) */
 
+/* ABI version (major * 100 + minor): 1.01 added the cache append, the
+ * per-KV-group entry points and the one-byte-key indexer. */
+#define S5_ABI_VERSION 101
+
 /* One attention layer's paged KV cache. */
 typedef struct {
   const void *k_pool;  /* device bf16 [num_pages][4][64][192], 16-byte aligned */
@@ -270,7 +274,7 @@ s5_status s5_get_device_error(void *workspace, s5_stream_t stream, int32_t *code
 /* Static English name of a status code. */
 const char *s5_status_string(s5_status status);
 
-/* ABI version of this header (major * 100 + minor). */
+/* S5_ABI_VERSION of the header the library was built with. */
 int32_t s5_abi_version(void);
 
 #ifdef __cplusplus

@@ -34,7 +34,9 @@ def test_every_declared_symbol_is_exported(s5):
 
 
 def test_status_strings_and_version(s5):
-    assert s5.s5_abi_version() == 100
+    assert s5.s5_abi_version() == s5.ABI_VERSION
+    m = re.search(r"#define S5_ABI_VERSION (\d+)", open(HEADER).read())
+    assert m and int(m.group(1)) == s5.ABI_VERSION
     for code in range(7):
         assert s5.s5_status_string(code).startswith("S5_")
     assert s5.s5_status_string(99) == "S5_ERR_UNKNOWN"
