@@ -2,9 +2,9 @@
 // 5th-generation tensor cores, over the shared set of selected blocks.
 //
 // SGLang day-0 blog ("Step 5 Preview: Day-0 Inference and RL Support with
-// SGLang and Miles"), "Kernels from StepFun": sparse prefill gathers the blocks
-// selected for a batch of queries into one shared set and runs attention over
-// that set with per-query masks.  Here the batch is a tile of up to 8
+// SGLang and Miles"), "Kernels from StepFun": for prefill, the union of the
+// blocks chosen by every query of a batch is attended once, with a mask that
+// keeps each query to its own blocks.  Here the batch is a tile of up to 8
 // consecutive query rows of one sequence:
 //
 //   tile_union_kernel   builds, per tile, the ascending list of distinct blocks

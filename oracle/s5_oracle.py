@@ -21,9 +21,9 @@ Sources (the pages give prose and a configuration table, no formulas or code):
       SGLang and Miles", section "Hybrid Attention": a sliding-window layer
       attends to a 512-token window and is followed (after two more such
       layers) by a sparse layer; the sparse layer rates each 8-token block of
-      history through a per-block summary, keeps at most 512 of them, and
-      attends to their tokens together with the tokens of the block the query
-      itself sits in.
+      history through a per-block summary, keeps no more than 512 blocks,
+      and reads the tokens of those blocks as well as the tokens of the block
+      that holds the query.
 [KS]  same page, section "Kernels from StepFun": the indexer rates each query
       against the compressed (per-block) history held in the paged cache;
       decode cuts a long selection into partitions and combines their partial
