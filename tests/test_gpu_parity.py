@@ -429,3 +429,22 @@ def test_cuda_graph_replay_matches_eager(lib):
     for a, b in zip(eager, results):
         assert torch.equal(a, b)
     _check_no_device_error(lib, d)
+
+
+@pytest.mark.parametrize("topk", [1, 64, 300])
+def test_smaller_topk_both_paths(lib, topk):
+    # k below 512: decode rows, a verify group and an 8-token chunk (tile
+    # path candidates), histories below and above k blocks
+    w = S.Workload(ctx=[5, 700, 3000, 9000, 12000], nq=[1, 1, 4, 1, 8], seed=47)
+    d = DeviceInputs(w, lib)
+    sel = torch.full((w.total_q, topk), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((w.total_q,), -7, dtype=torch.int32, device="cuda")
+    lib.s5_index_score_topk(d.key_pool, d.batch, d.qx, topk, sel, cnt, d.ws)
+    lib.s5_sparse_gqa_attn(d.k_pool, d.v_pool, d.batch, d.q, sel, cnt, topk, O.DEFAULT_SM_SCALE, d.out, d.lse, d.ws)
+    torch.cuda.synchronize()
+    _check_no_device_error(lib, d)
+    rows = list(range(w.total_q))
+    want = oracle_selection(w, rows, topk)
+    assert np.array_equal(sel.cpu().numpy(), want)
+    assert np.array_equal(cnt.cpu().numpy(), [O.selection_count(x) for x in want])
+    _check_sparse_out(d, rows, want, f"topk {topk}")
