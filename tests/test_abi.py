@@ -186,3 +186,26 @@ def test_fp8_key_entry_checks(s5):
     ix = s5.IndexDesc(0x1008, 8, 256)  # not 16-byte aligned
     assert s5._lib.s5_index_score_topk_fp8(ctypes.byref(ix), ctypes.byref(_batch()), fake, 512, fake, fake, fake,
                                            1 << 30, None) == s5.S5_ERR_INVALID_ARG
+
+
+def test_grouped_and_fp8_entries_validate_like_the_shared_ones(s5):
+    fake = ctypes.c_void_p(0x1000)
+    b = _batch()
+    kv = s5.KvDesc(0x1000, 0x1000, 8, 64, 4, 192)
+    # non-finite softmax scale, top-k out of range, short workspace
+    assert s5._lib.s5_sparse_gqa_attn_grouped(ctypes.byref(kv), ctypes.byref(b), fake, fake, fake, 512,
+                                              float("nan"), fake, None, fake, 1 << 30, None) == s5.S5_ERR_INVALID_ARG
+    assert s5._lib.s5_sparse_gqa_attn_grouped(ctypes.byref(kv), ctypes.byref(b), fake, fake, fake, 0, 0.1, fake,
+                                              None, fake, 1 << 30, None) == s5.S5_ERR_INVALID_ARG
+    assert s5._lib.s5_sparse_gqa_attn_grouped(ctypes.byref(kv), ctypes.byref(b), fake, fake, fake, 512, 0.1, fake,
+                                              None, fake, 16, None) == s5.S5_ERR_WORKSPACE
+    ix = s5.IndexDesc(0x1000, 8, 256)
+    for f in (s5._lib.s5_index_score_topk_grouped, s5._lib.s5_index_score_topk_fp8):
+        assert f(ctypes.byref(ix), ctypes.byref(b), fake, 513, fake, fake, fake, 1 << 30, None) == s5.S5_ERR_INVALID_ARG
+        assert f(ctypes.byref(ix), ctypes.byref(b), None, 512, fake, fake, fake, 1 << 30, None) == s5.S5_ERR_INVALID_ARG
+        assert f(ctypes.byref(ix), ctypes.byref(b), fake, 512, fake, fake, fake, 16, None) == s5.S5_ERR_WORKSPACE
+        # an empty batch enqueues nothing
+        assert f(ctypes.byref(ix), ctypes.byref(_batch(total_q=0)), None, 512, None, None, fake, 16,
+                 None) == s5.S5_OK
+    n = ctypes.c_size_t(0)
+    assert s5._lib.s5_workspace_size_grouped(ctypes.byref(b), -1, ctypes.byref(n)) == s5.S5_ERR_INVALID_ARG

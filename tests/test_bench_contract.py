@@ -6,6 +6,8 @@ import os
 import subprocess
 import sys
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -50,3 +52,10 @@ def test_reference_arm_under_torchrun_prints_one_line():
     sys.path.insert(0, ROOT)
     import bench
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["config"] == bench.bench_config(64, 2)
+
+
+@pytest.mark.parametrize("flags", [["--grouped", "--fp8-keys"], ["--append", "--fp8-keys"]])
+def test_unsupported_variant_combinations_are_refused(flags):
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--config", "0", *flags], cwd=ROOT,
+                         capture_output=True, text=True, timeout=120)
+    assert out.returncode != 0 and "error" in out.stderr
