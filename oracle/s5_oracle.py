@@ -74,7 +74,8 @@ as for two-byte keys.
 Parity status: the cache append is pinned by rebuilding the seeded pools of
 a whole batch from the pools of its cached prefix;
 block selection is pinned by brute force, tie cases and the
-subset characterisation of top-k; the attention functions are pinned by closed
+subset characterisation of top-k (the multi-row form also by brute force on
+tiny inputs, by history masking and by agreement with the one-row form); the attention functions are pinned by closed
 forms (one token, identical keys, two tokens), the reduction of sparse and
 sliding-window attention to full causal attention, weight normalisation and
 invariance to the order of the selected blocks.  The pages print no worked
@@ -161,6 +162,41 @@ def index_topk_query(qx, kx_seq, t: int, topk: int = TOPK) -> np.ndarray:
     return select_topk(block_scores(qx, kx_seq[np.arange(c)]), topk)
 
 
+def index_topk_rows(qx_rows, kx_seq, positions, topk: int = TOPK) -> np.ndarray:
+    """Selections [len(positions)][topk] of several query rows of ONE sequence.
+
+    Row i has indexer query ``qx_rows[i]`` and absolute position
+    ``positions[i]``; ``kx_seq`` is an array [>= c_max][256] of the sequence's
+    block keys.  Each row's result is exactly ``index_topk_query`` of that row:
+    the scores of the row's history blocks 0 .. c_i - 1 (c_i = t_i // 8), the
+    stable sort on descending score (which keeps equal scores in ascending
+    block order, i.e. the lower block wins a tie), the first ``topk``, reported
+    ascending and -1 padded.  The scores of all rows come from one product of
+    the stacked queries with the keys; blocks at or past a row's current block
+    are set to -inf for that row, so they sort after every history block and a
+    row with more than ``topk`` history blocks never selects one."""
+    qx_rows = np.asarray(qx_rows, dtype=np.float64).reshape(-1, INDEX_DIM)
+    positions = np.asarray(positions, dtype=np.int64).reshape(-1)
+    n = positions.shape[0]
+    out = np.full((n, topk), -1, dtype=np.int64)
+    if n == 0:
+        return out
+    c = positions // BLOCK
+    short = c <= topk
+    for i in np.nonzero(short)[0]:
+        out[i, :c[i]] = np.arange(c[i])
+    long_rows = np.nonzero(~short)[0]
+    if long_rows.size == 0:
+        return out
+    c_max = int(c[long_rows].max())
+    kx = np.asarray(kx_seq[np.arange(c_max)], dtype=np.float64)
+    scores = qx_rows[long_rows] @ kx.T                     # [rows][c_max]
+    scores[np.arange(c_max)[None, :] >= c[long_rows][:, None]] = -np.inf
+    order = np.argsort(-scores, axis=1, kind="stable")     # ties keep ascending block order
+    out[long_rows] = np.sort(order[:, :topk], axis=1)
+    return out
+
+
 def selection_count(sel) -> int:
     sel = np.asarray(sel)
     return int((sel >= 0).sum())
@@ -237,7 +273,7 @@ def swa_attention_query(q, t: int, k_seq, v_seq, window: int = WINDOW, sm_scale:
 
 
 # ----------------------------------------------------------------------------
-# batched drivers (varlen batches: per sequence, ctx cached tokens, then nq queries)
+# per-KV-group selection and attention; row positions of a varlen batch
 # ----------------------------------------------------------------------------
 
 def index_topk_query_grouped(qx_groups, kx_seq, t: int, topk: int = TOPK) -> np.ndarray:
@@ -269,49 +305,6 @@ def query_positions(ctx, nq):
         for j in range(n):
             rows.append((s, c + j))
     return rows
-
-
-def index_topk_batch(qx, kx_of_seq, ctx, nq, topk: int = TOPK, rows=None):
-    """Selections [n_rows][topk] (-1 padded) and counts for the given rows.
-
-    ``kx_of_seq(s)`` returns an array indexable by block ids of sequence s."""
-    pos = query_positions(ctx, nq)
-    rows = range(len(pos)) if rows is None else rows
-    sel, cnt = [], []
-    for r in rows:
-        s, t = pos[r]
-        x = index_topk_query(qx[r], kx_of_seq(s), t, topk)
-        sel.append(x)
-        cnt.append(selection_count(x))
-    return np.array(sel, dtype=np.int64).reshape(-1, topk), np.array(cnt, dtype=np.int64)
-
-
-def sparse_attention_batch(q, sel, ctx, nq, kv_of_seq, sm_scale: float = DEFAULT_SM_SCALE, rows=None):
-    """Sparse attention for the given rows: (out [n][64][192], lse [n][64])."""
-    pos = query_positions(ctx, nq)
-    rows = list(range(len(pos))) if rows is None else list(rows)
-    outs, lses = [], []
-    for i, r in enumerate(rows):
-        s, t = pos[r]
-        k_seq, v_seq = kv_of_seq(s)
-        o, l = sparse_attention_query(q[i], sel[i], t, k_seq, v_seq, sm_scale)
-        outs.append(o)
-        lses.append(l)
-    return np.array(outs), np.array(lses)
-
-
-def swa_attention_batch(q, ctx, nq, kv_of_seq, window: int = WINDOW, sm_scale: float = DEFAULT_SM_SCALE, rows=None):
-    """Sliding-window attention for the given rows: (out [n][64][192], lse [n][64])."""
-    pos = query_positions(ctx, nq)
-    rows = list(range(len(pos))) if rows is None else list(rows)
-    outs, lses = [], []
-    for i, r in enumerate(rows):
-        s, t = pos[r]
-        k_seq, v_seq = kv_of_seq(s)
-        o, l = swa_attention_query(q[i], t, k_seq, v_seq, window, sm_scale)
-        outs.append(o)
-        lses.append(l)
-    return np.array(outs), np.array(lses)
 
 
 # ----------------------------------------------------------------------------

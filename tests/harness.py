@@ -28,15 +28,6 @@ class LazyRows:
         return f(self.s, pos).double().numpy()
 
 
-class LazyKeys:
-    def __init__(self, w: S.Workload, s: int):
-        self.w, self.s = w, s
-
-    def __getitem__(self, blocks):
-        b = torch.as_tensor(np.asarray(blocks, dtype=np.int64))
-        return self.w.kx_blocks(self.s, b).double().numpy()
-
-
 class DeviceInputs:
     """Everything the CUDA path needs for one layer, resident on the device."""
 
@@ -55,13 +46,64 @@ class DeviceInputs:
         self.lse = torch.full((tq, 64), float("nan"), dtype=torch.float32, device=device)
 
 
-def oracle_selection(w: S.Workload, rows, topk=S.TOPK):
+def seq_keys(w: S.Workload, s: int, n_blocks: int, fp8: bool = False, chunk: int = 16384) -> np.ndarray:
+    """Block keys 0 .. n_blocks-1 of sequence s as float64 [n_blocks][256], drawn
+    once on the CPU (with ``fp8``: the exact E4M3 value of each stored byte)."""
+    out = np.empty((n_blocks, S.INDEX_DIM), dtype=np.float64)
+    for b0 in range(0, n_blocks, chunk):
+        b = torch.arange(b0, min(n_blocks, b0 + chunk), dtype=torch.int64)
+        if fp8:
+            out[b0:b0 + len(b)] = O.decode_e4m3(w.kx_blocks(s, b, fp8=True).numpy())
+        else:
+            out[b0:b0 + len(b)] = w.kx_blocks(s, b).double().numpy()
+    return out
+
+
+def oracle_selection(w: S.Workload, rows, topk=S.TOPK, qx=None, fp8=False, chunk=1024):
+    """Oracle selections [len(rows)][topk] of the given query rows.
+
+    ``qx`` [len(rows)][256] overrides the workload's indexer queries (one
+    per row).  Each sequence's keys are drawn once and all of its rows are
+    selected against them."""
+    rows = list(rows)
     seqs, pos = w.query_seq_pos()
-    qx = w.qx_rows(torch.as_tensor(list(rows), dtype=torch.int64)).double().numpy()
-    out = []
+    if qx is None:
+        qx = w.qx_rows(torch.as_tensor(rows, dtype=torch.int64)).double().numpy()
+    qx = np.asarray(qx, dtype=np.float64)
+    out = np.full((len(rows), topk), -1, dtype=np.int64)
+    by_seq = {}
     for i, r in enumerate(rows):
-        out.append(O.index_topk_query(qx[i], LazyKeys(w, seqs[r]), pos[r], topk))
-    return np.array(out)
+        by_seq.setdefault(seqs[r], []).append(i)
+    for s, idx in by_seq.items():
+        idx = np.array(idx)
+        p = np.array([pos[rows[i]] for i in idx], dtype=np.int64)
+        c_max = int((p // S.BLOCK).max())
+        keys = seq_keys(w, s, c_max, fp8) if c_max > topk else np.zeros((0, S.INDEX_DIM))
+        for k in range(0, len(idx), chunk):
+            part = idx[k:k + chunk]
+            out[part] = O.index_topk_rows(qx[part], keys, p[k:k + chunk], topk)
+    return out
+
+
+def oracle_selection_grouped(w: S.Workload, rows, topk=S.TOPK):
+    """Per-KV-group oracle selections [len(rows)][4][topk]: each (row, group)
+    pair is selected from that group's indexer query."""
+    rows = list(rows)
+    qx = w.qx_group_rows(torch.as_tensor(rows, dtype=torch.int64)).double().numpy()
+    flat = [r for r in rows for _ in range(S.N_KV)]  # row-major, group-minor, as qx
+    return oracle_selection(w, flat, topk, qx=qx.reshape(-1, S.INDEX_DIM)).reshape(len(rows), S.N_KV, topk)
+
+
+def check_all_selections(w: S.Workload, sel_dev, cnt_dev, topk=S.TOPK, fp8=False):
+    """Every row's selection and count against the oracle, bit for bit."""
+    rows = list(range(w.total_q))
+    want = oracle_selection(w, rows, topk, fp8=fp8)
+    got = sel_dev.cpu().numpy()
+    cnt = cnt_dev.cpu().numpy()
+    bad = np.nonzero(~np.all(got == want, axis=1))[0]
+    assert bad.size == 0, f"{bad.size} of {len(rows)} rows differ, first {bad[:8].tolist()}"
+    assert np.array_equal(cnt, (want >= 0).sum(axis=1)), "selection counts differ"
+    return want
 
 
 def oracle_sparse(w: S.Workload, rows, sel_rows, sm_scale=O.DEFAULT_SM_SCALE):

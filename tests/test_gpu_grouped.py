@@ -10,7 +10,7 @@ import torch
 
 from block_sparse_gqa_indexer_b200 import synth as S
 from oracle import s5_oracle as O
-from tests.harness import LSE_ABS, LazyKeys, LazyRows, assert_attn_close, sample_rows
+from tests.harness import LSE_ABS, LazyRows, assert_attn_close, oracle_selection_grouped, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -43,23 +43,33 @@ def _no_error(lib, ws):
     assert code == 0, (lib.s5_status_string(code), info)
 
 
-def _check(lib, g: GroupedInputs, rows):
+def _check_selections(g: GroupedInputs, rows=None):
+    """Every listed row's four selections and counts, bit for bit (default: all rows)."""
+    rows = list(range(g.w.total_q)) if rows is None else list(rows)
+    want = oracle_selection_grouped(g.w, rows)
+    sel = g.sel.cpu().numpy()[rows]
+    cnt = g.cnt.cpu().numpy()[rows]
+    bad = np.nonzero(~np.all(sel == want, axis=(1, 2)))[0]
+    assert bad.size == 0, f"{bad.size} rows with a differing group selection, first {[rows[i] for i in bad[:8]]}"
+    assert np.array_equal(cnt, (want >= 0).sum(axis=2)), "selection counts differ"
+    return want
+
+
+def _check(lib, g: GroupedInputs, rows, all_selections=False):
     torch.cuda.synchronize()
     _no_error(lib, g.ws)
     w = g.w
     seqs, pos = w.query_seq_pos()
     rows = list(rows)
-    qx = w.qx_group_rows(torch.as_tensor(rows, dtype=torch.int64)).double().numpy()
     q = w.q_rows(torch.as_tensor(rows, dtype=torch.int64)).double().numpy()
-    sel = g.sel.cpu().numpy()
-    cnt = g.cnt.cpu().numpy()
-    outs, lses, want_o, want_l = [], [], [], []
+    if all_selections:
+        want_sel = _check_selections(g)[rows]
+    else:
+        want_sel = _check_selections(g, rows)
+    want_o, want_l = [], []
     for i, r in enumerate(rows):
         s, t = seqs[r], pos[r]
-        want = O.index_topk_query_grouped(qx[i], LazyKeys(w, s), t)
-        assert np.array_equal(sel[r], want), f"row {r}: a group's selection differs"
-        for grp in range(S.N_KV):
-            assert cnt[r, grp] == O.selection_count(want[grp])
+        want = want_sel[i]
         o, l = O.sparse_attention_query_grouped(q[i], want, t, LazyRows(w, s, "k"), LazyRows(w, s, "v"))
         want_o.append(O.round_bf16(o))
         want_l.append(l)
@@ -87,15 +97,8 @@ def test_grouped_prefill_sized_tensor_core_scores(lib):
     # tcgen05 GEMM, rows token-major and group-minor
     g = GroupedInputs(S.Workload(ctx=[9000, 6007], nq=[40, 33], seed=42), lib)
     g.run(lib)
-    _check(lib, g, sample_rows(g.w.total_q, 12, 1))
-    torch.cuda.synchronize()
-    # every row's selection, not only the sampled attention rows
-    w = g.w
-    seqs, pos = w.query_seq_pos()
-    qx = w.qx_group_rows(torch.arange(w.total_q)).double().numpy()
-    sel = g.sel.cpu().numpy()
-    for r in range(w.total_q):
-        assert np.array_equal(sel[r], O.index_topk_query_grouped(qx[r], LazyKeys(w, seqs[r]), pos[r])), r
+    # every row's selection, attention on sampled rows
+    _check(lib, g, sample_rows(g.w.total_q, 12, 1), all_selections=True)
 
 
 def test_grouped_more_than_1024_selection_rows(lib):
@@ -103,7 +106,7 @@ def test_grouped_more_than_1024_selection_rows(lib):
     # and builds each row's histogram in shared memory
     g = GroupedInputs(S.Workload(ctx=[7000 + 37 * i for i in range(20)], nq=[16] * 20, seed=43), lib)
     g.run(lib)
-    _check(lib, g, sample_rows(g.w.total_q, 10, 2))
+    _check(lib, g, sample_rows(g.w.total_q, 10, 2), all_selections=True)
 
 
 def test_grouped_history_beyond_16k_blocks(lib):
@@ -150,4 +153,5 @@ def test_grouped_decode_b64_128k(lib):
     (w0,) = S.config_workloads(0)
     g = GroupedInputs(w0, lib)
     g.run(lib)
-    _check(lib, g, sample_rows(w0.total_q, 3, 3))
+    # all 64 x 4 selections; attention on sampled rows
+    _check(lib, g, sample_rows(w0.total_q, 3, 3), all_selections=True)

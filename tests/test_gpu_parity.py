@@ -10,8 +10,8 @@ import torch
 
 from block_sparse_gqa_indexer_b200 import synth as S
 from oracle import s5_oracle as O
-from tests.harness import (DeviceInputs, LSE_ABS, assert_attn_close, oracle_selection, oracle_sparse,
-                           oracle_swa, sample_rows)
+from tests.harness import (DeviceInputs, LSE_ABS, assert_attn_close, check_all_selections, oracle_selection,
+                           oracle_sparse, oracle_swa, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -186,14 +186,16 @@ def test_host_validation(lib):
 # ------------------------------------------------------------------ the configurations (sampled rows)
 
 def _config_sparse(lib, which, n_rows, seed=0):
+    # every row's selection bit for bit; attention on sampled rows
     (w,) = S.config_workloads(which)
     d = DeviceInputs(w, lib)
     lib.s5_reset_device_error(d.ws)
     _run_index(lib, d)
     _run_sparse(lib, d)
+    torch.cuda.synchronize()
+    want_all = check_all_selections(w, d.sel, d.sel_count)
     rows = sample_rows(w.total_q, n_rows, seed)
-    want_sel = _check_selection(lib, d, rows)
-    _check_sparse_out(d, rows, want_sel, f"config {which}")
+    _check_sparse_out(d, rows, want_all[rows], f"config {which}")
     _check_no_device_error(lib, d)
     return d
 
@@ -245,9 +247,10 @@ def test_config5_hybrid_1m(lib):
             d = DeviceInputs(w, lib)
             _run_index(lib, d)
             _run_sparse(lib, d)
+            torch.cuda.synchronize()
+            want_sel = check_all_selections(w, d.sel, d.sel_count)  # all 4 rows
             rows = sample_rows(w.total_q, 2, li)
-            want_sel = _check_selection(lib, d, rows)
-            _check_sparse_out(d, rows, want_sel, "config 5 sparse layer")
+            _check_sparse_out(d, rows, want_sel[rows], "config 5 sparse layer")
             _check_no_device_error(lib, d)
         del d
         torch.cuda.empty_cache()

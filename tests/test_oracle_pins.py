@@ -562,3 +562,50 @@ def test_e4m3_matches_the_library_type_on_every_byte():
     lib = torch.from_numpy(b).view(torch.float8_e4m3fn).double().numpy()
     assert np.array_equal(np.isnan(ours), np.isnan(lib))
     assert np.array_equal(ours[~np.isnan(ours)], lib[~np.isnan(lib)])
+
+
+# ---------------------------------------------------------------- multi-row selection
+
+@pytest.mark.parametrize("trial", range(12))
+def test_index_topk_rows_brute_force_tiny(trial):
+    # tiny histories with heavy ties: every row against repeated max extraction
+    # over its own history only
+    c_max = int(RNG.integers(2, 40))
+    k = int(RNG.choice([1, 3, 8]))
+    kx = RNG.integers(-2, 3, (c_max + 3, 256)).astype(np.float64)
+    pos = RNG.integers(0, 8 * c_max + 8, 7)
+    qx = RNG.integers(-2, 3, (7, 256)).astype(np.float64)
+    got = O.index_topk_rows(qx, kx, pos, k)
+    for i, t in enumerate(pos.tolist()):
+        c = t // 8
+        if c <= k:
+            want = list(range(c))
+        else:
+            want = _naive_topk([float(kx[b] @ qx[i]) for b in range(c)], k)
+        assert list(got[i][:len(want)]) == want, (i, t)
+        assert np.all(got[i][len(want):] == -1)
+
+
+def test_index_topk_rows_masks_each_rows_future():
+    # rows of one sequence at different positions: blocks at or after a row's
+    # current block score highest, yet no row may select them
+    c_hi = 900
+    kx = RNG.integers(-4, 5, (c_hi, 256)).astype(np.float64)
+    qx = np.tile(RNG.integers(-4, 5, 256).astype(np.float64), (4, 1))
+    kx[600:] = 4 * np.sign(qx[0])
+    pos = np.array([600 * 8, 600 * 8 + 7, 700 * 8 + 3, 899 * 8 + 1])
+    got = O.index_topk_rows(qx, kx, pos, 512)
+    for i, t in enumerate(pos.tolist()):
+        c = t // 8
+        assert got[i].max() < c and len(set(got[i].tolist())) == 512
+    # a row whose history holds the strong blocks takes all of them that fit
+    assert set(range(600, 700)) <= set(got[2].tolist())
+
+
+def test_index_topk_rows_agrees_with_one_row_form():
+    kx = RNG.integers(-4, 5, (3000, 256)).astype(np.float64)
+    pos = RNG.integers(0, 3000 * 8, 40)
+    qx = RNG.integers(-4, 5, (40, 256)).astype(np.float64)
+    got = O.index_topk_rows(qx, kx, pos, 512)
+    for i, t in enumerate(pos.tolist()):
+        assert np.array_equal(got[i], O.index_topk_query(qx[i], kx, t, 512))
