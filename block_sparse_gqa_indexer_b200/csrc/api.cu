@@ -23,6 +23,7 @@ constexpr int kSeg = 8192;          // ... segments of rows longer than 16,384 b
 constexpr int kMaxSeg = 32;         // (kSeg * kMaxSeg >= S5_MAX_LEN / 8)
 constexpr int kMaxSplit = 8;        // partitions per (row, group) beyond what kMaxList forces
 constexpr int kScorePagesPerCta = 64;  // indexer CTA: 64 pages = 512 block keys = 256 KB
+constexpr int kMaxGridYZ = 65535;      // CUDA limit on gridDim.y and gridDim.z
 
 static_assert((long long)kSeg * kMaxSeg >= S5_MAX_LEN / S5_BLOCK_SIZE, "segments must cover the longest row");
 
@@ -376,6 +377,7 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
 
   // (one selection per KV group: every row takes the per-row kernel)
   if (mode == kModeSparse && sel_groups == 1 && use_tiles(b)) {
+    if (b->batch > kMaxGridYZ) return S5_ERR_UNSUPPORTED;  // the union kernel's grid.y
     // union lists and per-tile choice, then the shared-set tiles; the per-row
     // kernel below skips the rows those tiles computed
     const TileWs tw = tile_ws(b, topk, device_slots() / kCtasPerSm, false, w.end);
@@ -458,6 +460,7 @@ s5_status index_common(const s5_index_desc *index, const s5_batch_desc *batch, c
   if (batch->total_q == 0) return S5_OK;
   if (q_index == nullptr || sel == nullptr || sel_count == nullptr || !aligned16(q_index))
     return S5_ERR_INVALID_ARG;
+  if (batch->batch > kMaxGridYZ) return S5_ERR_UNSUPPORTED;  // sequences index grid.y / grid.z
   const long long rows = (long long)batch->total_q * groups;
   const IndexWs w = index_ws(batch, groups);
   if (w.two_stage && rows > 65535) return S5_ERR_UNSUPPORTED;  // stage 1 has one grid row per selection

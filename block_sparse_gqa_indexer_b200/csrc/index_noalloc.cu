@@ -30,7 +30,10 @@ constexpr int kMaxDevices = 64;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch on the current device (looked up on the
-// first call made with that device current).
+// first call made with that device current and kept for the life of the
+// process; a device reset unloads the module and leaves the kept address
+// stale, so after cudaDeviceReset this entry point must not be called again
+// in that process).
 cudaError_t scratch_address(void **out) {
   static std::mutex mu;
   static void *addr[kMaxDevices] = {};
@@ -77,6 +80,10 @@ extern "C" s5_status s5_index_score_topk_noalloc(const s5_index_desc *index, con
   if (stride > kNoAllocMaxHistory) return S5_ERR_WORKSPACE;
   const size_t need = kWsHeader + (size_t)batch->total_q * stride * sizeof(float);
   if (need > kNoAllocScratchBytes) return S5_ERR_WORKSPACE;
+  // launch limits of the scoring grid (sequences x 4-row tiles), checked
+  // before anything is enqueued: short histories let the scratch hold more
+  // rows than one sequence's tiles may span
+  if (batch->batch > 65535 || (batch->max_q + 3) / 4 > 65535) return S5_ERR_UNSUPPORTED;
 
   void *scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return S5_ERR_CUDA;

@@ -140,7 +140,9 @@ s5_status s5_workspace_size(const s5_batch_desc *batch, int32_t window, size_t *
  * Selection: the `topk` best blocks by (score descending, block index
  * ascending); all c blocks when c <= topk.  Written to sel[r][0..n-1] in
  * ascending block order, sel[r][n..topk-1] = -1, sel_count[r] = n.
- * topk in [1, 512].  sel / sel_count are device int32. */
+ * topk in [1, 512].  sel / sel_count are device int32.  At most 65,535
+ * sequences per batch (S5_ERR_UNSUPPORTED otherwise; also for the sparse
+ * attention of multi-token batches). */
 s5_status s5_index_score_topk(const s5_index_desc *index, const s5_batch_desc *batch,
                               const void *q_index, int32_t topk, int32_t *sel,
                               int32_t *sel_count, void *workspace, size_t workspace_bytes,
@@ -221,11 +223,15 @@ s5_status s5_sparse_gqa_attn_grouped(const s5_kv_desc *kv, const s5_batch_desc *
  *   16,384 history blocks per row (max_len <= 131,080) and
  *   256 + 4 * total_q * S bytes <= 8 MiB, S = (max_len - 1) / 8 rounded up to a
  *   multiple of 4; larger requests
- *   return S5_ERR_WORKSPACE with nothing enqueued.
+ *   return S5_ERR_WORKSPACE with nothing enqueued.  batch <= 65,535 and
+ *   max_q <= 262,140 (the scoring grid); larger ones return
+ *   S5_ERR_UNSUPPORTED with nothing enqueued.
  *   The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
  *   library routine.  The first call on a device (with that device current)
  *   looks up the array's device address once; make that first call before
- *   any stream capture.
+ *   any stream capture.  The address is kept for the life of the process: a
+ *   device reset (cudaDeviceReset) makes it stale, so do not call this entry
+ *   point again in a process after resetting the device.
  *   Every call shares the one array and leaves its contents behind; each call
  *   clears the part that must start at zero.  Calls that can overlap on the
  *   GPU (other streams, other host threads) race on the array: serialise them.

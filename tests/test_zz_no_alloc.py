@@ -37,9 +37,14 @@ def _reference(lib, key_pool, batch, qx):
 
 
 def test_noalloc_matches_workspace_path_twice(lib):
-    # first call: a varlen batch with short and long histories and a verify row group
+    # varlen batches with short and long histories, a verify row group and a
+    # chunk row, called back to back
     cases = [([20000, 300, 9000, 131072], [1, 1, 4, 1], 31),
-             ([50000, 4500, 70000], [2, 1, 3], 32)]
+             ([50000, 4500, 70000], [2, 1, 3], 32),
+             # a chunk row: 200 new tokens of one sequence (more than 16 row
+             # tiles of the scoring grid; the workspace path scores these on
+             # the tensor cores instead)
+             ([6000, 300], [200, 1], 35)]
     for ctx, nq, seed in cases:
         w, key_pool, qx, batch = _inputs(lib, ctx, nq, seed)
         want_sel, want_cnt = _reference(lib, key_pool, batch, qx)
