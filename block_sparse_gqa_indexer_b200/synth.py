@@ -322,8 +322,11 @@ class Workload:
         return own_s, own_p
 
     def kv_pools(self, device, pt: Optional[torch.Tensor] = None, pages_per_chunk: int = 2048,
-                 window_only: Optional[int] = None, upto: Optional[Sequence[int]] = None):
+                 window_only: Optional[int] = None, upto: Optional[Sequence[int]] = None, fp8: bool = False):
         """K and V pools, bf16 [num_pages][4][64][192] each, filled through the page table.
+
+        With ``fp8`` the pools hold the same values as one-byte E4M3 codes
+        (uint8, same shape; rounded by torch's float8_e4m3fn conversion).
 
         With ``window_only = W`` only pages that can hold one of the last W
         tokens before any query of the sequence are filled (the rest stay
@@ -363,6 +366,8 @@ class Workload:
             kv = normal_bf16(self.seed, self.tid(TID_V), idx)
             v_pool[p0:p1] = torch.where(valid, kv, torch.zeros((), dtype=torch.bfloat16, device=device))
             del kv, idx, valid
+        if fp8:
+            return to_e4m3_codes(k_pool), to_e4m3_codes(v_pool)
         return k_pool, v_pool
 
     def index_pool(self, device, pt: Optional[torch.Tensor] = None, pages_per_chunk: int = 16384,

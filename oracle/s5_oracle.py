@@ -71,6 +71,15 @@ bits with bias 7, 3 mantissa bits, subnormals, no infinities, S.1111.111 is
 NaN); a key byte stands for its exact E4M3 value and scores are then formed
 as for two-byte keys.
 
+One-byte KV for the sparse layer (the StepFun open-weights blog, section
+"Fitting it on a node", notes that SGLang can hold the full-attention layers'
+KV cache in FP8, a lossy format to be re-checked, and "What I'd check before
+deploying it" asks for speed and accuracy with and without it; the pages name
+neither the 8-bit format nor a scale): reading taken here, the same E4M3 format as the
+one-byte block keys, with one scale for K and one for V per layer; a stored K
+byte b stands for k_scale * E4M3(b) and a V byte for v_scale * E4M3(b), and
+attention is then defined exactly as for bf16 KV on those values.
+
 Parity status: the cache append is pinned by rebuilding the seeded pools of
 a whole batch from the pools of its cached prefix;
 block selection is pinned by brute force, tie cases and the
@@ -270,6 +279,20 @@ def swa_attention_query(q, t: int, k_seq, v_seq, window: int = WINDOW, sm_scale:
     """Sliding-window attention of one query at t."""
     T = swa_token_set(t, window)
     return gqa_attention(q, k_seq[T], v_seq[T], sm_scale)
+
+
+def sparse_attention_query_fp8kv(q, sel, t: int, k_codes_seq, v_codes_seq, k_scale: float, v_scale: float,
+                                 sm_scale: float = DEFAULT_SM_SCALE):
+    """Sparse-layer attention of one query at t over one-byte KV.
+
+    ``k_codes_seq[pos]`` / ``v_codes_seq[pos]`` give the stored E4M3 bytes
+    (uint8 [4][192]) of the query's sequence; a K byte stands for
+    k_scale * E4M3(byte), a V byte for v_scale * E4M3(byte).  The token set is
+    the sparse layer's (selected blocks + current block)."""
+    T = sparse_token_set(sel, t)
+    k_rows = float(k_scale) * decode_e4m3(k_codes_seq[T])
+    v_rows = float(v_scale) * decode_e4m3(v_codes_seq[T])
+    return gqa_attention(q, k_rows, v_rows, sm_scale)
 
 
 # ----------------------------------------------------------------------------

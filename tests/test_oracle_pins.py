@@ -609,3 +609,88 @@ def test_index_topk_rows_agrees_with_one_row_form():
     got = O.index_topk_rows(qx, kx, pos, 512)
     for i, t in enumerate(pos.tolist()):
         assert np.array_equal(got[i], O.index_topk_query(qx[i], kx, t, 512))
+
+
+# ---------------------------------------------------------------- one-byte (E4M3) KV
+
+def _codes(x):
+    return torch.as_tensor(np.asarray(x, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_fp8kv_single_token_returns_scaled_value():
+    # one readable token (t = 0, nothing selected): every head returns that
+    # token's V of its group, decoded and multiplied by v_scale, whatever K is
+    vals = RNG.integers(-16, 17, (1, 4, 192)).astype(np.float64)
+    kc = _codes(RNG.standard_normal((1, 4, 192)))
+    vc = _codes(vals)
+    q = RNG.standard_normal((64, 192))
+    out, lse = O.sparse_attention_query_fp8kv(q, np.full(512, -1), 0, kc, vc, 0.7, 2.5)
+    for h in range(64):
+        assert np.array_equal(out[h], 2.5 * vals[0, h // 16])
+
+
+def test_fp8kv_identical_keys_average_scaled_values():
+    # every key equal: uniform weights, so out = v_scale * mean of the decoded values
+    t = 8 * 600 + 3
+    kc = np.tile(_codes(RNG.standard_normal((1, 4, 192))), (t + 1, 1, 1))
+    vals = RNG.integers(-8, 9, (t + 1, 4, 192)).astype(np.float64) / 4.0  # exact in E4M3
+    vc = _codes(vals)
+    sel = np.sort(RNG.choice(600, 512, replace=False))
+    q = RNG.standard_normal((64, 192))
+    out, _ = O.sparse_attention_query_fp8kv(q, sel, t, kc, vc, 1.3, 0.5)
+    T = O.sparse_token_set(sel, t)
+    for h in range(64):
+        assert np.allclose(out[h], 0.5 * vals[T, h // 16].mean(axis=0), rtol=0, atol=1e-12)
+
+
+def test_fp8kv_two_tokens_weights_follow_k_scale():
+    # two tokens: the weight of the second is sigmoid(sm_scale * k_scale * q.(k1 - k0))
+    k = np.zeros((2, 4, 192))
+    k[0, :, 0] = 1.0
+    k[1, :, 0] = 3.0
+    v = np.zeros((2, 4, 192))
+    v[1, :, :] = 1.0  # out = weight of token 1
+    q = np.zeros((64, 192))
+    q[:, 0] = np.linspace(-2, 2, 64)
+    for k_scale in (0.25, 1.0, 3.0):
+        out, lse = O.sparse_attention_query_fp8kv(q, np.full(512, -1), 1, _codes(k), _codes(v), k_scale, 1.0, 0.5)
+        z = 0.5 * k_scale * q[:, 0] * (3.0 - 1.0)
+        assert np.allclose(out[:, 5], 1.0 / (1.0 + np.exp(-z)), rtol=0, atol=1e-12)
+        s0, s1 = 0.5 * k_scale * q[:, 0] * 1.0, 0.5 * k_scale * q[:, 0] * 3.0
+        assert np.allclose(lse, np.logaddexp(s0, s1), rtol=0, atol=1e-12)
+
+
+def test_fp8kv_equals_bf16_attention_on_representable_values():
+    # values exactly representable in E4M3 (and bf16): with unit scales the
+    # one-byte layer is the two-byte layer on the same values; with scales
+    # a, b it is the two-byte layer on a*K and b*V
+    t = 8 * 700 + 6
+    kv_vals = RNG.integers(-16, 17, (2, t + 1, 4, 192)).astype(np.float64) / 8.0
+    kc, vc = _codes(kv_vals[0]), _codes(kv_vals[1])
+    assert np.array_equal(O.decode_e4m3(kc), kv_vals[0]) and np.array_equal(O.decode_e4m3(vc), kv_vals[1])
+    sel = np.sort(RNG.choice(700, 512, replace=False))
+    q = RNG.standard_normal((64, 192))
+    o8, l8 = O.sparse_attention_query_fp8kv(q, sel, t, kc, vc, 1.0, 1.0)
+    o2, l2 = O.sparse_attention_query(q, sel, t, kv_vals[0], kv_vals[1])
+    assert np.allclose(o8, o2, rtol=0, atol=1e-12) and np.allclose(l8, l2, rtol=0, atol=1e-12)
+    o8s, l8s = O.sparse_attention_query_fp8kv(q, sel, t, kc, vc, 0.75, 3.0)
+    o2s, l2s = O.sparse_attention_query(q, sel, t, 0.75 * kv_vals[0], 3.0 * kv_vals[1])
+    assert np.allclose(o8s, o2s, rtol=0, atol=1e-12) and np.allclose(l8s, l2s, rtol=0, atol=1e-12)
+
+
+def test_fp8kv_reads_only_the_sparse_token_set():
+    # bytes outside the selected blocks and past t never change the result
+    t = 8 * 650 + 2
+    kc = _codes(RNG.standard_normal((t + 9, 4, 192)))
+    vc = _codes(RNG.standard_normal((t + 9, 4, 192)))
+    sel = np.sort(RNG.choice(650, 512, replace=False))
+    q = RNG.standard_normal((64, 192))
+    o1, _ = O.sparse_attention_query_fp8kv(q, sel, t, kc, vc, 1.0, 1.0)
+    unsel = sorted(set(range(650)) - set(sel.tolist()))[0]
+    kc2, vc2 = kc.copy(), vc.copy()
+    kc2[unsel * 8:unsel * 8 + 8] = 0x7E  # 448
+    vc2[unsel * 8:unsel * 8 + 8] = 0x7E
+    kc2[t + 1:] = 0x7E
+    vc2[t + 1:] = 0x7E
+    o2, _ = O.sparse_attention_query_fp8kv(q, sel, t, kc2, vc2, 1.0, 1.0)
+    assert np.array_equal(o1, o2)
