@@ -165,23 +165,54 @@ def _oracle_time(items) -> float:
     return time.perf_counter() - t0
 
 
-def _threads() -> int:
-    try:
-        import threadpoolctl
-        return max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info())
-    except Exception:
-        return os.cpu_count() or 1
+def _oracle_worker(batch, rows, repeats, barrier, results):
+    """One process of the parallel oracle leg: draw the inputs of `rows`, wait
+    for every worker, then run the oracle over them `repeats` times on one
+    thread (BLAS limited to 1)."""
+    import threadpoolctl
+    with threadpoolctl.threadpool_limits(1):
+        torch.set_num_threads(1)
+        items = _oracle_sample(_workload(0, batch), rows)
+        barrier.wait(timeout=600)
+        t0 = time.time()
+        for _ in range(repeats):
+            _oracle_time(items)
+        results.put((t0, time.time(), len(rows) * repeats))
 
 
-def cpu_baseline(w: S.Workload, n_rows: int = 16) -> dict:
-    rows = list(range(0, w.total_q, max(1, w.total_q // n_rows)))[:n_rows]
-    items = _oracle_sample(w, rows)
-    dt = _oracle_time(items)
-    b = R.sparse_decode_bytes([w.ctx[0]] * len(rows), [1] * len(rows))["total"]
-    return {"value": b / dt / 1e9, "unit": UNIT, "cores": _threads(), "kind": "oracle",
-            "sample": f"{len(rows)} of the 64 query rows (float64 numpy oracle: full-sort top-512 over 16,384 "
-                      f"block scores + sparse attention); {dt:.2f} s; inputs drawn before timing",
-            "queries_per_s": len(rows) / dt}
+def parallel_oracle(batch: int, rows: list, workers: int, repeats: int):
+    """Run the oracle over `rows` of the bench workload in `workers` spawned
+    processes (one thread each; rows dealt round-robin), all starting together.
+    Returns (query rows processed, wall seconds from first start to last end)."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    barrier = ctx.Barrier(workers)
+    results = ctx.Queue()
+    procs = [ctx.Process(target=_oracle_worker, args=(batch, rows[k::workers], repeats, barrier, results))
+             for k in range(workers)]
+    for p in procs:
+        p.start()
+    got = [results.get(timeout=900) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    t0 = min(g[0] for g in got)
+    t1 = max(g[1] for g in got)
+    return sum(g[2] for g in got), t1 - t0
+
+
+def cpu_baseline(w: S.Workload, repeats: int = 2) -> dict:
+    """The oracle on the host cores: every query row of the workload, spread
+    over one single-threaded process per core (at most one per row), each row
+    evaluated `repeats` times (about 20 s of CPU work in all)."""
+    rows = list(range(w.total_q))
+    workers = max(1, min(os.cpu_count() or 1, len(rows)))
+    n, dt = parallel_oracle(w.batch, rows, workers, repeats)
+    b = R.sparse_decode_bytes([w.ctx[0]] * n, [1] * n)["total"]
+    return {"value": b / dt / 1e9, "unit": UNIT, "cores": workers, "kind": "oracle",
+            "sample": f"all {len(rows)} query rows x {repeats} (float64 numpy oracle: full-sort top-512 over 16,384 "
+                      f"block scores + sparse attention) in {workers} single-threaded processes; {dt:.2f} s wall; "
+                      "inputs drawn before timing",
+            "queries_per_s": n / dt}
 
 
 def bench_config(batch: int, n: int) -> dict:
@@ -203,11 +234,13 @@ def run_reference(args) -> None:
     n = (args.warmup + args.steps) * per_step
     rows = [(i * 7) % w.total_q for i in range(n)]
     items = _oracle_sample(w, rows)
-    for i in range(args.warmup):
-        _oracle_time(items[i * per_step:(i + 1) * per_step])
-    times = []
-    for i in range(args.warmup, args.warmup + args.steps):
-        times.append(_oracle_time(items[i * per_step:(i + 1) * per_step]))
+    import threadpoolctl
+    with threadpoolctl.threadpool_limits(1):  # the oracle as it stands, on one core
+        for i in range(args.warmup):
+            _oracle_time(items[i * per_step:(i + 1) * per_step])
+        times = []
+        for i in range(args.warmup, args.warmup + args.steps):
+            times.append(_oracle_time(items[i * per_step:(i + 1) * per_step]))
     total = sum(times)
     b = R.sparse_decode_bytes([w.ctx[0]] * per_step, [1] * per_step)["total"]
     value = b * args.steps / total / 1e9
@@ -216,9 +249,10 @@ def run_reference(args) -> None:
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": bench_config(w.batch, args.gpus),
             "queries_per_s": per_step * args.steps / total,
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"{per_step} of the 64 query rows per step (float64 numpy oracle: full-sort "
-                                       f"top-512 over 16,384 block scores + sparse attention), {args.steps} steps"},
+                                       f"top-512 over 16,384 block scores + sparse attention) on one thread "
+                                       f"(BLAS limited to 1), {args.steps} steps"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -404,18 +438,25 @@ def run_config(args) -> None:
     print a JSON line with its own bytes / FLOPs (a measurement aid; the bench
     line is the default mode).  The step and each call are captured in CUDA
     graphs and replayed, so small batches are timed on the device rather than
-    by the host's launch rate."""
+    by the host's launch rate.  Each step is timed twice: with a 512 MiB
+    write between replays, which leaves none of the step's inputs in the
+    126 MB L2 (``ms_per_step``, the HBM figure), and replayed back to back
+    (``ms_per_step_warm``; inputs smaller than L2 then stay resident)."""
     from block_sparse_gqa_indexer_b200 import s5
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     layers = [S.shard(w, 0, args.shard) for w in S.config_workloads(args.config)]
+    if args.ctx is not None:  # the same batch with another cached length (e.g. a smaller profiling case)
+        for w in layers:
+            w.ctx = [args.ctx] * w.batch
     stream = torch.cuda.current_stream(dev)
     scale = 1.0 / (192 ** 0.5)
     calls, kinds, bytes_total, flops_total = [], [], 0, 0
     for li, w in enumerate(layers):
         swa = (args.config == 2) or (args.config == 5 and li < 3)
         pt = w.page_table()
-        k_pool, v_pool = w.kv_pools(dev, pt, window_only=S.WINDOW if swa else None)
+        kv8 = args.fp8_kv and not swa  # one-byte KV: sparse (full-attention) layers only
+        k_pool, v_pool = w.kv_pools(dev, pt, window_only=S.WINDOW if swa else None, fp8=kv8)
         batch = s5.Batch.from_host(pt, w.ctx, w.nq, dev)
         ws = s5.new_workspace(batch, window=S.WINDOW, device=dev)
         q, qx = w.queries(dev)
@@ -461,12 +502,17 @@ def run_config(args) -> None:
             calls.append(lambda kp=key_pool, b=batch, qx=qx, sel=sel, cnt=cnt, ws=ws, f=index_fn:
                          f(kp, b, qx, S.TOPK, sel, cnt, ws))
             kinds.append("index_fp8keys" if args.fp8_keys else "index")
-            calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, sel=sel, cnt=cnt, o=out, l=lse, ws=ws:
-                         s5.s5_sparse_gqa_attn(k, v, b, q, sel, cnt, S.TOPK, scale, o, l, ws))
-            kinds.append("sparse")
+            if kv8:
+                calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, sel=sel, cnt=cnt, o=out, l=lse, ws=ws:
+                             s5.s5_sparse_gqa_attn_fp8kv(k, v, b, q, sel, cnt, S.TOPK, scale, 1.0, 1.0, o, l, ws))
+                kinds.append("sparse_fp8kv")
+            else:
+                calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, sel=sel, cnt=cnt, o=out, l=lse, ws=ws:
+                             s5.s5_sparse_gqa_attn(k, v, b, q, sel, cnt, S.TOPK, scale, o, l, ws))
+                kinds.append("sparse")
             sp = R.sparse_decode_bytes(w.ctx, w.nq)
-            # one-byte keys: the indexer reads half the key bytes
-            bytes_total += sp["total"] - (sp["keys"] // 2 if args.fp8_keys else 0)
+            # one-byte keys: the indexer reads half the key bytes; one-byte KV: half the KV bytes
+            bytes_total += sp["total"] - (sp["keys"] // 2 if args.fp8_keys else 0) - (sp["kv"] // 2 if kv8 else 0)
             flops_total += R.sparse_flops(w.ctx, w.nq)["total"]
     for _ in range(args.warmup):
         for c in calls:
@@ -482,6 +528,8 @@ def run_config(args) -> None:
 
     step_graph = capture(calls)
     call_graphs = [capture([c]) for c in calls]
+    scratch = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush_graph = capture([lambda: scratch.fill_(1)])
     torch.cuda.synchronize(dev)
 
     def replay_ms(g, n):
@@ -494,16 +542,35 @@ def run_config(args) -> None:
         torch.cuda.synchronize(dev)
         return t0.elapsed_time(t1) / n
 
-    ms = replay_ms(step_graph, args.steps)
-    per_call = [replay_ms(g, args.steps) for g in call_graphs]
+    def replay_cold_ms(g, n):
+        # the flush runs before each replay's start event, so the event pair
+        # brackets the step alone, enqueued behind the flush
+        n = min(n, 500)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for e0, e1 in evs:
+            flush_graph.replay()
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+
+    ms_warm = replay_ms(step_graph, args.steps)
+    ms = replay_cold_ms(step_graph, args.steps)
+    per_call = [replay_cold_ms(g, args.steps) for g in call_graphs]
     peak, kind = _peaks()
     line = {"config": args.config, "ms_per_step": ms, "calls_ms": dict(zip([f"{k}{i}" for i, k in enumerate(kinds)],
                                                                            per_call)),
-            "timing": "CUDA-graph replay of the step (and of each call), CUDA events",
+            "ms_per_step_warm": ms_warm,
+            "timing": "CUDA-graph replay of the step (and of each call), CUDA events; ms_per_step and calls_ms: "
+                      "median over replays each preceded by a 512 MiB write (L2 flushed); ms_per_step_warm: "
+                      "back-to-back replays",
             "algorithmic_bytes": bytes_total, "useful_flops": flops_total,
             "gbs": bytes_total / (ms * 1e-3) / 1e9, "pct_hbm_peak": 100 * bytes_total / (ms * 1e-3) / 1e9 / peak,
             "useful_tflops": flops_total / (ms * 1e-3) / 1e12, "steps": args.steps, "warmup": args.warmup,
-            "append": bool(args.append), "grouped": bool(args.grouped), "fp8_keys": bool(args.fp8_keys)}
+            "gbs_warm": bytes_total / (ms_warm * 1e-3) / 1e9,
+            "append": bool(args.append), "grouped": bool(args.grouped), "fp8_keys": bool(args.fp8_keys),
+            "fp8_kv": bool(args.fp8_kv), "ctx_override": args.ctx}
     print(json.dumps(line), flush=True)
 
 
@@ -524,6 +591,10 @@ def main():
                     help="with --config: sparse layers select per KV group (4 indexer queries per token)")
     ap.add_argument("--fp8-keys", action="store_true",
                     help="with --config: block keys stored as one-byte E4M3 codes")
+    ap.add_argument("--ctx", type=int, default=None,
+                    help="with --config: every sequence's cached tokens (default: the configuration's)")
+    ap.add_argument("--fp8-kv", action="store_true",
+                    help="with --config: the sparse layers' K/V stored as one-byte E4M3 codes")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -531,6 +602,8 @@ def main():
         ap.error("--grouped selection runs on bf16 block keys only")
     if args.append and args.fp8_keys:
         ap.error("the cache append writes bf16 block keys")
+    if args.fp8_kv and (args.grouped or args.append):
+        ap.error("--fp8-kv runs the shared-selection sparse layer on a resident cache")
     if args.impl == "reference":
         args.steps = min(args.steps, 20)
         run_reference(args)

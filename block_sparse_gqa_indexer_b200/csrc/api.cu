@@ -294,6 +294,22 @@ bool make_kv_map(CUtensorMap *m, const void *pool, int num_pages) {
   return r == CUDA_SUCCESS;
 }
 
+// A one-byte (E4M3) K or V pool uint8 [num_pages][4][64][192] viewed as rows of
+// 192 = 3 x 64 bytes; one box is one 8-token block of one group: {64, 3, 8},
+// 1,536 bytes, 64-byte swizzle.
+bool make_kv8_map(CUtensorMap *m, const void *pool, int num_pages) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {64, 3, (cuuint64_t)num_pages * kKv * kPage};
+  cuuint64_t strides[2] = {64, (cuuint64_t)kD};
+  cuuint32_t box[3] = {64, 3, (cuuint32_t)kBlk};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(pool), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // A K or V pool as rows of 192 dims, each 8-row box landing plane-major: box
 // {64 dims, 8 rows, 3 planes} with the planes (128 B apart in memory) as the
 // outermost box dimension, so one copy places a whole 8-token block as three
@@ -330,13 +346,18 @@ bool make_k256_map(CUtensorMap *m, const void *base, long long rows) {
 
 s5_status cuda_status(cudaError_t e) { return e == cudaSuccess ? S5_OK : S5_ERR_CUDA; }
 
+// kv8: the pools hold one-byte E4M3 codes (K value = k_scale * code value,
+// V value = v_scale * code value); every row then takes the per-row kernel.
 s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, const void *q, const int32_t *sel,
                       const int32_t *sel_count, int32_t topk, int32_t window, float sm_scale, void *out,
-                      float *lse, void *ws, size_t ws_bytes, cudaStream_t stream, int sel_groups = 1) {
+                      float *lse, void *ws, size_t ws_bytes, cudaStream_t stream, int sel_groups = 1,
+                      bool kv8 = false, float k_scale = 1.f, float v_scale = 1.f) {
   s5_status st = check_batch(b);
   if (st != S5_OK) return st;
   if ((st = check_kv(kv)) != S5_OK) return st;
   if (!std::isfinite(sm_scale)) return S5_ERR_INVALID_ARG;
+  if (kv8 && (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !std::isfinite(sm_scale * k_scale)))
+    return S5_ERR_INVALID_ARG;
   if (mode == kModeSparse && (topk < 1 || topk > kMaxTopk)) return S5_ERR_INVALID_ARG;
   if (mode == kModeSwa && window < 1) return S5_ERR_INVALID_ARG;
   if (ws == nullptr) return S5_ERR_WORKSPACE;
@@ -348,8 +369,12 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   const AttnWs w = attn_ws(b, bpr, device_slots());
   if (ws_bytes < w.end) return S5_ERR_WORKSPACE;
   CUtensorMap tk, tv;
-  if (!make_kv_map(&tk, kv->k_pool, kv->num_pages) || !make_kv_map(&tv, kv->v_pool, kv->num_pages))
+  if (kv8) {
+    if (!make_kv8_map(&tk, kv->k_pool, kv->num_pages) || !make_kv8_map(&tv, kv->v_pool, kv->num_pages))
+      return S5_ERR_CUDA;
+  } else if (!make_kv_map(&tk, kv->k_pool, kv->num_pages) || !make_kv_map(&tv, kv->v_pool, kv->num_pages)) {
     return S5_ERR_CUDA;
+  }
   AttnArgs a{};
   a.q = q;
   a.sel = sel;
@@ -365,7 +390,9 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   a.total_q = b->total_q;
   a.max_len = b->max_len;
   a.num_pages = kv->num_pages;
-  a.scale_log2 = sm_scale * 1.4426950408889634f;
+  a.scale_log2 = (kv8 ? sm_scale * k_scale : sm_scale) * 1.4426950408889634f;
+  a.kv8 = kv8 ? 1 : 0;
+  a.v_scale = kv8 ? v_scale : 1.f;
   a.n_split = w.n_split;
   a.out = out;
   a.lse = lse;
@@ -375,8 +402,8 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
   a.row_skip = nullptr;
   a.err = reinterpret_cast<int32_t *>(ws);
 
-  // (one selection per KV group: every row takes the per-row kernel)
-  if (mode == kModeSparse && sel_groups == 1 && use_tiles(b)) {
+  // (one selection per KV group, or one-byte KV: every row takes the per-row kernel)
+  if (mode == kModeSparse && sel_groups == 1 && !kv8 && use_tiles(b)) {
     if (b->batch > kMaxGridYZ) return S5_ERR_UNSUPPORTED;  // the union kernel's grid.y
     // union lists and per-tile choice, then the shared-set tiles; the per-row
     // kernel below skips the rows those tiles computed
@@ -584,6 +611,14 @@ s5_status s5_sparse_gqa_attn_grouped(const s5_kv_desc *kv, const s5_batch_desc *
                                      s5_stream_t stream) {
   return attn_common(kModeSparse, kv, batch, q, sel, sel_count, topk, 0, sm_scale, out, lse, workspace,
                      workspace_bytes, reinterpret_cast<cudaStream_t>(stream), kKv);
+}
+
+s5_status s5_sparse_gqa_attn_fp8kv(const s5_kv_desc *kv, const s5_batch_desc *batch, const void *q,
+                                   const int32_t *sel, const int32_t *sel_count, int32_t topk, float sm_scale,
+                                   float k_scale, float v_scale, void *out, float *lse, void *workspace,
+                                   size_t workspace_bytes, s5_stream_t stream) {
+  return attn_common(kModeSparse, kv, batch, q, sel, sel_count, topk, 0, sm_scale, out, lse, workspace,
+                     workspace_bytes, reinterpret_cast<cudaStream_t>(stream), 1, true, k_scale, v_scale);
 }
 
 s5_status s5_swa_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, const void *q, int32_t window,

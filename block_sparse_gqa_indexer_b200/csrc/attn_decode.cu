@@ -26,6 +26,17 @@
 // This path is HBM-bound (16 FLOPs per gathered byte); its QK^T / PV run on
 // the tensor pipe only because the FP32 CUDA cores could not keep up with the
 // bandwidth.
+//
+// One-byte KV (sparse layer; StepFun open-weights blog, "Fitting it on a
+// node": FP8 KV for the full-attention layers): the same kernel with E4M3
+// blocks of 1,536 bytes, four stages per warp in the same ring.  Each E4M3
+// pair widens exactly to an f16 pair in registers (cvt), Q is staged as f16,
+// and the MMAs are f16 m16n8k16 with fp32 accumulation; k_scale is folded into
+// the softmax scale and v_scale into the final normalisation.  The blocks land
+// through a 64-byte-swizzled TMA box; inside every 16-dim k-step the dims are
+// permuted identically for Q and K, and the tokens of a block are taken in the
+// order 0 1 3 2 4 5 7 6, which together make every fragment load from the
+// swizzled tiles free of bank conflicts.
 #include <cuda.h>
 
 #include "s5_common.cuh"
@@ -36,19 +47,68 @@ namespace s5 {
 constexpr int kWarps = 4;
 constexpr int kStages = 2;
 constexpr int kStageBytes = 4 * kBlockBytes;  // K block A, K block B, V block A, V block B
+constexpr int kBlockBytes8 = kBlk * kD;       // 1,536 bytes: one block of one group, one-byte KV
+constexpr int kStages8 = 4;                   // one-byte KV: twice the stages in the same ring
+constexpr int kStageBytes8 = 4 * kBlockBytes8;
+static_assert(kStages8 * kStageBytes8 == kStages * kStageBytes, "both KV widths share one ring layout");
+constexpr int kMaxStages = kStages8;
 constexpr int kQStride = kD * 2 + 16;         // padded q row (bytes): conflict-free ldmatrix
 constexpr int kRingBytes = kWarps * kStages * kStageBytes;
 constexpr int kQBytes = kHpg * kQStride;
 constexpr int kListOff = kRingBytes + kQBytes;
 constexpr int kBarOff = kListOff + 2 * kMaxList * 4;
-constexpr int kAttnSmem = kBarOff + kWarps * kStages * 8 + 1024;  // + alignment slack
+constexpr int kAttnSmem = kBarOff + (kWarps * kMaxStages + 1) * 8 + 1024;  // + a stall barrier, alignment slack
 constexpr uint64_t kWaitNs = 2000000000ull;                       // 2 s per wait
+constexpr float kLazyMax = 8.0f;  // log2 units: a softmax reference max moves only when exceeded by more
 constexpr int kMaxSplitMerge = 32;
 
 // byte offset of (token row r, dim d) inside a 128B-swizzled [8][192] bf16 tile
 __device__ __forceinline__ uint32_t swz(int r, int d) {
   const uint32_t off = (uint32_t)((r * 3 + (d >> 6)) * 128 + (d & 63) * 2);
   return off ^ (((off >> 7) & 7u) << 4);
+}
+
+// byte offset of (token row r, dim d) inside a 64B-swizzled [8][192] one-byte
+// tile: the 16-byte unit of every 64-byte segment is XORed with bits 7..8 of
+// the offset (the TMA 64-byte swizzle)
+__device__ __forceinline__ uint32_t swz8(int r, int d) {
+  const uint32_t off = (uint32_t)(r * kD + d);
+  return off ^ (((off >> 7) & 3u) << 4);
+}
+
+// token of a block behind mma column n in the one-byte path (0 1 3 2 4 5 7 6)
+__device__ __forceinline__ int tok8(int n) { return n ^ ((n >> 1) & 1); }
+
+// f16 m16n8k16 with fp32 accumulate (both operands f16)
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// four E4M3 codes (byte i = element i) to their exact values as two f16 pairs:
+// lo = elements 0, 1 and hi = elements 2, 3 (first element in the low half);
+// one conversion instruction per pair, straight into the MMA operand register
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
+// eight bf16 values to f16 (round to nearest; exact within the f16 normal range)
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+  return make_uint4(pack_f16(bf16lo(v.x), bf16hi(v.x)), pack_f16(bf16lo(v.y), bf16hi(v.y)),
+                    pack_f16(bf16lo(v.z), bf16hi(v.z)), pack_f16(bf16lo(v.w), bf16hi(v.w)));
 }
 
 // Merge weights of the partitions of one (row, head): w[p] = exp2(lse_p - M) / L
@@ -110,10 +170,13 @@ __global__ void __launch_bounds__(kD / 4) s5_combine_kernel(const AttnArgs a) {
   if (threadIdx.x == 0 && a.lse != nullptr) a.lse[rh] = lse;
 }
 
-template <int MODE>
+template <int MODE, bool KV8>
 __global__ void __launch_bounds__(kWarps * 32, 2)
     gqa_decode_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v) {
+  constexpr int NST = KV8 ? kStages8 : kStages;         // ring stages per warp
+  constexpr int BB = KV8 ? kBlockBytes8 : kBlockBytes;  // one block of one group (K or V)
+  constexpr int SB = 4 * BB;                            // one stage: K A, K B, V A, V B
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *ring = smem;
@@ -133,12 +196,17 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   const int g = rg / a.total_q;
 
   // ---- the unit's token range -------------------------------------------------
-  if (tid < kWarps * kStages) mbar_init(bars + tid, 1);
+  uint64_t *stall_bar = bars + kWarps * NST;  // nothing ever arrives on it (expired-wait test hook)
+  if (tid <= kWarps * NST) mbar_init(bars + tid, 1);
   fence_mbar_init();
   // programmatic launch: everything above touches shared memory only; every
   // global input (batch data, q, the selection) is read after this wait
   pdl_wait();
   if (a.row_skip != nullptr && ld_cg(a.row_skip + r) != 0) return;  // row computed by the tile kernel
+  // expired-wait test hook (workspace header, zero in normal use): a nonzero
+  // count of nanoseconds makes each warp's first stage wait also wait that long
+  // on stall_bar and then leave through the expired-wait path below
+  const uint64_t stall_ns = (a.err != nullptr) ? ld_cg_u64(reinterpret_cast<const uint64_t *>(a.err) + kWsStallWord) : 0;
   int s = -1, t = -1, lo_tok = 0, n_list = 0, b_first = 0, n_sel = 0;
   // the selection this unit reads: the row's, or its KV group's (sel_groups = 4)
   const int srow = a.sel_groups > 1 ? r * a.sel_groups + g : r;
@@ -181,28 +249,28 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   const int w_beg = min(n_items, warp * per_w);
   const int w_n = min(n_items, w_beg + per_w) - w_beg;
   const int n_pairs = (w_n + 1) / 2;
-  uint8_t *wring = ring + warp * kStages * kStageBytes;
-  uint64_t *wbar = bars + warp * kStages;
+  uint8_t *wring = ring + warp * NST * SB;
+  uint64_t *wbar = bars + warp * NST;
   const uint64_t policy = policy_evict_first();
 
   auto issue = [&](int j) {  // lane 0 only
-    const int st = j % kStages;
-    uint8_t *buf = wring + st * kStageBytes;
+    const int st = j % NST;
+    uint8_t *buf = wring + st * SB;
     uint32_t bytes = 0;
     int rows[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int it = 2 * j + h;
       rows[h] = (it < w_n) ? brow[w_beg + it] : -1;
-      if (rows[h] >= 0) bytes += 2 * kBlockBytes;
+      if (rows[h] >= 0) bytes += 2 * BB;
     }
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(wbar + st, bytes);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       if (rows[h] >= 0) {
-        tma_load_3d(buf + h * kBlockBytes, &tm_k, 0, 0, rows[h], wbar + st, policy);
-        tma_load_3d(buf + (2 + h) * kBlockBytes, &tm_v, 0, 0, rows[h], wbar + st, policy);
+        tma_load_3d(buf + h * BB, &tm_k, 0, 0, rows[h], wbar + st, policy);
+        tma_load_3d(buf + (2 + h) * BB, &tm_v, 0, 0, rows[h], wbar + st, policy);
       }
     }
   };
@@ -235,7 +303,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   if (lane < w_n) resolve(lane);
   __syncwarp();
   if (lane == 0) {
-    for (int j = 0; j < kStages && j < n_pairs; ++j) issue(j);
+    for (int j = 0; j < NST && j < n_pairs; ++j) issue(j);
   }
   // the query tile of the group (16 heads x 192, padded rows) is read while
   // the first blocks are in flight: every thread's loads issued together
@@ -250,7 +318,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     for (int x = 0; x < kQv; ++x) {
       const int i = tid + x * kWarps * 32;
       const int h = i / (kD / 8), cc = i % (kD / 8);
-      *reinterpret_cast<uint4 *>(q_s + h * kQStride + cc * 16) = qv[x];
+      // one-byte KV: the f16 MMAs take Q as f16
+      *reinterpret_cast<uint4 *>(q_s + h * kQStride + cc * 16) = KV8 ? bf16x8_to_f16x8(qv[x]) : qv[x];
     }
   }
   for (int k = lane + 32; k < w_n; k += 32) resolve(k);
@@ -258,11 +327,41 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
 
   // Q fragments (A operand) for the 12 k-steps of 16 dims
   uint32_t qa[kD / 16][4];
-  {
+  if constexpr (KV8) {
+    // k-step 4c + j: lanes with lane % 4 == i hold dims 64c + 16i + 4j + {0,1} (k slots 2i, 2i+1)
+    // and + {2,3} (k slots 2i+8, 2i+9); the K fragments below use the same map
+    const int gq = lane >> 2, iq = lane & 3;
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      const uint4 *r0 = reinterpret_cast<const uint4 *>(q_s + gq * kQStride + (64 * c + 16 * iq) * 2);
+      const uint4 *r1 = reinterpret_cast<const uint4 *>(q_s + (gq + 8) * kQStride + (64 * c + 16 * iq) * 2);
+      const uint4 x0 = r0[0], x1 = r0[1], y0 = r1[0], y1 = r1[1];
+      const uint32_t wa[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      const uint32_t wb[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        qa[4 * c + j][0] = wa[2 * j];
+        qa[4 * c + j][1] = wb[2 * j];
+        qa[4 * c + j][2] = wa[2 * j + 1];
+        qa[4 * c + j][3] = wb[2 * j + 1];
+      }
+    }
+  } else {
     const int m = lane >> 3, rr = lane & 7;
     const uint32_t base = smem_u32(q_s) + ((m & 1) * 8 + rr) * kQStride + (m >> 1) * 16;
 #pragma unroll
     for (int kk = 0; kk < kD / 16; ++kk) ldsm_x4(base + kk * 32, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+  }
+  // one-byte KV: swizzled byte offsets of this lane's fragment loads inside a block tile
+  // (K: token tok8(lane/4), 16 dims per 64-dim chunk; V: tokens tok8(2i), tok8(2i+1), 8 dims)
+  uint32_t koff[3], voff0[3], voff1[3];
+  if constexpr (KV8) {
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      koff[c] = swz8(tok8(lane >> 2), 64 * c + 16 * (lane & 3));
+      voff0[c] = swz8(tok8(2 * (lane & 3)), 64 * c + 8 * (lane >> 2));
+      voff1[c] = swz8(tok8(2 * (lane & 3) + 1), 64 * c + 8 * (lane >> 2));
+    }
   }
 
   float o[kD / 8][4];
@@ -276,10 +375,12 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   int j_fail = n_pairs;
 
   for (int j = 0; j < n_pairs; ++j) {
-    const int st = j % kStages;
-    uint8_t *buf = wring + st * kStageBytes;
+    const int st = j % NST;
+    uint8_t *buf = wring + st * SB;
     // warp-uniform outcome: every lane leaves together if any lane's wait expired
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(wbar + st, (j / kStages) & 1, kWaitNs))) {
+    bool landed = mbar_wait_bounded(wbar + st, (j / NST) & 1, kWaitNs);
+    if (stall_ns != 0 && j == 0) landed = landed && mbar_wait_bounded(stall_bar, 0, stall_ns);
+    if (!__all_sync(0xffffffffu, landed)) {
       timed_out = true;
       j_fail = j;
       break;
@@ -295,40 +396,75 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       if (!full[h]) {
         // zero V rows of tokens that are not read (absent block, or outside
         // [lo_tok, t]): masked P is 0, and 0 * (stale or non-finite) must not leak
-        uint8_t *vb = buf + (2 + h) * kBlockBytes;
-        for (int x = lane; x < kBlk * 3 * 8; x += 32) {  // 24 rows of 128 B, 8 x 16 B each
-          const int row128 = x >> 3;
-          const int tok = row128 / 3;
-          const int pos = bk[h] * kBlk + tok;
-          if (bk[h] < 0 || pos < lo_tok || pos > t)
-            *reinterpret_cast<uint4 *>(vb + row128 * 128 + (x & 7) * 16) = make_uint4(0, 0, 0, 0);
+        uint8_t *vb = buf + (2 + h) * BB;
+        if constexpr (KV8) {
+          for (int x = lane; x < kBlk * (kD / 16); x += 32) {  // 8 token rows of 12 x 16 B
+            const int tok = x / (kD / 16);                      // (the swizzle stays inside a row)
+            const int pos = bk[h] * kBlk + tok;
+            if (bk[h] < 0 || pos < lo_tok || pos > t)
+              *reinterpret_cast<uint4 *>(vb + x * 16) = make_uint4(0, 0, 0, 0);
+          }
+        } else {
+          for (int x = lane; x < kBlk * 3 * 8; x += 32) {  // 24 rows of 128 B, 8 x 16 B each
+            const int row128 = x >> 3;
+            const int tok = row128 / 3;
+            const int pos = bk[h] * kBlk + tok;
+            if (bk[h] < 0 || pos < lo_tok || pos > t)
+              *reinterpret_cast<uint4 *>(vb + row128 * 128 + (x & 7) * 16) = make_uint4(0, 0, 0, 0);
+          }
         }
       }
     }
     __syncwarp();
     // ---- S = Q K^T for the two blocks ----
-    float sa[2][4];
+    // two accumulators per block (even / odd k-steps) halve the dependent MMA chain
+    float sa[2][4], sb[2][4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) sa[h][0] = sa[h][1] = sa[h][2] = sa[h][3] = 0.f;
-    const uint32_t kbase = smem_u32(buf);
+    for (int h = 0; h < 2; ++h) sa[h][0] = sa[h][1] = sa[h][2] = sa[h][3] = sb[h][0] = sb[h][1] = sb[h][2] = sb[h][3] = 0.f;
+    if constexpr (KV8) {
 #pragma unroll
-    for (int kk = 0; kk < kD / 16; kk += 2) {
-      const uint32_t off = swz(lr, 16 * kk + 8 * lm);
+      for (int c = 0; c < 3; ++c) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kbase + h * kBlockBytes + off, b0, b1, b2, b3);
-        mma_bf16_16816(sa[h], qa[kk], b0, b1);
-        mma_bf16_16816(sa[h], qa[kk + 1], b2, b3);
+        for (int h = 0; h < 2; ++h) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(buf + h * BB + koff[c]);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t b0, b1;
+            e4m3x4_to_f16x2x2(ww[j], b0, b1);
+            mma_f16_16816((j & 1) ? sb[h] : sa[h], qa[4 * c + j], b0, b1);
+          }
+        }
+      }
+    } else {
+      const uint32_t kbase = smem_u32(buf);
+#pragma unroll
+      for (int kk = 0; kk < kD / 16; kk += 2) {
+        const uint32_t off = swz(lr, 16 * kk + 8 * lm);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(kbase + h * BB + off, b0, b1, b2, b3);
+          mma_bf16_16816(sa[h], qa[kk], b0, b1);
+          mma_bf16_16816(sb[h], qa[kk + 1], b2, b3);
+        }
       }
     }
-    // ---- online softmax (rows: head tq-quad row lane/4 and lane/4 + 8) ----
-    float mx0 = m0, mx1 = m1;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sa[h][e] += sb[h][e];
+    // ---- online softmax (rows: head lane/4 and lane/4 + 8) ----
+    // m0 / m1 are reference maxima: the weights are exp2(s - m), and a
+    // reference moves (and O is rescaled) only when a row's maximum exceeds it
+    // by more than kLazyMax, so weights stay below 2^8 and after the first
+    // blocks O is almost never rescaled
+    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int pos = bk[h] * kBlk + 2 * tq + e;
+        const int pos = bk[h] * kBlk + (KV8 ? tok8(2 * tq + e) : 2 * tq + e);
         const bool v = bk[h] >= 0 && pos >= lo_tok && pos <= t;
         sa[h][e] = v ? sa[h][e] * sl2 : -INFINITY;
         sa[h][2 + e] = v ? sa[h][2 + e] * sl2 : -INFINITY;
@@ -340,11 +476,13 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float u0 = (mx0 == -INFINITY) ? 0.f : mx0;
-    const float u1 = (mx1 == -INFINITY) ? 0.f : mx1;
-    const float cr0 = hw_exp2(m0 - u0), cr1 = hw_exp2(m1 - u1);
-    m0 = mx0;
-    m1 = mx1;
+    const bool grow0 = mx0 > m0 + kLazyMax, grow1 = mx1 > m1 + kLazyMax;  // any finite max grows a -inf reference
+    const float cr0 = grow0 ? hw_exp2(m0 - mx0) : 1.f;  // (a -inf reference: 0, and O, l are still 0)
+    const float cr1 = grow1 ? hw_exp2(m1 - mx1) : 1.f;
+    if (grow0) m0 = mx0;
+    if (grow1) m1 = mx1;
+    const float u0 = (m0 == -INFINITY) ? 0.f : m0;  // still -inf: every score so far masked
+    const float u1 = (m1 == -INFINITY) ? 0.f : m1;
     float pr[2][4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -355,36 +493,63 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     }
     l0 = l0 * cr0 + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
     l1 = l1 * cr1 + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
+    if (__any_sync(0xffffffffu, grow0 || grow1)) {
 #pragma unroll
-    for (int i = 0; i < kD / 8; ++i) {
-      o[i][0] *= cr0;
-      o[i][1] *= cr0;
-      o[i][2] *= cr1;
-      o[i][3] *= cr1;
+      for (int i = 0; i < kD / 8; ++i) {
+        o[i][0] *= cr0;
+        o[i][1] *= cr0;
+        o[i][2] *= cr1;
+        o[i][3] *= cr1;
+      }
     }
-    const uint32_t pa[4] = {pack_bf16(pr[0][0], pr[0][1]), pack_bf16(pr[0][2], pr[0][3]),
-                            pack_bf16(pr[1][0], pr[1][1]), pack_bf16(pr[1][2], pr[1][3])};
     // ---- O += P V ----
-    const uint32_t vbase = smem_u32(buf) + 2 * kBlockBytes + (lm & 1) * kBlockBytes;
+    if constexpr (KV8) {
+      const uint32_t pa[4] = {pack_f16(pr[0][0], pr[0][1]), pack_f16(pr[0][2], pr[0][3]),
+                              pack_f16(pr[1][0], pr[1][1]), pack_f16(pr[1][2], pr[1][3])};
+      // n-tile 8c + e, column n = lane / 4: dim 64c + 8n + e; k slots 2i, 2i+1 (+8 for
+      // block B) are tokens tok8(2i), tok8(2i+1), as in S
 #pragma unroll
-    for (int np = 0; np < kD / 16; ++np) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(vbase + swz(lr, 16 * np + 8 * (lm >> 1)), b0, b1, b2, b3);
-      mma_bf16_16816(o[2 * np], pa, b0, b1);
-      mma_bf16_16816(o[2 * np + 1], pa, b2, b3);
+      for (int c = 0; c < 3; ++c) {
+        uint32_t bv[2][8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint8_t *vb = buf + (2 + h) * BB;
+          const uint2 x0 = *reinterpret_cast<const uint2 *>(vb + voff0[c]);  // token tok8(2i), 8 dims
+          const uint2 x1 = *reinterpret_cast<const uint2 *>(vb + voff1[c]);  // token tok8(2i+1)
+          const uint32_t p01 = __byte_perm(x0.x, x1.x, 0x5140), p23 = __byte_perm(x0.x, x1.x, 0x7362);
+          const uint32_t p45 = __byte_perm(x0.y, x1.y, 0x5140), p67 = __byte_perm(x0.y, x1.y, 0x7362);
+          e4m3x4_to_f16x2x2(p01, bv[h][0], bv[h][1]);
+          e4m3x4_to_f16x2x2(p23, bv[h][2], bv[h][3]);
+          e4m3x4_to_f16x2x2(p45, bv[h][4], bv[h][5]);
+          e4m3x4_to_f16x2x2(p67, bv[h][6], bv[h][7]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mma_f16_16816(o[8 * c + e], pa, bv[0][e], bv[1][e]);
+      }
+    } else {
+      const uint32_t pa[4] = {pack_bf16(pr[0][0], pr[0][1]), pack_bf16(pr[0][2], pr[0][3]),
+                              pack_bf16(pr[1][0], pr[1][1]), pack_bf16(pr[1][2], pr[1][3])};
+      const uint32_t vbase = smem_u32(buf) + 2 * BB + (lm & 1) * BB;
+#pragma unroll
+      for (int np = 0; np < kD / 16; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vbase + swz(lr, 16 * np + 8 * (lm >> 1)), b0, b1, b2, b3);
+        mma_bf16_16816(o[2 * np], pa, b0, b1);
+        mma_bf16_16816(o[2 * np + 1], pa, b2, b3);
+      }
     }
     // order this stage's generic reads / zero fills before the next async-proxy write into it
     fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0 && j + kStages < n_pairs) issue(j + kStages);
+    if (lane == 0 && j + NST < n_pairs) issue(j + NST);
   }
   // a warp may leave the loop early only after a wait expired
   timed_out = __any_sync(0xffffffffu, timed_out);
   if (timed_out) {
     if (lane == 0) record_error(a.err, S5_ERR_TIMEOUT, r);
     // drain: wait (bounded) for the copies still in flight (issued, not consumed)
-    for (int j2 = j_fail; j2 < n_pairs && j2 < j_fail + kStages; ++j2)
-      mbar_wait_bounded(wbar + (j2 % kStages), (j2 / kStages) & 1, kWaitNs);
+    for (int j2 = j_fail; j2 < n_pairs && j2 < j_fail + NST; ++j2)
+      mbar_wait_bounded(wbar + (j2 % NST), (j2 / NST) & 1, kWaitNs);
     m0 = m1 = -INFINITY;
     l0 = l1 = 0.f;
   }
@@ -397,12 +562,32 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   float *ow = reinterpret_cast<float *>(wring);  // [16][192] fp32, then m[16], l[16]
   {
     const int r0 = lane >> 2;
+    const float z = timed_out ? 0.f : 1.f;
+    if constexpr (KV8) {
+      // n-tile 8c + e holds dims 64c + 16 tq + e (o[.][0], o[.][2]) and 64c + 16 tq + 8 + e ([1], [3])
 #pragma unroll
-    for (int i = 0; i < kD / 8; ++i) {
-      const int col = i * 8 + 2 * tq;
-      const float z = timed_out ? 0.f : 1.f;
-      *reinterpret_cast<float2 *>(ow + r0 * kD + col) = make_float2(o[i][0] * z, o[i][1] * z);
-      *reinterpret_cast<float2 *>(ow + (r0 + 8) * kD + col) = make_float2(o[i][2] * z, o[i][3] * z);
+      for (int c = 0; c < 3; ++c) {
+        float *d0 = ow + r0 * kD + 64 * c + 16 * tq;
+        float *d1 = ow + (r0 + 8) * kD + 64 * c + 16 * tq;
+#pragma unroll
+        for (int e = 0; e < 8; e += 4) {
+          *reinterpret_cast<float4 *>(d0 + e) = make_float4(o[8 * c + e][0] * z, o[8 * c + e + 1][0] * z,
+                                                            o[8 * c + e + 2][0] * z, o[8 * c + e + 3][0] * z);
+          *reinterpret_cast<float4 *>(d0 + 8 + e) = make_float4(o[8 * c + e][1] * z, o[8 * c + e + 1][1] * z,
+                                                                o[8 * c + e + 2][1] * z, o[8 * c + e + 3][1] * z);
+          *reinterpret_cast<float4 *>(d1 + e) = make_float4(o[8 * c + e][2] * z, o[8 * c + e + 1][2] * z,
+                                                            o[8 * c + e + 2][2] * z, o[8 * c + e + 3][2] * z);
+          *reinterpret_cast<float4 *>(d1 + 8 + e) = make_float4(o[8 * c + e][3] * z, o[8 * c + e + 1][3] * z,
+                                                                o[8 * c + e + 2][3] * z, o[8 * c + e + 3][3] * z);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < kD / 8; ++i) {
+        const int col = i * 8 + 2 * tq;
+        *reinterpret_cast<float2 *>(ow + r0 * kD + col) = make_float2(o[i][0] * z, o[i][1] * z);
+        *reinterpret_cast<float2 *>(ow + (r0 + 8) * kD + col) = make_float2(o[i][2] * z, o[i][3] * z);
+      }
     }
     if (tq == 0) {
       ow[kHpg * kD + r0] = m0;
@@ -419,7 +604,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
-      const float *oww = reinterpret_cast<const float *>(ring + w * kStages * kStageBytes);
+      const float *oww = reinterpret_cast<const float *>(ring + w * NST * SB);
       mw[w] = oww[kHpg * kD + h];
       lw[w] = oww[kHpg * kD + kHpg + h];
       M = fmaxf(M, mw[w]);
@@ -431,7 +616,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       sc[w] = (lw[w] > 0.f) ? hw_exp2(mw[w] - Mu) : 0.f;
       L += lw[w] * sc[w];
     }
-    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    // (one-byte KV: the values are v_scale times their codes)
+    const float inv = (L > 0.f) ? (KV8 ? a.v_scale : 1.f) / L : 0.f;
     const int hg = g * kHpg + h;
     const size_t rh = (size_t)r * kHeads + hg;
     float acc[24];
@@ -439,7 +625,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     for (int e = 0; e < 24; ++e) acc[e] = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
-      const float *oww = reinterpret_cast<const float *>(ring + w * kStages * kStageBytes) + h * kD + d0;
+      const float *oww = reinterpret_cast<const float *>(ring + w * NST * SB) + h * kD + d0;
 #pragma unroll
       for (int e = 0; e < 24; e += 4) {
         const float4 v = *reinterpret_cast<const float4 *>(oww + e);
@@ -533,7 +719,9 @@ cudaError_t launch_gqa_decode(int mode, const AttnArgs &a, const CUtensorMap &tk
   if (n_cta > 0x7fffffffLL) return cudaErrorInvalidValue;
   dim3 grid((unsigned)n_cta);
   cudaError_t e;
-  auto kernel = (mode == kModeSparse) ? gqa_decode_kernel<kModeSparse> : gqa_decode_kernel<kModeSwa>;
+  auto kernel = (mode == kModeSparse) ? (a.kv8 ? gqa_decode_kernel<kModeSparse, true>
+                                                : gqa_decode_kernel<kModeSparse, false>)
+                                      : gqa_decode_kernel<kModeSwa, false>;
   e = ensure_dynamic_smem(reinterpret_cast<const void *>(kernel), kAttnSmem);
   if (e != cudaSuccess) return e;
   // programmatic stream serialization: launch and barrier setup overlap the

@@ -27,6 +27,9 @@ constexpr int kBlockBytes = kBlk * kD * 2;  // 3,072 bytes: one block of one gro
 constexpr size_t kWsHeader = 256;
 constexpr size_t kWsCounterBytes = 16384;
 constexpr size_t kWsFixed = kWsHeader + kWsCounterBytes;  // first byte of per-call scratch
+// 64-bit word 8 of the header (bytes 64..71): the expired-wait test hook of
+// the per-row attention kernel (S5_WS_TEST_STALL_OFFSET), zero in normal use
+constexpr int kWsStallWord = S5_WS_TEST_STALL_OFFSET / 8;
 
 // Loads that stay after a preceding wait or fence in program order (asm
 // volatile, L2-coherent).  Used for every read of data another kernel or CTA
@@ -40,6 +43,11 @@ __device__ __forceinline__ int32_t ld_cg(const int32_t *p) {
 __device__ __forceinline__ uint32_t ld_cg(const uint32_t *p) {
   uint32_t v;
   asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t ld_cg_u64(const uint64_t *p) {
+  uint64_t v;
+  asm volatile("ld.global.cg.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
 __device__ __forceinline__ float ld_cg(const float *p) {

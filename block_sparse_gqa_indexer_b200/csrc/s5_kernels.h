@@ -78,6 +78,8 @@ struct AttnArgs {
   uint32_t *merge_cnt;  // [total_q * 4] arrival counters (zero between calls), or null: separate merge kernel
   const int32_t *row_skip;  // [total_q]: nonzero for rows the shared-set tile kernel computes, or null
   int32_t *err;
+  int kv8;        // nonzero: K / V pools hold one-byte E4M3 codes (sparse mode only)
+  float v_scale;  // one-byte KV: value of a V code = v_scale * E4M3(code) (k_scale is in scale_log2)
 };
 
 // Prefill-sized batches: block keys gathered per sequence, then a tcgen05 GEMM.

@@ -21,17 +21,19 @@ if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m block_sparse_gqa_indexer_b200.build`")
 _lib = ctypes.CDLL(LIB_PATH)
 
-ABI_VERSION = 101  # S5_ABI_VERSION of the header this binding follows
+ABI_VERSION = 102  # S5_ABI_VERSION of the header this binding follows
 N_HEADS, N_KV, HEAD_DIM, PAGE, BLOCK, INDEX_DIM, MAX_TOPK = 64, 4, 192, 64, 8, 256, 512
 MAX_LEN = 1 << 21
 DEFAULT_SM_SCALE = 1.0 / math.sqrt(HEAD_DIM)
 
 S5_OK, S5_ERR_INVALID_ARG, S5_ERR_UNSUPPORTED, S5_ERR_CUDA, S5_ERR_DEVICE_BOUNDS, S5_ERR_TIMEOUT, \
     S5_ERR_WORKSPACE = range(7)
+S5_WS_FIXED_BYTES = 256 + 16384
+S5_WS_TEST_STALL_OFFSET = 64  # expired-wait test hook (include/s5attn.h); zero in normal use
 
 # exported symbols (every declaration of include/s5attn.h)
 SYMBOLS = ("s5_workspace_size", "s5_index_score_topk", "s5_sparse_gqa_attn", "s5_swa_gqa_attn",
-           "s5_index_score_topk_fp8",
+           "s5_index_score_topk_fp8", "s5_sparse_gqa_attn_fp8kv",
            "s5_workspace_size_grouped", "s5_index_score_topk_grouped", "s5_sparse_gqa_attn_grouped",
            "s5_index_score_topk_noalloc", "s5_append_kv", "s5_reset_device_error", "s5_get_device_error",
            "s5_status_string", "s5_abi_version")
@@ -62,6 +64,9 @@ _lib.s5_sparse_gqa_attn.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(Batch
 _lib.s5_swa_gqa_attn.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(BatchDesc), _P, _I, ctypes.c_float, _P,
                                  _P, _P, ctypes.c_size_t, _P]
 _lib.s5_index_score_topk_fp8.argtypes = _lib.s5_index_score_topk.argtypes
+_lib.s5_sparse_gqa_attn_fp8kv.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(BatchDesc), _P, _P, _P, _I,
+                                          ctypes.c_float, ctypes.c_float, ctypes.c_float, _P, _P, _P,
+                                          ctypes.c_size_t, _P]
 _lib.s5_workspace_size_grouped.argtypes = _lib.s5_workspace_size.argtypes
 _lib.s5_index_score_topk_grouped.argtypes = _lib.s5_index_score_topk.argtypes
 _lib.s5_sparse_gqa_attn_grouped.argtypes = _lib.s5_sparse_gqa_attn.argtypes
@@ -245,6 +250,28 @@ def s5_sparse_gqa_attn(k_pool, v_pool, batch: Batch, q, sel, sel_count, topk: in
     _check(_lib.s5_sparse_gqa_attn(ctypes.byref(kv), ctypes.byref(batch.desc), _ptr(q), _ptr(sel),
                                    _ptr(sel_count), int(topk), float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws),
                                    ws.numel(), _stream(stream)), "s5_sparse_gqa_attn")
+
+
+def s5_sparse_gqa_attn_fp8kv(k_pool, v_pool, batch: Batch, q, sel, sel_count, topk: int, sm_scale: float,
+                             k_scale: float, v_scale: float, out, lse, ws, stream=None):
+    """Sparse attention over one-byte KV: k_pool / v_pool uint8 E4M3 codes
+    [num_pages][4][64][192]; a K code stands for k_scale times its value, a V
+    code for v_scale times its value."""
+    _need(k_pool, torch.uint8, "k_pool")
+    _need(v_pool, torch.uint8, "v_pool", tuple(k_pool.shape))
+    sh = k_pool.shape
+    kv = KvDesc(k_pool.data_ptr(), v_pool.data_ptr(), sh[0], sh[2], sh[1], sh[3])
+    _need(q, torch.bfloat16, "q", (batch.total_q, N_HEADS, HEAD_DIM))
+    _need(sel, torch.int32, "sel", (batch.total_q, topk))
+    _need(sel_count, torch.int32, "sel_count", (batch.total_q,))
+    _need(out, torch.bfloat16, "out", (batch.total_q, N_HEADS, HEAD_DIM))
+    if lse is not None:
+        _need(lse, torch.float32, "lse", (batch.total_q, N_HEADS))
+    _need(ws, torch.uint8, "ws")
+    _check(_lib.s5_sparse_gqa_attn_fp8kv(ctypes.byref(kv), ctypes.byref(batch.desc), _ptr(q), _ptr(sel),
+                                         _ptr(sel_count), int(topk), float(sm_scale), float(k_scale),
+                                         float(v_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                         _stream(stream)), "s5_sparse_gqa_attn_fp8kv")
 
 
 def s5_sparse_gqa_attn_grouped(k_pool, v_pool, batch: Batch, q, sel, sel_count, topk: int, sm_scale: float,

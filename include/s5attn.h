@@ -87,8 +87,9 @@ typedef enum {
 #define S5_MAX_LEN (1 << 21) /* longest sequence (cached + new tokens) */
 
 /* ABI version (major * 100 + minor): 1.01 added the cache append, the
- * per-KV-group entry points and the one-byte-key indexer. */
-#define S5_ABI_VERSION 101
+ * per-KV-group entry points and the one-byte-key indexer; 1.02 the sparse
+ * attention over one-byte KV. */
+#define S5_ABI_VERSION 102
 
 /* One attention layer's paged KV cache. */
 typedef struct {
@@ -127,6 +128,15 @@ typedef struct {
  * rest is per-call scratch with no state between calls.  Calls that share a
  * workspace must be ordered (one stream). */
 #define S5_WS_FIXED_BYTES (256 + 16384)
+/* Test hook for the bounded waits (not for normal use): a nonzero unsigned
+ * 64-bit count of nanoseconds stored at this byte offset of a workspace makes
+ * every CTA of the per-row attention kernel (s5_sparse_gqa_attn decode rows,
+ * s5_sparse_gqa_attn_grouped, s5_sparse_gqa_attn_fp8kv, s5_swa_gqa_attn)
+ * wait that long, after its first block copies land, on a barrier that nothing
+ * arrives on, and then take the expired-wait path: it records S5_ERR_TIMEOUT,
+ * waits (bounded) for its copies still in flight and returns with zero output
+ * for its unit.  Zeroing the workspace or s5_reset_device_error clears it. */
+#define S5_WS_TEST_STALL_OFFSET 64
 s5_status s5_workspace_size(const s5_batch_desc *batch, int32_t window, size_t *bytes);
 
 /* Indexer: score every history block of every query row and keep the best
@@ -184,6 +194,24 @@ s5_status s5_swa_gqa_attn(const s5_kv_desc *kv, const s5_batch_desc *batch, cons
 s5_status s5_index_score_topk_fp8(const s5_index_desc *index, const s5_batch_desc *batch, const void *q_index,
                                   int32_t topk, int32_t *sel, int32_t *sel_count, void *workspace,
                                   size_t workspace_bytes, s5_stream_t stream);
+
+/* Sparse gathered GQA over one-byte KV (StepFun open-weights blog, "Fitting
+ * it on a node": the full-attention layers' KV cache can be held in FP8, a
+ * lossy format to be re-checked).  kv->k_pool / kv->v_pool hold E4M3 codes,
+ * uint8 [num_pages][4][64][192] (one block of one group = 1,536 contiguous
+ * bytes), 16-byte aligned; a K code stands for k_scale * E4M3(code) and a V
+ * code for v_scale * E4M3(code) (E4M3: the 8-bit float of the OCP FP8
+ * specification, bias 7, 3 mantissa bits, no infinities).  With those values
+ * the result is defined exactly as for s5_sparse_gqa_attn; every row takes
+ * the per-row kernel.  Products run on f16 tensor cores: every E4M3 value is
+ * an f16 value, and q is rounded to f16 (exact for bf16 values of magnitude
+ * 2^-14 .. 65,504; larger magnitudes overflow).  k_scale, v_scale and
+ * sm_scale * k_scale must be finite (S5_ERR_INVALID_ARG).  The workspace of
+ * s5_workspace_size covers this call. */
+s5_status s5_sparse_gqa_attn_fp8kv(const s5_kv_desc *kv, const s5_batch_desc *batch, const void *q,
+                                   const int32_t *sel, const int32_t *sel_count, int32_t topk, float sm_scale,
+                                   float k_scale, float v_scale, void *out, float *lse, void *workspace,
+                                   size_t workspace_bytes, s5_stream_t stream);
 
 /* Per-KV-group selection (StepFun open-weights blog, "What sparse attention
  * does and doesn't save": each KV group picks its own blocks).  The block

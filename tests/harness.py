@@ -29,14 +29,20 @@ class LazyRows:
 
 
 class DeviceInputs:
-    """Everything the CUDA path needs for one layer, resident on the device."""
+    """Everything the CUDA path needs for one layer, resident on the device.
 
-    def __init__(self, w: S.Workload, s5, device="cuda", window_only=None, with_index=True):
+    ``draw`` is where the generator runs (default: on ``device``; "cpu" draws
+    on the host and copies the tensors over once)."""
+
+    def __init__(self, w: S.Workload, s5, device="cuda", window_only=None, with_index=True, draw=None):
         self.w = w
         self.pt = w.page_table()
-        self.k_pool, self.v_pool = w.kv_pools(device, self.pt, window_only=window_only)
-        self.key_pool = w.index_pool(device, self.pt) if with_index else None
-        self.q, self.qx = w.queries(device)
+        draw = device if draw is None else draw
+        k_pool, v_pool = w.kv_pools(draw, self.pt, window_only=window_only)
+        self.k_pool, self.v_pool = k_pool.to(device), v_pool.to(device)
+        self.key_pool = w.index_pool(draw, self.pt).to(device) if with_index else None
+        q, qx = w.queries(draw)
+        self.q, self.qx = q.to(device), qx.to(device)
         self.batch = s5.Batch.from_host(self.pt, w.ctx, w.nq, device)
         self.ws = s5.new_workspace(self.batch, window=S.WINDOW, device=device)
         tq = w.total_q

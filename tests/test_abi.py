@@ -209,3 +209,34 @@ def test_grouped_and_fp8_entries_validate_like_the_shared_ones(s5):
                  None) == s5.S5_OK
     n = ctypes.c_size_t(0)
     assert s5._lib.s5_workspace_size_grouped(ctypes.byref(b), -1, ctypes.byref(n)) == s5.S5_ERR_INVALID_ARG
+
+
+def test_workspace_constants_match_header(s5):
+    text = open(HEADER).read()
+    m = re.search(r"#define S5_WS_FIXED_BYTES \((\d+) \+ (\d+)\)", text)
+    assert m and int(m.group(1)) + int(m.group(2)) == s5.S5_WS_FIXED_BYTES
+    m = re.search(r"#define S5_WS_TEST_STALL_OFFSET (\d+)", text)
+    assert m and int(m.group(1)) == s5.S5_WS_TEST_STALL_OFFSET
+    # the hook lies in the zeroed header, clear of the error record (bytes 0..7)
+    assert 8 <= s5.S5_WS_TEST_STALL_OFFSET and s5.S5_WS_TEST_STALL_OFFSET + 8 <= 256
+
+
+def test_fp8_kv_entry_checks(s5):
+    fake = ctypes.c_void_p(0x1000)
+    b = _batch()
+    kv = s5.KvDesc(0x1000, 0x1000, 8, 64, 4, 192)
+    f = s5._lib.s5_sparse_gqa_attn_fp8kv
+    # non-finite scales (or an overflowing sm_scale * k_scale), bad top-k, short workspace, unaligned pool
+    for ks, vs, sm in [(float("nan"), 1.0, 0.1), (1.0, float("inf"), 0.1), (1e38, 1.0, 1e3)]:
+        assert f(ctypes.byref(kv), ctypes.byref(b), fake, fake, fake, 512, sm, ks, vs, fake, None, fake, 1 << 30,
+                 None) == s5.S5_ERR_INVALID_ARG
+    assert f(ctypes.byref(kv), ctypes.byref(b), fake, fake, fake, 0, 0.1, 1.0, 1.0, fake, None, fake, 1 << 30,
+             None) == s5.S5_ERR_INVALID_ARG
+    assert f(ctypes.byref(kv), ctypes.byref(b), fake, fake, fake, 512, 0.1, 1.0, 1.0, fake, None, fake, 16,
+             None) == s5.S5_ERR_WORKSPACE
+    kv_bad = s5.KvDesc(0x1008, 0x1000, 8, 64, 4, 192)
+    assert f(ctypes.byref(kv_bad), ctypes.byref(b), fake, fake, fake, 512, 0.1, 1.0, 1.0, fake, None, fake, 1 << 30,
+             None) == s5.S5_ERR_INVALID_ARG
+    kv_geo = s5.KvDesc(0x1000, 0x1000, 8, 64, 4, 128)
+    assert f(ctypes.byref(kv_geo), ctypes.byref(b), fake, fake, fake, 512, 0.1, 1.0, 1.0, fake, None, fake, 1 << 30,
+             None) == s5.S5_ERR_UNSUPPORTED
