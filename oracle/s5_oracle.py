@@ -375,6 +375,47 @@ def append_to_paged_cache(k_pool, v_pool, key_pool, page_table, ctx, nq, k_new, 
 # one-byte block keys: the E4M3 value of each byte   [SAV]
 # ----------------------------------------------------------------------------
 
+def encode_e4m3(x) -> np.ndarray:
+    """E4M3 code (uint8) of each value: the nearest E4M3 value, ties to the
+    code with an even last mantissa bit; magnitudes beyond the largest finite
+    value (448) saturate to it; NaN gives the NaN code 0x7F.  -0.0 keeps its
+    sign (0x80).  Values are compared exactly in float64 against the 127
+    non-negative finite codes listed by ``decode_e4m3``."""
+    x = np.asarray(x, dtype=np.float64)
+    grid = decode_e4m3(np.arange(0x7F, dtype=np.uint8))  # codes 0x00 .. 0x7E, ascending values
+    mag = np.minimum(np.abs(x), grid[-1])
+    hi = np.clip(np.searchsorted(grid, mag, side="left"), 0, len(grid) - 1)  # first grid value >= mag
+    lo = np.maximum(hi - 1, 0)
+    d_lo = mag - grid[lo]
+    d_hi = grid[hi] - mag
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.int64)
+    code = np.where(mag == grid[hi], hi, code)  # exact hits (including 0)
+    code = code | np.where(np.signbit(x), 0x80, 0)
+    return np.where(np.isnan(x), 0x7F, code).astype(np.uint8)
+
+
+def quantize_kv_e4m3(x, scale: float) -> np.ndarray:
+    """One-byte codes stored for values x with a per-layer scale: the E4M3
+    code of the fp32 product x * fl32(1 / scale) (one fp32 rounding, then
+    encode_e4m3), so that a code stands for about x / scale."""
+    inv = np.float32(1.0) / np.float32(scale)
+    prod = np.asarray(x, dtype=np.float32) * inv  # IEEE fp32 multiply
+    return encode_e4m3(prod.astype(np.float64))
+
+
+def append_to_paged_cache_fp8(k_pool, v_pool, page_table, ctx, nq, k_new, v_new, k_scale: float, v_scale: float):
+    """The one-byte K / V pools after appending the new tokens of a varlen
+    batch: row r's values are stored as quantize_kv_e4m3(k_new[r], k_scale)
+    and quantize_kv_e4m3(v_new[r], v_scale), at the slots the bf16 append
+    uses (no block keys: the block-key pool is written by the bf16-key or
+    one-byte-key path of the indexer's own append)."""
+    k_codes = quantize_kv_e4m3(np.asarray(k_new, dtype=np.float64), k_scale)
+    v_codes = quantize_kv_e4m3(np.asarray(v_new, dtype=np.float64), v_scale)
+    k_out, v_out, _ = append_to_paged_cache(k_pool, v_pool, None, page_table, ctx, nq, k_codes, v_codes, None)
+    return k_out, v_out
+
+
 def decode_e4m3(b) -> np.ndarray:
     """Exact float64 value of each E4M3 byte (uint8 array of any shape).
 

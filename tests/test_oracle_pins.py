@@ -694,3 +694,59 @@ def test_fp8kv_reads_only_the_sparse_token_set():
     vc2[t + 1:] = 0x7E
     o2, _ = O.sparse_attention_query_fp8kv(q, sel, t, kc2, vc2, 1.0, 1.0)
     assert np.array_equal(o1, o2)
+
+
+# ---------------------------------------------------------------- E4M3 encoding (one-byte KV append)
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    b = np.arange(256, dtype=np.uint8)
+    v = O.decode_e4m3(b)
+    fin = ~np.isnan(v)
+    assert np.array_equal(O.encode_e4m3(v[fin]), b[fin])  # -0.0 -> 0x80 included
+
+
+def test_e4m3_encode_ties_saturation_nan():
+    # midpoints go to the code with an even mantissa: 1.0 = 0x38, 1.125 = 0x39, 1.25 = 0x3A
+    assert O.encode_e4m3(1.0625) == 0x38
+    assert O.encode_e4m3(1.1875) == 0x3A
+    assert O.encode_e4m3(-1.0625) == 0xB8
+    # smallest subnormal 2^-9: half of it ties to zero, just above rounds up
+    assert O.encode_e4m3(2.0 ** -10) == 0x00 and O.encode_e4m3(2.0 ** -10 * 1.0001) == 0x01
+    # beyond 448 (0x7E) saturates; NaN keeps the NaN code
+    assert O.encode_e4m3(500.0) == 0x7E and O.encode_e4m3(-1e9) == 0xFE
+    assert O.encode_e4m3(float("nan")) == 0x7F
+
+
+def test_e4m3_encode_matches_the_library_conversion():
+    # an independent implementation: torch's float8_e4m3fn conversion, in range
+    g = np.random.default_rng(5)
+    x = (g.standard_normal(100000) * np.exp(g.uniform(-9, 6, 100000))).astype(np.float32)
+    x = x[np.abs(x) < 440]
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.encode_e4m3(x.astype(np.float64)), want)
+
+
+def test_quantize_kv_scale_is_one_fp32_product():
+    g = np.random.default_rng(6)
+    x = torch.from_numpy(g.standard_normal(5000).astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(O.quantize_kv_e4m3(x, 1.0), O.encode_e4m3(x))
+    assert np.array_equal(O.quantize_kv_e4m3(x, 4.0), O.encode_e4m3(x / 4.0))  # power of two: exact
+    # a general scale: the fp32 product, not the exact quotient, is encoded
+    s = 0.37
+    prod = (x.astype(np.float32) * (np.float32(1.0) / np.float32(s))).astype(np.float64)
+    assert np.array_equal(O.quantize_kv_e4m3(x, s), O.encode_e4m3(prod))
+
+
+def test_fp8_append_rebuilds_the_seeded_one_byte_cache():
+    # appending the new tokens' values (scale 1) to the one-byte pools of the
+    # cached prefix gives the whole batch's one-byte pools, as the generator
+    # draws them independently through the page table
+    from block_sparse_gqa_indexer_b200 import synth as S
+    w = S.Workload(ctx=[60, 130, 0], nq=[9, 2, 70], seed=21)
+    pt = w.page_table()
+    k0, v0 = w.kv_pools("cpu", pt, upto=w.ctx, fp8=True)
+    kn, vn, _ = w.new_tokens("cpu")
+    k1, v1 = O.append_to_paged_cache_fp8(k0.numpy(), v0.numpy(), pt.numpy(), w.ctx, w.nq,
+                                         kn.double().numpy(), vn.double().numpy(), 1.0, 1.0)
+    kw, vw = w.kv_pools("cpu", pt, fp8=True)
+    assert np.array_equal(k1, kw.numpy()) and np.array_equal(v1, vw.numpy())
