@@ -456,7 +456,12 @@ def run_config(args) -> None:
         swa = (args.config == 2) or (args.config == 5 and li < 3)
         pt = w.page_table()
         kv8 = args.fp8_kv and not swa  # one-byte KV: sparse (full-attention) layers only
-        k_pool, v_pool = w.kv_pools(dev, pt, window_only=S.WINDOW if swa else None, fp8=kv8)
+        if args.index_only and swa:
+            continue
+        if args.index_only:  # the indexer alone: no KV pools
+            k_pool = v_pool = None
+        else:
+            k_pool, v_pool = w.kv_pools(dev, pt, window_only=S.WINDOW if swa else None, fp8=kv8)
         batch = s5.Batch.from_host(pt, w.ctx, w.nq, dev)
         ws = s5.new_workspace(batch, window=S.WINDOW, device=dev)
         q, qx = w.queries(dev)
@@ -502,6 +507,13 @@ def run_config(args) -> None:
             calls.append(lambda kp=key_pool, b=batch, qx=qx, sel=sel, cnt=cnt, ws=ws, f=index_fn:
                          f(kp, b, qx, S.TOPK, sel, cnt, ws))
             kinds.append("index_fp8keys" if args.fp8_keys else "index")
+            sp = R.sparse_decode_bytes(w.ctx, w.nq)
+            if args.index_only:
+                # keys (at one or two bytes per value) + indexer queries + selections
+                bytes_total += (sp["keys"] // 2 if args.fp8_keys else sp["keys"]) + w.total_q * (
+                    R.index_key_bytes() + 4 * (R.TOPK + 1))
+                flops_total += R.sparse_flops(w.ctx, w.nq)["index"]
+                continue
             if kv8:
                 calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, sel=sel, cnt=cnt, o=out, l=lse, ws=ws:
                              s5.s5_sparse_gqa_attn_fp8kv(k, v, b, q, sel, cnt, S.TOPK, scale, 1.0, 1.0, o, l, ws))
@@ -510,7 +522,6 @@ def run_config(args) -> None:
                 calls.append(lambda k=k_pool, v=v_pool, b=batch, q=q, sel=sel, cnt=cnt, o=out, l=lse, ws=ws:
                              s5.s5_sparse_gqa_attn(k, v, b, q, sel, cnt, S.TOPK, scale, o, l, ws))
                 kinds.append("sparse")
-            sp = R.sparse_decode_bytes(w.ctx, w.nq)
             # one-byte keys: the indexer reads half the key bytes; one-byte KV: half the KV bytes
             bytes_total += sp["total"] - (sp["keys"] // 2 if args.fp8_keys else 0) - (sp["kv"] // 2 if kv8 else 0)
             flops_total += R.sparse_flops(w.ctx, w.nq)["total"]
@@ -570,7 +581,7 @@ def run_config(args) -> None:
             "useful_tflops": flops_total / (ms * 1e-3) / 1e12, "steps": args.steps, "warmup": args.warmup,
             "gbs_warm": bytes_total / (ms_warm * 1e-3) / 1e9,
             "append": bool(args.append), "grouped": bool(args.grouped), "fp8_keys": bool(args.fp8_keys),
-            "fp8_kv": bool(args.fp8_kv), "ctx_override": args.ctx}
+            "fp8_kv": bool(args.fp8_kv), "ctx_override": args.ctx, "index_only": bool(args.index_only)}
     print(json.dumps(line), flush=True)
 
 
@@ -591,6 +602,8 @@ def main():
                     help="with --config: sparse layers select per KV group (4 indexer queries per token)")
     ap.add_argument("--fp8-keys", action="store_true",
                     help="with --config: block keys stored as one-byte E4M3 codes")
+    ap.add_argument("--index-only", action="store_true",
+                    help="with --config: time the sparse layers' indexer call alone (no KV pools)")
     ap.add_argument("--ctx", type=int, default=None,
                     help="with --config: every sequence's cached tokens (default: the configuration's)")
     ap.add_argument("--fp8-kv", action="store_true",
@@ -602,6 +615,8 @@ def main():
         ap.error("--grouped selection runs on bf16 block keys only")
     if args.append and args.fp8_keys:
         ap.error("the cache append writes bf16 block keys")
+    if args.index_only and (args.grouped or args.append or args.fp8_kv):
+        ap.error("--index-only times the shared indexer call alone")
     if args.fp8_kv and (args.grouped or args.append):
         ap.error("--fp8-kv runs the shared-selection sparse layer on a resident cache")
     if args.impl == "reference":

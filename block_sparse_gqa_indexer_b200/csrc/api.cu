@@ -23,6 +23,7 @@ constexpr int kSeg = 8192;          // ... segments of rows longer than 16,384 b
 constexpr int kMaxSeg = 32;         // (kSeg * kMaxSeg >= S5_MAX_LEN / 8)
 constexpr int kMaxSplit = 8;        // partitions per (row, group) beyond what kMaxList forces
 constexpr int kScorePagesPerCta = 64;  // indexer CTA: 64 pages = 512 block keys = 256 KB
+constexpr int kScoreMinPagesPerCta = 4;  // ... and at least 4 pages (two per warp pair in flight)
 constexpr int kMaxGridYZ = 65535;      // CUDA limit on gridDim.y and gridDim.z
 
 static_assert((long long)kSeg * kMaxSeg >= S5_MAX_LEN / S5_BLOCK_SIZE, "segments must cover the longest row");
@@ -543,7 +544,18 @@ s5_status index_common(const s5_index_desc *index, const s5_batch_desc *batch, c
     if (launch_index_gemm(gm, tq, tk, batch->batch, batch->max_q * groups, cs) != cudaSuccess) return S5_ERR_CUDA;
   } else {
     const int pages = (w.stride + kBpp - 1) / kBpp;
-    const int grid_pages = (pages + kScorePagesPerCta - 1) / kScorePagesPerCta;
+    // 64 pages (256 KB of keys) per CTA, or fewer when that leaves the SMs
+    // idle: a small batch is spread over at least two CTAs per SM
+    const long long row_tiles = ((long long)batch->max_q * groups + 3) / 4;
+    const long long want = 2LL * (device_slots() / kCtasPerSm);
+    long long ppc = kScorePagesPerCta;
+    const long long ctas64 = (long long)((pages + kScorePagesPerCta - 1) / kScorePagesPerCta) * batch->batch * row_tiles;
+    if (ctas64 < want) {
+      ppc = ((long long)pages * batch->batch * row_tiles + want - 1) / want;
+      ppc = ppc < kScoreMinPagesPerCta ? kScoreMinPagesPerCta : (ppc > kScorePagesPerCta ? kScorePagesPerCta : ppc);
+    }
+    ia.pages_per_cta = (int)ppc;
+    const int grid_pages = (int)((pages + ppc - 1) / ppc);
     if (launch_index_score(ia, batch->max_q * groups, grid_pages, batch->batch, cs) != cudaSuccess)
       return S5_ERR_CUDA;
   }

@@ -460,16 +460,29 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     // by more than kLazyMax, so weights stay below 2^8 and after the first
     // blocks O is almost never rescaled
     float mx0 = -INFINITY, mx1 = -INFINITY;
+    if (full[0] && full[1]) {  // (warp-uniform) every token of both blocks is read: no masks
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < 2; ++h) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int pos = bk[h] * kBlk + (KV8 ? tok8(2 * tq + e) : 2 * tq + e);
-        const bool v = bk[h] >= 0 && pos >= lo_tok && pos <= t;
-        sa[h][e] = v ? sa[h][e] * sl2 : -INFINITY;
-        sa[h][2 + e] = v ? sa[h][2 + e] * sl2 : -INFINITY;
-        mx0 = fmaxf(mx0, sa[h][e]);
-        mx1 = fmaxf(mx1, sa[h][2 + e]);
+        for (int e = 0; e < 2; ++e) {
+          sa[h][e] *= sl2;
+          sa[h][2 + e] *= sl2;
+          mx0 = fmaxf(mx0, sa[h][e]);
+          mx1 = fmaxf(mx1, sa[h][2 + e]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int pos = bk[h] * kBlk + (KV8 ? tok8(2 * tq + e) : 2 * tq + e);
+          const bool v = bk[h] >= 0 && pos >= lo_tok && pos <= t;
+          sa[h][e] = v ? sa[h][e] * sl2 : -INFINITY;
+          sa[h][2 + e] = v ? sa[h][2 + e] * sl2 : -INFINITY;
+          mx0 = fmaxf(mx0, sa[h][e]);
+          mx1 = fmaxf(mx1, sa[h][2 + e]);
+        }
       }
     }
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));

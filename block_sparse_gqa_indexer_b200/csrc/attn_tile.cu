@@ -17,17 +17,17 @@
 //   gqa_tile_kernel     a persistent kernel, one CTA per SM, walking work items
 //                       (tile, KV group, partition of the tile's list).  The
 //                       8 rows x 16 heads of a group are the M = 128 rows of
-//                       the MMAs.  Warp 16 streams 8-block chunks of K and
-//                       warp 17 of V by TMA (one 3 KB copy per block,
+//                       the MMAs.  Warp 4 streams 8-block chunks of K and
+//                       warp 5 of V by TMA (one 3 KB copy per block,
 //                       plane-major, 128-byte swizzled) through 4-stage rings;
-//                       warp 18 issues S = Q K^T (N = 64 tokens, K = 192) into
-//                       two tensor-memory buffers and warp 19 O += P V, both
+//                       warp 6 issues S = Q K^T (N = 64 tokens, K = 192) into
+//                       two tensor-memory buffers and warp 7 O += P V, both
 //                       with their A operand (Q, P) in tensor memory (two
 //                       issuing threads, so S of a later chunk never waits
-//                       behind the PV of an earlier one); warps 0-15 load Q into
-//                       tensor memory, run the masked online softmax (four
-//                       warps per 32 rows, one per quarter of the chunk's
-//                       columns, row maxima exchanged through shared memory),
+//                       behind the PV of an earlier one); warps 0-3 (one
+//                       thread per tile row, all 64 columns of a chunk, so a
+//                       row's maximum and sum never leave its thread) load Q
+//                       into tensor memory, run the masked online softmax,
 //                       write P back to tensor memory as bf16 and finish each
 //                       item.
 //
@@ -49,12 +49,13 @@ constexpr int kTChunkBlocks = 8;           // blocks per chunk
 constexpr int kTN = kTChunkBlocks * kBlk;  // 64 tokens per chunk
 constexpr int kTStages = 4;                // depth of the K ring and of the V ring
 constexpr int kTKvBytes = kTChunkBlocks * kBlockBytes;  // K (or V) of one chunk
-constexpr int kTSoftWarps = 16;                // softmax / epilogue warps
+constexpr int kTSoftWarps = 8;                 // softmax / epilogue warps: two threads per tile row
 constexpr int kTSoftThreads = kTSoftWarps * 32;
 constexpr int kTSplit = kTSoftWarps / 4;        // warps per tensor-memory lane quarter
 constexpr int kTCols = kTN / kTSplit;           // S columns per softmax warp (16)
 constexpr int kTBlocksW = kTCols / kBlk;        // blocks per softmax warp and chunk (2)
-constexpr int kTOCols = kD / kTSplit;           // O columns (= Q dims) per softmax warp (48)
+constexpr int kTOCols = kD / kTSplit;           // O columns (= Q dims) per softmax warp
+static_assert(kTCols == 16 || kTCols % 32 == 0, "S columns per softmax thread: 16 or a multiple of 32");
 constexpr int kTWarpK = kTSoftWarps, kTWarpV = kTSoftWarps + 1, kTWarpS = kTSoftWarps + 2,
               kTWarpPv = kTSoftWarps + 3;
 constexpr int kTThreads = (kTSoftWarps + 4) * 32;
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
   };
 
   if (warp == kTWarpK || warp == kTWarpV) {
-    // ---------------- TMA producers: warp 16 K, warp 17 V ----------------
+    // ---------------- TMA producers: warp kTWarpK streams K, warp kTWarpV V ----------------
     // Lane b < 8 copies block b of each chunk (one 3 KB box: 3 planes x 8
     // tokens x 64 dims); lane 0 keeps the barrier bookkeeping.
     const bool is_k = warp == kTWarpK;
@@ -498,11 +499,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
       tc::commit(bars + kBFinal);
     }
   } else {
-    // ---------------- softmax / epilogue: warps 0-15 ----------------
+    // ---------------- softmax / epilogue: warps 0 .. kTSoftWarps-1 ----------------
     // Warp w reads lanes 32 (w % 4) .. + 31 (tile rows m = lane index: query
-    // j = m / 16, head h = m % 16) and columns 16 (w / 4) .. + 15 of each S
-    // (blocks 2 (w / 4), + 1 of the chunk); it owns Q dims and O columns
-    // 48 (w / 4) .. + 47 of its rows.
+    // j = m / 16, head h = m % 16) and columns kTCols (w / 4) .. + kTCols - 1
+    // of each S (blocks kTBlocksW (w / 4) ..); it owns Q dims and O columns
+    // kTOCols (w / 4) .. + kTOCols - 1 of its rows.  With four warps every
+    // thread owns a whole row: all 64 columns of S, all 192 of Q and O.
     const int q4 = warp & 3, qq = warp >> 2;
     const int m = q4 * 32 + lane;
     const int j = m >> 4, h = m & 15;
@@ -558,39 +560,73 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
         tc::fence_after_sync();
         uint32_t v[kTCols];
-        tc::ld_16cols(tmem + lane_base + kTmemS + sb * kTN + qq * kTCols, v);
+        if constexpr (kTCols % 32 == 0) {
+#pragma unroll
+          for (int x = 0; x < kTCols / 32; ++x)
+            tc::ld_32cols(tmem + lane_base + kTmemS + sb * kTN + qq * kTCols + 32 * x,
+                          *reinterpret_cast<uint32_t(*)[32]>(v + 32 * x));
+        } else {
+          tc::ld_16cols(tmem + lane_base + kTmemS + sb * kTN + qq * kTCols, *reinterpret_cast<uint32_t(*)[16]>(v));
+        }
         tc::wait_ld();
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + kBSEmpty + sb);
         // mask: column x = 8 ib + tok is token tok of block (2 qq + ib) of the chunk
         float sc[kTCols];  // scaled, masked scores
-        float mx = -INFINITY;
+        float mxb[kTBlocksW];  // per-block maxima (independent chains), then a tree
+        int lim[kTBlocksW];    // tokens 0 .. lim of block ib are visible to this row
+        bool partial = false;  // a block with only some tokens visible: the row's current block
 #pragma unroll
         for (int ib = 0; ib < kTBlocksW; ++ib) {
+          mxb[ib] = -INFINITY;
           const uint32_t e = __shfl_sync(0xffffffffu, e_cur, ib);
           const bool valid = row_ok && (c * kTChunkBlocks + qq * kTBlocksW + ib < it.ne);
           const int blk = (int)(e & 0xFFFFFFu);
           const bool sel = valid && ((e >> (24 + j)) & 1u);
-          const int lim = sel ? kBlk - 1 : ((valid && blk == cj) ? t - blk * kBlk : -1);  // tokens 0..lim visible
+          lim[ib] = sel ? kBlk - 1 : ((valid && blk == cj) ? t - blk * kBlk : -1);
+          partial |= (lim[ib] >= 0 && lim[ib] < kBlk - 1);
+        }
+        if (__any_sync(0xffffffffu, partial)) {  // (a row's last chunk) token-by-token masks
 #pragma unroll
-          for (int tok = 0; tok < kBlk; ++tok) {
-            const float s = (tok <= lim) ? __uint_as_float(v[ib * kBlk + tok]) * sl2 : -INFINITY;
-            sc[ib * kBlk + tok] = s;
-            mx = fmaxf(mx, s);
+          for (int ib = 0; ib < kTBlocksW; ++ib) {
+#pragma unroll
+            for (int tok = 0; tok < kBlk; ++tok) {
+              const float s = (tok <= lim[ib]) ? __uint_as_float(v[ib * kBlk + tok]) * sl2 : -INFINITY;
+              sc[ib * kBlk + tok] = s;
+              mxb[ib] = fmaxf(mxb[ib], s);
+            }
+          }
+        } else {  // every block is visible whole or not at all: one FMA with a 0 / -inf bias
+#pragma unroll
+          for (int ib = 0; ib < kTBlocksW; ++ib) {
+            const float bias = (lim[ib] >= 0) ? 0.f : -INFINITY;
+#pragma unroll
+            for (int tok = 0; tok < kBlk; ++tok) {
+              const float s = fmaf(__uint_as_float(v[ib * kBlk + tok]), sl2, bias);
+              sc[ib * kBlk + tok] = s;
+              mxb[ib] = fmaxf(mxb[ib], s);
+            }
           }
         }
-        // row max over the four column quarters
-        float *xmb = xm + sb * kTSplit * kTM;
-        xmb[qq * kTM + m] = mx;
-        mbar_arrive(bars + kBXm + q4 * 2 + sb);
-        if (!wait(bars + kBXm + q4 * 2 + sb, (gc >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        float rmax = mx;
 #pragma unroll
-        for (int o = 1; o < kTSplit; ++o) rmax = fmaxf(rmax, xmb[((qq + o) % kTSplit) * kTM + m]);
+        for (int w2 = kTBlocksW / 2; w2 > 0; w2 /= 2)
+#pragma unroll
+          for (int ib = 0; ib < w2; ++ib) mxb[ib] = fmaxf(mxb[ib], mxb[ib + w2]);
+        const float mx = mxb[0];
+        float rmax = mx;
+        if constexpr (kTSplit > 1) {
+          // row max over the column quarters of the row's kTSplit threads
+          float *xmb = xm + sb * kTSplit * kTM;
+          xmb[qq * kTM + m] = mx;
+          mbar_arrive(bars + kBXm + q4 * 2 + sb);
+          if (!wait(bars + kBXm + q4 * 2 + sb, (gc >> 1) & 1)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int o = 1; o < kTSplit; ++o) rmax = fmaxf(rmax, xmb[((qq + o) % kTSplit) * kTM + m]);
+        }
         // lazy rescale: keep the reference max unless the row max grows by more than 2^8
         const bool grow = rmax > m_ref + kLazyRescale;
         const bool resc = grow && m_ref != -INFINITY;
@@ -623,36 +659,53 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
         uint32_t pk[kTCols / 2];
-        float ps = 0.f;
+        float psb[kTBlocksW];  // per-block sums, then a tree
+#pragma unroll
+        for (int ib = 0; ib < kTBlocksW; ++ib) psb[ib] = 0.f;
 #pragma unroll
         for (int x = 0; x < kTCols / 2; ++x) {
           const float p0 = hw_exp2(sc[2 * x] - mu);
           const float p1 = hw_exp2(sc[2 * x + 1] - mu);
-          ps += p0 + p1;
+          psb[(2 * x) / kBlk] += p0 + p1;
           pk[x] = pack_bf16(p0, p1);
         }
-        l += ps;
-        tc::st_8cols(tmem + lane_base + kTmemP + sb * 32 + qq * (kTCols / 2), pk);
+#pragma unroll
+        for (int w2 = kTBlocksW / 2; w2 > 0; w2 /= 2)
+#pragma unroll
+          for (int ib = 0; ib < w2; ++ib) psb[ib] += psb[ib + w2];
+        l += psb[0];
+        if constexpr ((kTCols / 2) % 16 == 0) {
+#pragma unroll
+          for (int x = 0; x < kTCols / 32; ++x)
+            tc::st_16cols(tmem + lane_base + kTmemP + sb * 32 + qq * (kTCols / 2) + 16 * x,
+                          *reinterpret_cast<const uint32_t(*)[16]>(pk + 16 * x));
+        } else {
+          tc::st_8cols(tmem + lane_base + kTmemP + sb * 32 + qq * (kTCols / 2),
+                       *reinterpret_cast<const uint32_t(*)[8]>(pk));
+        }
         // V rows no row may read (padding slots, tokens past the tile's last
         // position, all in the item's last chunk) must be finite: zero them
-        // (P is 0 there, but 0 * NaN is NaN).  Warp w < 8 checks block w.
-        if (c == it.n_chunks - 1 && warp < kTChunkBlocks) {
-          const int ir = c * kTChunkBlocks + warp;
-          const int blk = (ir < it.ne) ? (int)(ld_cg(ent + ir) & 0xFFFFFFu) : -1;
-          const int first_bad = (blk < 0) ? 0 : t_max - blk * kBlk + 1;  // tokens >= first_bad are zeroed
-          if (first_bad < kBlk) {
-            if (!wait(bars + kBVFull + gc % kTStages, (gc / kTStages) & 1)) {
-              ok = false;
-              break;
+        // (P is 0 there, but 0 * NaN is NaN).  Warp w checks blocks w, w + 4, ...
+        if (c == it.n_chunks - 1) {
+          for (int wb = warp; wb < kTChunkBlocks && ok; wb += kTSoftWarps) {
+            const int ir = c * kTChunkBlocks + wb;
+            const int blk = (ir < it.ne) ? (int)(ld_cg(ent + ir) & 0xFFFFFFu) : -1;
+            const int first_bad = (blk < 0) ? 0 : t_max - blk * kBlk + 1;  // tokens >= first_bad are zeroed
+            if (first_bad < kBlk) {
+              if (!wait(bars + kBVFull + gc % kTStages, (gc / kTStages) & 1)) {
+                ok = false;
+                break;
+              }
+              uint8_t *vb = sv + (gc % kTStages) * kTKvBytes + wb * kBlockBytes;
+              for (int x = lane; x < 3 * kBlk * 8; x += 32) {  // plane, token, 16-byte chunk
+                const int tok = (x >> 3) & 7;
+                if (tok >= first_bad)
+                  *reinterpret_cast<uint4 *>(vb + (x >> 6) * 1024 + tok * 128 + (x & 7) * 16) = make_uint4(0, 0, 0, 0);
+              }
+              fence_proxy_async_smem();
             }
-            uint8_t *vb = sv + (gc % kTStages) * kTKvBytes + warp * kBlockBytes;
-            for (int x = lane; x < 3 * kBlk * 8; x += 32) {  // plane, token, 16-byte chunk
-              const int tok = (x >> 3) & 7;
-              if (tok >= first_bad)
-                *reinterpret_cast<uint4 *>(vb + (x >> 6) * 1024 + tok * 128 + (x & 7) * 16) = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
           }
+          if (!ok) break;
         }
         tc::wait_st();
         tc::fence_before_sync();
@@ -664,14 +717,18 @@ __global__ void __launch_bounds__(kTThreads, 1)
       float lt = 0.f;
       const bool have = it.n_chunks > 0;
       if (have) {
-        xl[qq * kTM + m] = l;
-        mbar_arrive(bars + kBXl + q4);
-        if (!wait(bars + kBXl + q4, qi & 1)) {
-          ok = false;
-          break;
-        }
+        if constexpr (kTSplit > 1) {
+          xl[qq * kTM + m] = l;
+          mbar_arrive(bars + kBXl + q4);
+          if (!wait(bars + kBXl + q4, qi & 1)) {
+            ok = false;
+            break;
+          }
 #pragma unroll
-        for (int o = 0; o < kTSplit; ++o) lt += xl[o * kTM + m];
+          for (int o = 0; o < kTSplit; ++o) lt += xl[o * kTM + m];
+        } else {
+          lt = l;
+        }
         if (!wait(bars + kBPFree + ((gc - 1) & 1), ((gc - 1) >> 1) & 1)) {
           ok = false;
           break;

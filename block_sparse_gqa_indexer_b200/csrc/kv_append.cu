@@ -13,8 +13,16 @@
 // row is contiguous.  The kernel is a pure copy (about 3.6 KB read and
 // written per token), so it is bound by latency at decode sizes and by HBM in
 // prefill.
+//
+// s5_append_kv_fp8 is the same kernel for a cache whose K / V are one-byte
+// E4M3 codes (StepFun open-weights blog, "Fitting it on a node": FP8 KV for
+// the full-attention layers): each thread's 8 bf16 values are multiplied in
+// fp32 by the reciprocal of the layer's scale and rounded to the nearest E4M3
+// value (ties to even, saturating at 448), and 8 code bytes are stored; block
+// keys stay bf16.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 
 #include "s5_common.cuh"
@@ -48,12 +56,35 @@ struct AppendArgs {
   const uint8_t *v_new;
   const uint8_t *key_new;
   int32_t *err;
+  float k_inv, v_inv;  // one-byte K / V: fp32 reciprocals of the scales
 };
+
+// Two fp32 values to their E4M3 codes (round to nearest even, saturating at
+// 448), first value in the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint32_t d;
+  asm("{\n\t.reg .b16 c;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 c, %2, %1;\n\t"
+      "cvt.u32.u16 %0, c;\n\t}"
+      : "=r"(d)
+      : "f"(lo), "f"(hi));
+  return d;
+}
+
+// Eight bf16 values (16 bytes) times `inv` in fp32, as eight E4M3 code bytes.
+__device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 v, float inv) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = f32x2_to_e4m3x2(__fmul_rn(bf16lo(w[i]), inv), __fmul_rn(bf16hi(w[i]), inv));
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
 
 // One pass of a CTA covers kAppendRows rows: first one thread per row finds
 // its sequence, position and physical page (dependent lookups, all rows at
 // once), then every thread issues its 16-byte loads for all rows before any
 // store, so each thread keeps kAppendRows independent loads in flight.
+template <bool KV8>
 __global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(const AppendArgs a) {
   __shared__ int s_page[kAppendRows];
   __shared__ int s_pos[kAppendRows];
@@ -100,9 +131,15 @@ __global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(const AppendA
       if (!on[i]) continue;
       const size_t page = (size_t)s_page[i];
       const int slot = s_pos[i] % kPage;
-      uint8_t *dst = is_key ? a.key_pool + ((page * kBpp + slot / kBlk) * kKeyChunks + c) * 16
-                            : (is_v ? a.v_pool : a.k_pool) + (((page * kKv + g) * kPage + slot) * kRowChunks + w) * 16;
-      *reinterpret_cast<uint4 *>(dst) = v[i];
+      if (is_key) {
+        *reinterpret_cast<uint4 *>(a.key_pool + ((page * kBpp + slot / kBlk) * kKeyChunks + c) * 16) = v[i];
+      } else if (KV8) {  // 8 code bytes per chunk of 8 values
+        *reinterpret_cast<uint2 *>((is_v ? a.v_pool : a.k_pool) + (((page * kKv + g) * kPage + slot) * kRowChunks + w) * 8) =
+            bf16x8_to_e4m3x8(v[i], is_v ? a.v_inv : a.k_inv);
+      } else {
+        *reinterpret_cast<uint4 *>((is_v ? a.v_pool : a.k_pool) + (((page * kKv + g) * kPage + slot) * kRowChunks + w) * 16) =
+            v[i];
+      }
     }
     __syncthreads();  // s_page / s_pos are rewritten by the next pass
   }
@@ -110,12 +147,15 @@ __global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(const AppendA
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-}  // namespace
-
-extern "C" s5_status s5_append_kv(const s5_kv_desc *kv, const s5_index_desc *index, const s5_batch_desc *batch,
-                                  const void *k_new, const void *v_new, const void *key_new, void *workspace,
-                                  size_t workspace_bytes, s5_stream_t stream) {
+// kv8: the K / V pools hold one-byte E4M3 codes (k_scale, v_scale used);
+// otherwise bf16.
+s5_status append_common(const s5_kv_desc *kv, const s5_index_desc *index, const s5_batch_desc *batch,
+                        const void *k_new, const void *v_new, const void *key_new, void *workspace,
+                        size_t workspace_bytes, s5_stream_t stream, bool kv8, float k_scale, float v_scale) {
   if (batch == nullptr || kv == nullptr) return S5_ERR_INVALID_ARG;
+  if (kv8 && (!(std::isfinite(k_scale) && std::isfinite(v_scale)) || k_scale == 0.f || v_scale == 0.f ||
+              !std::isfinite(1.f / k_scale) || !std::isfinite(1.f / v_scale)))
+    return S5_ERR_INVALID_ARG;
   if (batch->batch < 1 || batch->max_pages < 1 || batch->total_q < 0) return S5_ERR_INVALID_ARG;
   if (batch->page_table == nullptr || batch->ctx_lens == nullptr || batch->cu_q == nullptr)
     return S5_ERR_INVALID_ARG;
@@ -149,8 +189,28 @@ extern "C" s5_status s5_append_kv(const s5_kv_desc *kv, const s5_index_desc *ind
   a.v_new = static_cast<const uint8_t *>(v_new);
   a.key_new = index != nullptr ? static_cast<const uint8_t *>(key_new) : nullptr;
   a.err = static_cast<int32_t *>(workspace);
+  a.k_inv = kv8 ? 1.f / k_scale : 1.f;
+  a.v_inv = kv8 ? 1.f / v_scale : 1.f;
   const int passes = (batch->total_q + kAppendRows - 1) / kAppendRows;
   const int grid = passes < kAppendMaxCtas ? passes : kAppendMaxCtas;
-  kv_append_kernel<<<grid, kAppendThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  if (kv8)
+    kv_append_kernel<true><<<grid, kAppendThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  else
+    kv_append_kernel<false><<<grid, kAppendThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return cudaGetLastError() == cudaSuccess ? S5_OK : S5_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" s5_status s5_append_kv(const s5_kv_desc *kv, const s5_index_desc *index, const s5_batch_desc *batch,
+                                  const void *k_new, const void *v_new, const void *key_new, void *workspace,
+                                  size_t workspace_bytes, s5_stream_t stream) {
+  return append_common(kv, index, batch, k_new, v_new, key_new, workspace, workspace_bytes, stream, false, 1.f, 1.f);
+}
+
+extern "C" s5_status s5_append_kv_fp8(const s5_kv_desc *kv, const s5_index_desc *index, const s5_batch_desc *batch,
+                                      const void *k_new, const void *v_new, const void *key_new, float k_scale,
+                                      float v_scale, void *workspace, size_t workspace_bytes, s5_stream_t stream) {
+  return append_common(kv, index, batch, k_new, v_new, key_new, workspace, workspace_bytes, stream, true, k_scale,
+                       v_scale);
 }

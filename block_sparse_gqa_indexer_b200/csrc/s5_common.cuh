@@ -250,16 +250,22 @@ __device__ __forceinline__ uint32_t score_key(float s) {
 }
 
 // Four one-byte E4M3 codes (byte i of w is element i) to their exact values:
-// every E4M3 value is a half-precision value, and every half a float.
+// every E4M3 value is a half-precision value, and every half a float.  The
+// codes widen pairwise to f16 pairs (first element in the low half), then
+// each half to fp32.
 __device__ __forceinline__ void e4m3x4_to_float(uint32_t w, float &f0, float &f1, float &f2, float &f3) {
-  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
-  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
-  const float2 a = __half22float2(__half2(lo));
-  const float2 b = __half22float2(__half2(hi));
-  f0 = a.x;
-  f1 = a.y;
-  f2 = b.x;
-  f3 = b.y;
+  asm("{\n\t.reg .b16 a, b, h0, h1, h2, h3;\n\t.reg .b32 p, q;\n\t"
+      "mov.b32 {a, b}, %4;\n\t"
+      "cvt.rn.f16x2.e4m3x2 p, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 q, b;\n\t"
+      "mov.b32 {h0, h1}, p;\n\t"
+      "mov.b32 {h2, h3}, q;\n\t"
+      "cvt.f32.f16 %0, h0;\n\t"
+      "cvt.f32.f16 %1, h1;\n\t"
+      "cvt.f32.f16 %2, h2;\n\t"
+      "cvt.f32.f16 %3, h3;\n\t}"
+      : "=f"(f0), "=f"(f1), "=f"(f2), "=f"(f3)
+      : "r"(w));
 }
 
 // Hardware base-2 exponential / logarithm (PTX ex2.approx / lg2.approx).

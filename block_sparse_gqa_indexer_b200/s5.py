@@ -35,7 +35,7 @@ S5_WS_TEST_STALL_OFFSET = 64  # expired-wait test hook (include/s5attn.h); zero 
 SYMBOLS = ("s5_workspace_size", "s5_index_score_topk", "s5_sparse_gqa_attn", "s5_swa_gqa_attn",
            "s5_index_score_topk_fp8", "s5_sparse_gqa_attn_fp8kv",
            "s5_workspace_size_grouped", "s5_index_score_topk_grouped", "s5_sparse_gqa_attn_grouped",
-           "s5_index_score_topk_noalloc", "s5_append_kv", "s5_reset_device_error", "s5_get_device_error",
+           "s5_index_score_topk_noalloc", "s5_append_kv", "s5_append_kv_fp8", "s5_reset_device_error", "s5_get_device_error",
            "s5_status_string", "s5_abi_version")
 
 
@@ -74,6 +74,8 @@ _lib.s5_index_score_topk_noalloc.argtypes = [ctypes.POINTER(IndexDesc), ctypes.P
                                              _P, _P]
 _lib.s5_append_kv.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(IndexDesc), ctypes.POINTER(BatchDesc), _P, _P,
                               _P, _P, ctypes.c_size_t, _P]
+_lib.s5_append_kv_fp8.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(IndexDesc), ctypes.POINTER(BatchDesc), _P,
+                                  _P, _P, ctypes.c_float, ctypes.c_float, _P, ctypes.c_size_t, _P]
 _lib.s5_reset_device_error.argtypes = [_P, _P]
 _lib.s5_get_device_error.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
 _lib.s5_status_string.argtypes = [ctypes.c_int]
@@ -318,6 +320,29 @@ def s5_append_kv(k_pool, v_pool, key_pool, batch: Batch, k_new, v_new, key_new, 
     _check(_lib.s5_append_kv(ctypes.byref(kv), None if idx is None else ctypes.byref(idx), ctypes.byref(batch.desc),
                              _ptr(k_new), _ptr(v_new), None if idx is None else _ptr(key_new), _ptr(ws),
                              ws.numel(), _stream(stream)), "s5_append_kv")
+
+
+def s5_append_kv_fp8(k_pool, v_pool, key_pool, batch: Batch, k_new, v_new, key_new, k_scale: float, v_scale: float,
+                     ws, stream=None):
+    """s5_append_kv into one-byte (E4M3) K / V pools (uint8 [num_pages][4][64][192]):
+    each bf16 value x is stored as the code nearest to x / scale (an fp32
+    product with the reciprocal); block keys as in s5_append_kv."""
+    _need(k_pool, torch.uint8, "k_pool")
+    _need(v_pool, torch.uint8, "v_pool", tuple(k_pool.shape))
+    sh = k_pool.shape
+    kv = KvDesc(k_pool.data_ptr(), v_pool.data_ptr(), sh[0], sh[2], sh[1], sh[3])
+    _need(k_new, torch.bfloat16, "k_new", (batch.total_q, N_KV, HEAD_DIM))
+    _need(v_new, torch.bfloat16, "v_new", (batch.total_q, N_KV, HEAD_DIM))
+    idx = None
+    if key_pool is not None:
+        _need(key_pool, torch.bfloat16, "key_pool")
+        _need(key_new, torch.bfloat16, "key_new", (batch.total_q, INDEX_DIM))
+        idx = IndexDesc(key_pool.data_ptr(), key_pool.shape[0], key_pool.shape[-1])
+    _need(ws, torch.uint8, "ws")
+    _check(_lib.s5_append_kv_fp8(ctypes.byref(kv), None if idx is None else ctypes.byref(idx),
+                                 ctypes.byref(batch.desc), _ptr(k_new), _ptr(v_new),
+                                 None if idx is None else _ptr(key_new), float(k_scale), float(v_scale), _ptr(ws),
+                                 ws.numel(), _stream(stream)), "s5_append_kv_fp8")
 
 
 def s5_reset_device_error(ws: torch.Tensor, stream=None):

@@ -88,7 +88,7 @@ typedef enum {
 
 /* ABI version (major * 100 + minor): 1.01 added the cache append, the
  * per-KV-group entry points and the one-byte-key indexer; 1.02 the sparse
- * attention over one-byte KV. */
+ * attention over one-byte KV and its cache append. */
 #define S5_ABI_VERSION 102
 
 /* One attention layer's paged KV cache. */
@@ -296,6 +296,21 @@ s5_status s5_index_score_topk_noalloc(const s5_index_desc *index, const s5_batch
 s5_status s5_append_kv(const s5_kv_desc *kv, const s5_index_desc *index, const s5_batch_desc *batch,
                        const void *k_new, const void *v_new, const void *key_new, void *workspace,
                        size_t workspace_bytes, s5_stream_t stream);
+
+/* s5_append_kv for a cache whose K / V are one-byte E4M3 codes (the pools of
+ * s5_sparse_gqa_attn_fp8kv; StepFun open-weights blog, "Fitting it on a
+ * node": FP8 KV for the full-attention layers).  k_new / v_new are bf16 as in
+ * s5_append_kv; value x of a K row is stored as the E4M3 code nearest to the
+ * fp32 product x * (1 / k_scale) (1 / k_scale rounded to fp32; ties to an even
+ * mantissa; magnitudes beyond 448 saturate to +-448), V likewise with v_scale,
+ * so a stored code stands for about x / scale and s5_sparse_gqa_attn_fp8kv
+ * with the same scales reads it back as scale * code.  kv->k_pool / v_pool
+ * are uint8 [num_pages][4][64][192]; block keys (index, key_new) are bf16
+ * exactly as in s5_append_kv.  k_scale and v_scale must be finite and nonzero
+ * with finite reciprocals (S5_ERR_INVALID_ARG).  Otherwise as s5_append_kv. */
+s5_status s5_append_kv_fp8(const s5_kv_desc *kv, const s5_index_desc *index, const s5_batch_desc *batch,
+                           const void *k_new, const void *v_new, const void *key_new, float k_scale, float v_scale,
+                           void *workspace, size_t workspace_bytes, s5_stream_t stream);
 
 /* Zero the first S5_WS_FIXED_BYTES of a workspace: the device error record
  * and the partition counters (asynchronous, on `stream`). */

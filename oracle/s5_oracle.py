@@ -404,16 +404,16 @@ def quantize_kv_e4m3(x, scale: float) -> np.ndarray:
     return encode_e4m3(prod.astype(np.float64))
 
 
-def append_to_paged_cache_fp8(k_pool, v_pool, page_table, ctx, nq, k_new, v_new, k_scale: float, v_scale: float):
-    """The one-byte K / V pools after appending the new tokens of a varlen
-    batch: row r's values are stored as quantize_kv_e4m3(k_new[r], k_scale)
-    and quantize_kv_e4m3(v_new[r], v_scale), at the slots the bf16 append
-    uses (no block keys: the block-key pool is written by the bf16-key or
-    one-byte-key path of the indexer's own append)."""
+def append_to_paged_cache_fp8(k_pool, v_pool, key_pool, page_table, ctx, nq, k_new, v_new, key_new,
+                              k_scale: float, v_scale: float):
+    """The pools after appending the new tokens of a varlen batch to a cache
+    with one-byte K / V: row r's values are stored as
+    quantize_kv_e4m3(k_new[r], k_scale) and quantize_kv_e4m3(v_new[r], v_scale)
+    at the slots the bf16 append uses; block keys (bf16, key_pool may be None)
+    are stored exactly as by append_to_paged_cache."""
     k_codes = quantize_kv_e4m3(np.asarray(k_new, dtype=np.float64), k_scale)
     v_codes = quantize_kv_e4m3(np.asarray(v_new, dtype=np.float64), v_scale)
-    k_out, v_out, _ = append_to_paged_cache(k_pool, v_pool, None, page_table, ctx, nq, k_codes, v_codes, None)
-    return k_out, v_out
+    return append_to_paged_cache(k_pool, v_pool, key_pool, page_table, ctx, nq, k_codes, v_codes, key_new)
 
 
 def decode_e4m3(b) -> np.ndarray:

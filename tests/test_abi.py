@@ -240,3 +240,14 @@ def test_fp8_kv_entry_checks(s5):
     kv_geo = s5.KvDesc(0x1000, 0x1000, 8, 64, 4, 128)
     assert f(ctypes.byref(kv_geo), ctypes.byref(b), fake, fake, fake, 512, 0.1, 1.0, 1.0, fake, None, fake, 1 << 30,
              None) == s5.S5_ERR_UNSUPPORTED
+
+
+def test_fp8_append_rejects_bad_scales_before_launch(s5):
+    fake = ctypes.c_void_p(0x1000)
+    kv = s5.KvDesc(0x1000, 0x1000, 8, 64, 4, 192)
+    f = s5._lib.s5_append_kv_fp8
+    for ks, vs in [(0.0, 1.0), (1.0, float("nan")), (float("inf"), 1.0), (1e-45, 1.0)]:
+        assert f(ctypes.byref(kv), None, ctypes.byref(_batch()), fake, fake, None, ks, vs, fake, 1 << 20,
+                 None) == s5.S5_ERR_INVALID_ARG
+    assert f(ctypes.byref(kv), None, ctypes.byref(_batch()), fake, fake, None, 1.0, 1.0, fake, 16,
+             None) == s5.S5_ERR_WORKSPACE

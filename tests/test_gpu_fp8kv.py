@@ -143,3 +143,106 @@ def test_fp8kv_accuracy_against_bf16_kv(lib):
     rel_rms = float(np.sqrt((err ** 2).sum() / (want_bf16 ** 2).sum()))
     print(f"fp8 KV vs bf16 KV: max_abs={np.abs(err).max():.3e} rel_rms={rel_rms:.3e}")
     assert rel_rms < 0.10
+
+
+# ---------------------------------------------------------------- the one-byte cache append
+
+def _fp8_append_inputs(lib, w):
+    pt = w.page_table()
+    k0, v0 = w.kv_pools("cuda", pt, upto=w.ctx, fp8=True)
+    x0 = w.index_pool("cuda", pt, upto=w.ctx)
+    kn, vn, xn = w.new_tokens("cuda")
+    batch = lib.Batch.from_host(pt, w.ctx, w.nq, "cuda")
+    ws = lib.new_workspace(batch)
+    return pt, k0, v0, x0, kn, vn, xn, batch, ws
+
+
+@pytest.mark.parametrize("ctx,nq", [
+    ([60, 5000, 0, 130], [9, 3, 70, 1]),   # page and block edges on both sides, a fresh sequence
+    ([131072, 7, 4095], [1, 4, 2]),        # decode / verify rows
+    ([2000], [300]),                       # a prefill chunk
+])
+def test_fp8_append_matches_the_oracle_and_the_generator(lib, ctx, nq):
+    w = S.Workload(ctx=ctx, nq=nq, seed=65)
+    pt, k0, v0, x0, kn, vn, xn, batch, ws = _fp8_append_inputs(lib, w)
+    # unit scales: the codes the generator draws for the whole batch
+    k1, v1, x1 = k0.clone(), v0.clone(), x0.clone()
+    lib.s5_append_kv_fp8(k1, v1, x1, batch, kn, vn, xn, 1.0, 1.0, ws)
+    torch.cuda.synchronize()
+    code, info = lib.s5_get_device_error(ws)
+    assert code == 0, (lib.s5_status_string(code), info)
+    kw, vw = w.kv_pools("cuda", pt, fp8=True)
+    assert torch.equal(k1, kw) and torch.equal(v1, vw)
+    assert torch.equal(x1, w.index_pool("cuda", pt))
+    # other scales: the oracle's codes of x * fl32(1 / scale), bit for bit
+    if w.num_pages <= 4096:
+        k2, v2, x2 = k0.clone(), v0.clone(), x0.clone()
+        lib.s5_append_kv_fp8(k2, v2, x2, batch, kn, vn, xn, 0.37, 1.9, ws)
+        torch.cuda.synchronize()
+        ko, vo, xo = O.append_to_paged_cache_fp8(k0.cpu().numpy(), v0.cpu().numpy(), x0.double().cpu().numpy(),
+                                                 pt.numpy(), w.ctx, w.nq, kn.double().cpu().numpy(),
+                                                 vn.double().cpu().numpy(), xn.double().cpu().numpy(), 0.37, 1.9)
+        assert np.array_equal(k2.cpu().numpy(), ko) and np.array_equal(v2.cpu().numpy(), vo)
+        assert np.array_equal(x2.double().cpu().numpy(), xo)
+
+
+def test_fp8_append_reports_an_unmapped_page(lib):
+    w = S.Workload(ctx=[100, 700], nq=[2, 1], seed=66)
+    pt, k0, v0, x0, kn, vn, xn, batch, ws = _fp8_append_inputs(lib, w)
+    batch.page_table[1, 700 // 64] = -1
+    lib.s5_reset_device_error(ws)
+    lib.s5_append_kv_fp8(k0, v0, None, batch, kn, vn, None, 1.0, 1.0, ws)
+    code, info = lib.s5_get_device_error(ws)
+    assert code == lib.S5_ERR_DEVICE_BOUNDS and info == 2
+
+
+def test_fp8_append_then_attend_matches_the_oracle(lib):
+    # one decode / verify step on a one-byte cache: append (scales 0.5, 2),
+    # score and select, attend with the same scales
+    w = S.Workload(ctx=[9000, 20000, 300], nq=[1, 4, 2], seed=67)
+    pt, k0, v0, x0, kn, vn, xn, batch, ws = _fp8_append_inputs(lib, w)
+    ks, vs = 0.5, 2.0
+    lib.s5_append_kv_fp8(k0, v0, x0, batch, kn, vn, xn, ks, vs, ws)
+    _, qx = w.queries("cuda")
+    q = w.q_rows(torch.arange(w.total_q), "cuda")
+    sel = torch.empty((w.total_q, S.TOPK), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((w.total_q,), dtype=torch.int32, device="cuda")
+    out = torch.empty((w.total_q, 64, 192), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.total_q, 64), dtype=torch.float32, device="cuda")
+    lib.s5_index_score_topk(x0, batch, qx, S.TOPK, sel, cnt, ws)
+    lib.s5_sparse_gqa_attn_fp8kv(k0, v0, batch, q, sel, cnt, S.TOPK, O.DEFAULT_SM_SCALE, ks, vs, out, lse, ws)
+    torch.cuda.synchronize()
+    code, info = lib.s5_get_device_error(ws)
+    assert code == 0, (lib.s5_status_string(code), info)
+    rows = list(range(w.total_q))
+    want_sel = oracle_selection(w, rows)
+    assert np.array_equal(sel.cpu().numpy(), want_sel)
+    # the oracle reads the codes its own append stores: cached tokens carry the
+    # generator's unit-scale codes, new tokens the scaled ones
+    seqs, pos = w.query_seq_pos()
+    new_at = {(seqs[r], pos[r]): r for r in rows}
+    kn_np, vn_np = kn.double().cpu().numpy(), vn.double().cpu().numpy()
+
+    class Codes:
+        def __init__(self, s, which):
+            self.s, self.which = s, which
+
+        def __getitem__(self, ps):
+            ps = np.asarray(ps, dtype=np.int64)
+            f = w.k_tokens if self.which == "k" else w.v_tokens
+            out_c = S.to_e4m3_codes(f(self.s, torch.as_tensor(ps))).numpy()
+            for i, p in enumerate(ps.tolist()):
+                if (self.s, p) in new_at:
+                    x = (kn_np if self.which == "k" else vn_np)[new_at[(self.s, p)]]
+                    out_c[i] = O.quantize_kv_e4m3(x, ks if self.which == "k" else vs)
+            return out_c
+
+    q_np = q.double().cpu().numpy()
+    want, want_l = [], []
+    for r in rows:
+        s = seqs[r]
+        o, l = O.sparse_attention_query_fp8kv(q_np[r], want_sel[r], pos[r], Codes(s, "k"), Codes(s, "v"), ks, vs)
+        want.append(O.round_bf16(o))
+        want_l.append(l)
+    assert_attn_close(out.float().cpu().numpy(), np.array(want), "append then attend, one-byte KV")
+    assert np.abs(lse.cpu().numpy() - np.array(want_l)).max() <= LSE_ABS

@@ -745,8 +745,10 @@ def test_fp8_append_rebuilds_the_seeded_one_byte_cache():
     w = S.Workload(ctx=[60, 130, 0], nq=[9, 2, 70], seed=21)
     pt = w.page_table()
     k0, v0 = w.kv_pools("cpu", pt, upto=w.ctx, fp8=True)
-    kn, vn, _ = w.new_tokens("cpu")
-    k1, v1 = O.append_to_paged_cache_fp8(k0.numpy(), v0.numpy(), pt.numpy(), w.ctx, w.nq,
-                                         kn.double().numpy(), vn.double().numpy(), 1.0, 1.0)
+    x0 = w.index_pool("cpu", pt, upto=w.ctx)
+    kn, vn, xn = w.new_tokens("cpu")
+    k1, v1, x1 = O.append_to_paged_cache_fp8(k0.numpy(), v0.numpy(), x0.double().numpy(), pt.numpy(), w.ctx, w.nq,
+                                             kn.double().numpy(), vn.double().numpy(), xn.double().numpy(), 1.0, 1.0)
     kw, vw = w.kv_pools("cpu", pt, fp8=True)
     assert np.array_equal(k1, kw.numpy()) and np.array_equal(v1, vw.numpy())
+    assert np.array_equal(x1, w.index_pool("cpu", pt).double().numpy())
