@@ -17,16 +17,17 @@
 //   gqa_tile_kernel     a persistent kernel, one CTA per SM, walking work items
 //                       (tile, KV group, partition of the tile's list).  The
 //                       8 rows x 16 heads of a group are the M = 128 rows of
-//                       the MMAs.  Warp 4 streams 8-block chunks of K and
-//                       warp 5 of V by TMA (one 3 KB copy per block,
+//                       the MMAs.  Warp 8 streams 8-block chunks of K and
+//                       warp 9 of V by TMA (one 3 KB copy per block,
 //                       plane-major, 128-byte swizzled) through 4-stage rings;
-//                       warp 6 issues S = Q K^T (N = 64 tokens, K = 192) into
-//                       two tensor-memory buffers and warp 7 O += P V, both
+//                       warp 10 issues S = Q K^T (N = 64 tokens, K = 192) into
+//                       two tensor-memory buffers and warp 11 O += P V, both
 //                       with their A operand (Q, P) in tensor memory (two
 //                       issuing threads, so S of a later chunk never waits
-//                       behind the PV of an earlier one); warps 0-3 (one
-//                       thread per tile row, all 64 columns of a chunk, so a
-//                       row's maximum and sum never leave its thread) load Q
+//                       behind the PV of an earlier one); warps 0-7 (two per
+//                       tensor-memory lane quarter, one thread per tile row
+//                       each, 32 of a chunk's 64 columns each, row maxima of
+//                       the two halves exchanged through shared memory) load Q
 //                       into tensor memory, run the masked online softmax,
 //                       write P back to tensor memory as bf16 and finish each
 //                       item.
