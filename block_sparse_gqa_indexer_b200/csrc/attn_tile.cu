@@ -44,6 +44,28 @@
 
 namespace s5 {
 
+// Packed fp32 pairs (one instruction for two lanes of work on sm_100):
+// element-wise a * b + c and a + b, each rounded to nearest as fmaf / __fadd_rn.
+__device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)),
+        "l"(*reinterpret_cast<uint64_t *>(&c)));
+  return *reinterpret_cast<float2 *>(&d);
+}
+// max(a, b, c) in one instruction (sm_100 three-input max)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&d);
+}
+
 constexpr int kTRows = kTileRows;          // query rows per tile
 constexpr int kTM = kTRows * kHpg;         // 128 MMA rows = tensor-memory lanes
 constexpr int kTChunkBlocks = 8;           // blocks per chunk
@@ -573,8 +595,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + kBSEmpty + sb);
-        // mask: column x = 8 ib + tok is token tok of block (2 qq + ib) of the chunk
-        float sc[kTCols];  // scaled, masked scores
+        // mask: column x = 8 ib + tok is token tok of block (2 qq + ib) of the chunk.
+        // Scores are taken relative to the row's current reference max, so the
+        // weights need no subtraction unless the reference moves (rare).
+        const float mu0 = (m_ref == -INFINITY) ? 0.f : m_ref;
+        float sc[kTCols];  // scaled, masked scores minus mu0
         float mxb[kTBlocksW];  // per-block maxima (independent chains), then a tree
         int lim[kTBlocksW];    // tokens 0 .. lim of block ib are visible to this row
         bool partial = false;  // a block with only some tokens visible: the row's current block
@@ -593,20 +618,24 @@ __global__ void __launch_bounds__(kTThreads, 1)
           for (int ib = 0; ib < kTBlocksW; ++ib) {
 #pragma unroll
             for (int tok = 0; tok < kBlk; ++tok) {
-              const float s = (tok <= lim[ib]) ? __uint_as_float(v[ib * kBlk + tok]) * sl2 : -INFINITY;
+              const float s = (tok <= lim[ib]) ? fmaf(__uint_as_float(v[ib * kBlk + tok]), sl2, -mu0) : -INFINITY;
               sc[ib * kBlk + tok] = s;
               mxb[ib] = fmaxf(mxb[ib], s);
             }
           }
-        } else {  // every block is visible whole or not at all: one FMA with a 0 / -inf bias
+        } else {  // every block is visible whole or not at all: one FMA with a -mu0 / -inf bias
+          const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
           for (int ib = 0; ib < kTBlocksW; ++ib) {
-            const float bias = (lim[ib] >= 0) ? 0.f : -INFINITY;
+            const float bias = (lim[ib] >= 0) ? -mu0 : -INFINITY;
+            const float2 bias2 = make_float2(bias, bias);
 #pragma unroll
-            for (int tok = 0; tok < kBlk; ++tok) {
-              const float s = fmaf(__uint_as_float(v[ib * kBlk + tok]), sl2, bias);
-              sc[ib * kBlk + tok] = s;
-              mxb[ib] = fmaxf(mxb[ib], s);
+            for (int tok = 0; tok < kBlk; tok += 2) {  // two columns per packed FMA
+              const float2 s2 = fma_f32x2(
+                  make_float2(__uint_as_float(v[ib * kBlk + tok]), __uint_as_float(v[ib * kBlk + tok + 1])), sl2x2, bias2);
+              sc[ib * kBlk + tok] = s2.x;
+              sc[ib * kBlk + tok + 1] = s2.y;
+              mxb[ib] = fmax3(mxb[ib], s2.x, s2.y);
             }
           }
         }
@@ -628,11 +657,13 @@ __global__ void __launch_bounds__(kTThreads, 1)
 #pragma unroll
           for (int o = 1; o < kTSplit; ++o) rmax = fmaxf(rmax, xmb[((qq + o) % kTSplit) * kTM + m]);
         }
-        // lazy rescale: keep the reference max unless the row max grows by more than 2^8
-        const bool grow = rmax > m_ref + kLazyRescale;
+        // lazy rescale: keep the reference max unless the row max grows by more than
+        // 2^8 (rmax is relative to mu0; a row without a reference takes its first max)
+        const bool grow = (m_ref == -INFINITY) ? (rmax > -INFINITY) : (rmax > kLazyRescale);
         const bool resc = grow && m_ref != -INFINITY;
-        const float corr = resc ? hw_exp2(m_ref - rmax) : 1.f;
-        if (grow) m_ref = rmax;
+        const float corr = resc ? hw_exp2(-rmax) : 1.f;  // exp2(old reference - new)
+        const float shift = grow ? rmax : 0.f;           // new reference - mu0
+        if (grow) m_ref = mu0 + rmax;
         if (__any_sync(0xffffffffu, resc) && c > 0) {
           // O holds chunks up to gc - 1: wait for that PV (in-order completion covers the rest)
           if (!wait(bars + kBPFree + ((gc - 1) & 1), ((gc - 1) >> 1) & 1)) {
@@ -658,23 +689,30 @@ __global__ void __launch_bounds__(kTThreads, 1)
           ok = false;
           break;
         }
-        const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-        uint32_t pk[kTCols / 2];
-        float psb[kTBlocksW];  // per-block sums, then a tree
+        if (__any_sync(0xffffffffu, grow)) {  // (rare) scores relative to the moved reference
+          const float2 ns2 = make_float2(-shift, -shift);
 #pragma unroll
-        for (int ib = 0; ib < kTBlocksW; ++ib) psb[ib] = 0.f;
+          for (int x = 0; x < kTCols / 2; ++x) {
+            const float2 d2 = add_f32x2(make_float2(sc[2 * x], sc[2 * x + 1]), ns2);
+            sc[2 * x] = d2.x;
+            sc[2 * x + 1] = d2.y;
+          }
+        }
+        uint32_t pk[kTCols / 2];
+        float2 psb[kTBlocksW];  // per-block sums of column pairs, then a tree
+#pragma unroll
+        for (int ib = 0; ib < kTBlocksW; ++ib) psb[ib] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int x = 0; x < kTCols / 2; ++x) {
-          const float p0 = hw_exp2(sc[2 * x] - mu);
-          const float p1 = hw_exp2(sc[2 * x + 1] - mu);
-          psb[(2 * x) / kBlk] += p0 + p1;
-          pk[x] = pack_bf16(p0, p1);
+          const float2 p2 = make_float2(hw_exp2(sc[2 * x]), hw_exp2(sc[2 * x + 1]));
+          psb[(2 * x) / kBlk] = add_f32x2(psb[(2 * x) / kBlk], p2);
+          pk[x] = pack_bf16(p2.x, p2.y);
         }
 #pragma unroll
         for (int w2 = kTBlocksW / 2; w2 > 0; w2 /= 2)
 #pragma unroll
-          for (int ib = 0; ib < w2; ++ib) psb[ib] += psb[ib + w2];
-        l += psb[0];
+          for (int ib = 0; ib < w2; ++ib) psb[ib] = add_f32x2(psb[ib], psb[ib + w2]);
+        l += psb[0].x + psb[0].y;
         if constexpr ((kTCols / 2) % 16 == 0) {
 #pragma unroll
           for (int x = 0; x < kTCols / 32; ++x)
