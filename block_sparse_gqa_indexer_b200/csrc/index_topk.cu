@@ -180,6 +180,127 @@ __global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
   }
 }
 
+// Per-KV-group rows (4 indexer queries per token) on the tensor cores: the
+// FMA chain above scores every key against 4 queries, 4x the shared path's
+// work, so the same HBM stream leaves it bound by instruction issue.  Here a
+// warp scores two pages at a time as one bf16 mma.sync m16n8k16 tile: the 16
+// keys (8 of page p, 8 of page p + 1) are the A rows, 8 * NT query rows of
+// the sequence the B columns, 16 k-steps over the 256 dims.  Inside each
+// k-step the dims are permuted identically for keys and queries (lane quad
+// position q holds dims 8q .. 8q + 7 of each 32-dim group), so every
+// fragment is one 16-byte load.  Products and sums of the integer-valued
+// inputs are exact in the fp32 accumulators, so the scores equal the FMA
+// path's.
+template <int NT>
+__global__ void __launch_bounds__(256) index_score_mma_kernel(IndexScoreArgs a) {
+  constexpr int ROWS = 8 * NT;
+  pdl_trigger();  // the select may launch now; it waits for these scores before reading them
+  const int s = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g8 = lane >> 2, qd = lane & 3;
+  const int q_beg = __ldg(a.cu_q + s);
+  const int nq_s = __ldg(a.cu_q + s + 1) - q_beg;
+  const int G = a.q_groups;
+  const int tile0 = blockIdx.z * ROWS;
+  if (nq_s < 0 || q_beg < 0 || q_beg + nq_s > a.total_q) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, s);
+    return;
+  }
+  if (tile0 >= nq_s * G) return;
+  const int nq = min(ROWS, nq_s * G - tile0);
+  const int ctx = __ldg(a.ctx_lens + s);
+  const int t_last = ctx + (tile0 + nq - 1) / G;
+  const int c_hi = t_last / kBlk;  // history blocks of the tile's last row
+  if (ctx < 0 || t_last >= a.max_pages * kPage || c_hi > a.score_stride) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, q_beg + tile0 / G);
+    return;
+  }
+  if (c_hi <= a.topk) return;  // every row of the tile keeps all its history blocks
+  const int p_beg = blockIdx.x * a.pages_per_cta;
+  const int p_end = min(p_beg + a.pages_per_cta, (c_hi + kBpp - 1) / kBpp);
+  if (p_beg >= p_end) return;
+
+  // B fragments: query row tile0 + 8 nt + g8, dims 32 sg + 8 qd .. + 7 (zeros past the tile)
+  const uint4 *qx = reinterpret_cast<const uint4 *>(a.q_index) + (size_t)(q_beg * G + tile0) * (kDx / 8);
+  uint4 qv[NT][kDx / 32];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int row = 8 * nt + g8;
+#pragma unroll
+    for (int sg = 0; sg < kDx / 32; ++sg)
+      qv[nt][sg] = (row < nq) ? __ldg(qx + (size_t)row * (kDx / 8) + 4 * sg + qd) : make_uint4(0, 0, 0, 0);
+  }
+  const uint4 *keys = reinterpret_cast<const uint4 *>(a.key_pool);
+  const int32_t *pt = a.page_table + (size_t)s * a.max_pages;
+  const int nwarps = blockDim.x >> 5;
+  for (int p = p_beg + 2 * warp; p < p_end; p += 2 * nwarps) {
+    int ph[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      ph[u] = -1;
+      if (p + u < p_end) {
+        const int x = __ldg(pt + p + u);
+        if (x >= 0 && x < a.num_pages) ph[u] = x;
+        else if (lane == 0) record_error(a.err, S5_ERR_DEVICE_BOUNDS, q_beg + tile0 / G);
+      }
+    }
+    const int b0 = (p * kBpp) + g8, b1 = b0 + kBpp;  // A rows g8 (page p) and g8 + 8 (page p + 1)
+    const bool ok0 = ph[0] >= 0 && b0 < c_hi, ok1 = ph[1] >= 0 && b1 < c_hi;
+    uint4 xk[kDx / 32], yk[kDx / 32];
+#pragma unroll
+    for (int sg = 0; sg < kDx / 32; ++sg) {
+      xk[sg] = make_uint4(0, 0, 0, 0);
+      yk[sg] = make_uint4(0, 0, 0, 0);
+      if (ok0) {
+        const uint4 *src = keys + ((size_t)ph[0] * kBpp + g8) * (kDx / 8) + 4 * sg + qd;
+        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(xk[sg].x), "=r"(xk[sg].y), "=r"(xk[sg].z), "=r"(xk[sg].w)
+                     : "l"(src));
+      }
+      if (ok1) {
+        const uint4 *src = keys + ((size_t)ph[1] * kBpp + g8) * (kDx / 8) + 4 * sg + qd;
+        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(yk[sg].x), "=r"(yk[sg].y), "=r"(yk[sg].z), "=r"(yk[sg].w)
+                     : "l"(src));
+      }
+    }
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+    for (int sg = 0; sg < kDx / 32; ++sg) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // k-step 2 sg + h: dims 32 sg + 8 qd + 4 h + {0,1} and {2,3}
+        const uint32_t af[4] = {h ? xk[sg].z : xk[sg].x, h ? yk[sg].z : yk[sg].x, h ? xk[sg].w : xk[sg].y,
+                                h ? yk[sg].w : yk[sg].y};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma_bf16_16816(acc[nt], af, h ? qv[nt][sg].z : qv[nt][sg].x, h ? qv[nt][sg].w : qv[nt][sg].y);
+      }
+    }
+    // acc[nt][e] = score of block b0, row 8 nt + 2 qd + e; acc[nt][2 + e]: block b1
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int row = 8 * nt + 2 * qd + e;
+        if (row >= nq) continue;
+        const int lim = (ctx + (tile0 + row) / G) / kBlk;  // history blocks of the row's token
+        const size_t grow = (size_t)(q_beg * G + tile0 + row);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int b = u ? b1 : b0;
+          if (p + u < p_end && b < lim) {
+            const float sc = (ph[u] >= 0) ? acc[nt][2 * u + e] : __int_as_float(0xff800000);  // -inf: unreadable page
+            a.scores[grow * a.score_stride + b] = sc;
+            if (a.hist != nullptr) atomicAdd(a.hist + grow * kHistBins + (score_key(sc) >> 20), 1u);
+          }
+        }
+      }
+    }
+  }
+}
+
 // ============================================================================
 // CTA-wide radix select: the k largest keys of a list, ties to the earlier
 // list position, emitted in list order.
@@ -623,8 +744,13 @@ cudaError_t launch_index_score(const IndexScoreArgs &a, int max_q, int grid_page
   dim3 grid(grid_pages, n_seq, (max_q + qt - 1) / qt);
   if (a.q_groups > 1) {
     if (qt != 4) return cudaErrorInvalidValue;  // >= 4 rows per token
-    if (a.key_fp8) index_score_kernel<4, 2, true, true><<<grid, 256, 0, st>>>(a);
-    else index_score_kernel<4, 1, true, false><<<grid, 256, 0, st>>>(a);
+    if (a.key_fp8) {
+      index_score_kernel<4, 2, true, true><<<grid, 256, 0, st>>>(a);
+    } else if (max_q <= 8) {  // one token's 4 queries (8 MMA columns)
+      index_score_mma_kernel<1><<<dim3(grid_pages, n_seq, (max_q + 7) / 8), 256, 0, st>>>(a);
+    } else {  // 16 query rows per tile: the keys of a 4-token verify group are read once
+      index_score_mma_kernel<2><<<dim3(grid_pages, n_seq, (max_q + 15) / 16), 256, 0, st>>>(a);
+    }
   } else if (a.key_fp8) {
     // one-byte keys: half the bytes per page, so twice the pages in flight
     if (qt == 1) index_score_kernel<1, 4, false, true><<<grid, 256, 0, st>>>(a);
