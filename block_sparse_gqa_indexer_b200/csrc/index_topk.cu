@@ -479,17 +479,15 @@ __device__ __forceinline__ void write_all(int32_t *out, int n, int topk, int nt)
   for (int i = threadIdx.x; i < topk; i += nt) out[i] = (i < n) ? i : -1;
 }
 
-constexpr int kWarpRefine = 2048;  // threshold bins up to this size are refined by one warp
+constexpr int kCandMax = 2048;  // threshold bins up to this size are refined over their gathered keys
 
 struct HistSmem {
   uint32_t h1[kHistBins];       // row histogram of the top 12 key bits, when not given
   uint32_t h2[1024];            // block-wide refinement of a large threshold bin
-  uint32_t cand[kWarpRefine];   // keys of the threshold bin (any order)
+  uint32_t cand[kCandMax];      // keys of the threshold bin (any order)
   int scan_a[32];
   int ncand;
   uint32_t digit, above, bin_cnt;
-  uint32_t t_val;
-  int t_kk;
 };
 
 // Bin of the kk-th largest key when thread t owns the NB consecutive bins
@@ -523,14 +521,14 @@ __device__ __forceinline__ void find_bin_desc(const uint32_t (&c)[NB], int top, 
 
 // Single stage from a row histogram of the top 12 key bits (built while the
 // scores were produced, or here in shared memory from the keys when a.hist is
-// null).  The histogram gives the threshold bin; its keys are
-// then resolved either by one warp (a bit-by-bit search over the remaining 20
-// bits, when the bin holds at most kWarpRefine keys and WARP_REFINE is set) or
-// by two more block-wide radix passes of 10 bits.  MINB CTAs per SM: 1 keeps
+// null).  The histogram gives the threshold bin; its keys are then resolved
+// by two block-wide radix passes of 10 bits over the bin's keys, gathered into
+// shared memory (over all keys when the bin holds more than kCandMax), and the
+// selection is written in list order through one bit per owned key.  MINB CTAs per SM: 1 keeps
 // every key in registers (short launches: one CTA per row of a decode batch),
 // 2 caps registers at 32 per thread so that batches of many rows (prefill)
 // run twice as many rows at a time.
-template <int NT, int EMAX, bool WARP_REFINE, int MINB, bool GROUPED>
+template <int NT, int EMAX, int MINB, bool GROUPED>
 __global__ void __launch_bounds__(NT, MINB) topk_select_hist_kernel(SelectArgs a) {
   static_assert(NT == 512 || NT == 1024, "row-histogram and refinement bins are split evenly over threads");
   constexpr int NB1 = kHistBins / NT;  // row-histogram bins per thread
@@ -593,66 +591,74 @@ __global__ void __launch_bounds__(NT, MINB) topk_select_hist_kernel(SelectArgs a
   const int nb = (int)sm.bin_cnt;
   uint32_t t_lo = b1 << 20, t_hi = t_lo | 0xFFFFFu;
   if (nb != kk) {
-    if (WARP_REFINE && nb <= kWarpRefine) {
-      // gather the bin's keys, then one warp finds the kk-th largest among them
+    // the threshold bin's keys are resolved by two more radix passes of 10
+    // bits: over the bin's keys gathered into shared memory when they fit
+    // (any order: the counts are the same), else over every key again
+    bool gathered = nb <= kCandMax;
+    if (gathered) {
 #pragma unroll
       for (int j = 0; j < EMAX; ++j)
         if (j < mine && (key[j] >> 20) == b1) {
           const int slot = atomicAdd(&sm.ncand, 1);
-          if (slot < kWarpRefine) sm.cand[slot] = key[j];
+          if (slot < kCandMax) sm.cand[slot] = key[j];
         }
       __syncthreads();
-      if (warp == 0) {
-        const int ncand = min(sm.ncand, kWarpRefine);
-        uint32_t T = b1 << 20;
-        int ab = 0;
-        for (int b = 19; b >= 0; --b) {
-          const uint32_t cand = T | (1u << b);
-          int ge = 0;
-          for (int i = lane; i < ncand; i += 32) {
-            const uint32_t x = sm.cand[i];
-            ge += ((x >> (b + 1)) == (T >> (b + 1))) & (x >= cand);
-          }
-          ge = __reduce_add_sync(0xffffffffu, ge);
-          if (ab + ge >= kk) T = cand;
-          else ab += ge;
-        }
-        if (lane == 0) {
-          sm.t_val = T;
-          sm.t_kk = kk - ab;
-        }
-      }
-      __syncthreads();
-      t_lo = t_hi = sm.t_val;
-      kk = sm.t_kk;
-    } else {
-      uint32_t prefix = b1 << 20, mask = 0xFFF00000u;
-      bool stop = false;
-      __syncthreads();
-      for (int shift = 10; shift >= 0 && !stop; shift -= 10) {
+      gathered = sm.ncand <= kCandMax;  // (always, with a histogram of these keys)
+    }
+    const int ncand = gathered ? sm.ncand : 0;
+    uint32_t prefix = b1 << 20, mask = 0xFFF00000u;
+    for (int shift = 10; shift >= 0; shift -= 10) {
 #pragma unroll
-        for (int i = 0; i < NB2; ++i) sm.h2[tid + i * NT] = 0;
-        __syncthreads();
+      for (int i = 0; i < NB2; ++i) sm.h2[tid + i * NT] = 0;
+      __syncthreads();
+      if (gathered) {
+        for (int i = tid; i < ncand; i += NT) {
+          const uint32_t x = sm.cand[i];
+          if ((x & mask) == prefix) atomicAdd(&sm.h2[(x >> shift) & 1023u], 1u);
+        }
+      } else {
 #pragma unroll
         for (int j = 0; j < EMAX; ++j)
           if (j < mine && (key[j] & mask) == prefix) atomicAdd(&sm.h2[(key[j] >> shift) & 1023u], 1u);
-        __syncthreads();
-        uint32_t cc2[NB2];
-#pragma unroll
-        for (int i = 0; i < NB2; ++i) cc2[i] = sm.h2[1023 - NB2 * tid - i];
-        find_bin_desc<NT, NB2>(cc2, 1023, kk, sm);
-        kk -= (int)sm.above;
-        prefix |= sm.digit << shift;
-        mask |= 1023u << shift;
-        stop = ((int)sm.bin_cnt == kk);
-        __syncthreads();
       }
-      t_lo = prefix;
-      t_hi = prefix | ~mask;
+      __syncthreads();
+      uint32_t cc2[NB2];
+#pragma unroll
+      for (int i = 0; i < NB2; ++i) cc2[i] = sm.h2[1023 - NB2 * tid - i];
+      find_bin_desc<NT, NB2>(cc2, 1023, kk, sm);
+      kk -= (int)sm.above;
+      prefix |= sm.digit << shift;
+      mask |= 1023u << shift;
+      const bool stop = ((int)sm.bin_cnt == kk);
+      __syncthreads();  // sm.digit / above / bin_cnt and h2 are rewritten by the next pass
+      if (stop) break;
+    }
+    t_lo = prefix;
+    t_hi = prefix | ~mask;
+  }
+  // emission in list order: keys above the range, then the first kk keys in it
+  // (one bit per owned key; the loop visits only the taken ones)
+  static_assert(EMAX <= 32, "one mask bit per owned key");
+  uint32_t above = 0u, inside = 0u;
+#pragma unroll
+  for (int j = 0; j < EMAX; ++j) {
+    if (j < mine) {
+      above |= (uint32_t)(key[j] > t_hi) << j;
+      inside |= (uint32_t)((key[j] >= t_lo) & (key[j] <= t_hi)) << j;
     }
   }
-  emit_selected<NT, EMAX>(key, mine, first, t_lo, t_hi, kk, a.topk, sm.scan_a,
-                          [&](int pos, int i, uint32_t) { out[pos] = i; });
+  const int before = block_excl_scan<NT>((__popc(above) << 16) | __popc(inside), sm.scan_a);  // list length <= 65535
+  const int in_before = before & 0xFFFF;
+  int pos = (before >> 16) + min(in_before, kk);
+  int rin = in_before;
+  for (uint32_t m = above | inside; m != 0u; m &= m - 1u) {
+    const int j = __ffs(m) - 1;
+    const bool inr = (inside >> j) & 1u;
+    const bool tk = !inr || rin < kk;
+    rin += inr;
+    if (tk && pos < a.topk) out[pos] = first + j;  // never past the k outputs
+    pos += tk;
+  }
   if (tid == 0) a.sel_count[r] = a.topk;
 }
 
@@ -792,11 +798,11 @@ cudaError_t launch_topk_select(const SelectArgs &a, int total_q, bool two_stage,
     const dim3 grid(total_q), block(kSelThreads);
     if (a.q_groups > 1) {
       if (total_q > 1024)
-        return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 2, true>, grid, block, st, a);
-      return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 1, true>, grid, block, st, a);
+        return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, 2, true>, grid, block, st, a);
+      return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, 1, true>, grid, block, st, a);
     }
-    if (total_q > 1024) return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 2, false>, grid, block, st, a);
-    return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, false, 1, false>, grid, block, st, a);
+    if (total_q > 1024) return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, 2, false>, grid, block, st, a);
+    return launch_pdl(topk_select_hist_kernel<kSelThreads, 16, 1, false>, grid, block, st, a);
   }
   cudaError_t e = launch_pdl(topk_segment_kernel<kSegThreads, 32>, dim3(a.n_seg, total_q), dim3(kSegThreads), st, a);
   if (e != cudaSuccess) return e;
