@@ -35,7 +35,9 @@ constexpr int kGTileBytes = kGM * 128;     // one 128-row x 64-element swizzled 
 constexpr int kGOperand = kGKb * kGTileBytes;  // 64 KB: a full 128 x 256 operand
 constexpr int kGStages = 2;
 constexpr int kGThreads = 192;             // warps 0-3 epilogue, 4 TMA, 5 MMA
-constexpr int kGSmem = kGOperand * (1 + kGStages) + 256 + 1024;
+constexpr int kGStRow = 36;                // floats per row of an epilogue staging tile (16-byte aligned, conflict-free)
+constexpr int kGStageBytes = 4 * 32 * kGStRow * 4;  // 4 warps x 32 rows x 32 columns (padded)
+constexpr int kGSmem = kGOperand * (1 + kGStages) + kGStageBytes + 256 + 1024;
 constexpr uint32_t kGTmemCols = 2 * kGN;   // two fp32 accumulators
 constexpr uint64_t kGWaitNs = 2000000000ull;
 
@@ -84,7 +86,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sa = smem;                                 // query tile
   uint8_t *sb = smem + kGOperand;                     // key stages
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kGOperand * (1 + kGStages));
+  float *stage_all = reinterpret_cast<float *>(smem + kGOperand * (1 + kGStages));  // epilogue staging
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kGOperand * (1 + kGStages) + kGStageBytes);
   uint64_t *bar_a = bars + 0;
   uint64_t *bar_full = bars + 1;    // [2]
   uint64_t *bar_empty = bars + 3;   // [2]
@@ -193,10 +196,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
   } else {
     // ---------------- epilogue: warps 0-3, TMEM lanes 32w .. 32w+31 ----------------
+    // Thread = row of the tile in tensor memory; stores go through a staging
+    // tile so that 8 lanes write one row's 32 columns (128 bytes) together.
     const int row = warp * 32 + lane;
-    const int grow = row0 + row;
-    const int c_row = (row < rows) ? (ctx + (m0 + row) / G) / kBlk : 0;
-    float *dst_row = a.scores + (size_t)grow * a.score_stride;
+    const int c_row = (row < rows) ? (ctx + (m0 + row) / G) / kBlk : 0;  // visible blocks of this row
+    float *stage = stage_all + warp * 32 * kGStRow;
+    const int sub = lane >> 3, q4 = (lane & 7) * 4;  // row within a group of 4, first column of the lane
     for (int jj = 0; jj < nt; ++jj) {
       const int db = jj % 2;
       if (!wait(bar_dfull + db, (jj / 2) & 1)) break;
@@ -210,22 +215,33 @@ __global__ void __launch_bounds__(kGThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_dempty + db);
       const int n0 = (j_beg + jj) * kGN;
-      if (row < rows && n0 < c_row) {
+      if (!__any_sync(0xffffffffu, row < rows && n0 < c_row)) continue;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 4; ++c) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const int b = n0 + c * 32 + e;
-            if (b + 3 < c_row) {
-              *reinterpret_cast<float4 *>(dst_row + b) =
-                  make_float4(__uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]), __uint_as_float(v[c][e + 2]),
-                              __uint_as_float(v[c][e + 3]));
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4 *>(stage + lane * kGStRow + e) =
+              make_float4(__uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]), __uint_as_float(v[c][e + 2]),
+                          __uint_as_float(v[c][e + 3]));
+        __syncwarp();
+        const int b = n0 + c * 32 + q4;  // first of this lane's 4 blocks
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int r = it * 4 + sub;  // row of the warp's 32
+          const int cr = __shfl_sync(0xffffffffu, c_row, r);
+          if (warp * 32 + r < rows && b < cr) {
+            const float4 x = *reinterpret_cast<const float4 *>(stage + r * kGStRow + q4);
+            float *dst = a.scores + (size_t)(row0 + warp * 32 + r) * a.score_stride + b;
+            if (b + 3 < cr) {
+              *reinterpret_cast<float4 *>(dst) = x;
             } else {
-              for (int u = 0; u < 4; ++u)
-                if (b + u < c_row) dst_row[b + u] = __uint_as_float(v[c][e + u]);
+              dst[0] = x.x;
+              if (b + 1 < cr) dst[1] = x.y;
+              if (b + 2 < cr) dst[2] = x.z;
             }
           }
         }
+        __syncwarp();  // the staging tile is rewritten by the next column group
       }
     }
   }
