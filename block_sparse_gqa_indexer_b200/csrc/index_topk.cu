@@ -451,7 +451,7 @@ __device__ __forceinline__ void load_keys(const float *row, int n, int E, uint32
   float4 v[EMAX / 4];
 #pragma unroll
   for (int q = 0; q < EMAX / 4; ++q)
-    if (4 * q < E && t * E + 4 * q < n) v[q] = ld_cg(r4 + q);
+    v[q] = (4 * q < E && t * E + 4 * q < n) ? ld_cg(r4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int q = 0; q < EMAX / 4; ++q) {
     key[4 * q] = score_key(v[q].x);
@@ -536,7 +536,6 @@ __global__ void __launch_bounds__(NT, MINB) topk_select_hist_kernel(SelectArgs a
   __shared__ HistSmem sm;
   const int r = blockIdx.x;
   const int tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
   int32_t *out = a.sel + (size_t)r * a.topk;
   pdl_trigger();
   pdl_wait();  // every input (batch data, scores, histograms) is read after this point
@@ -639,14 +638,15 @@ __global__ void __launch_bounds__(NT, MINB) topk_select_hist_kernel(SelectArgs a
   // emission in list order: keys above the range, then the first kk keys in it
   // (one bit per owned key; the loop visits only the taken ones)
   static_assert(EMAX <= 32, "one mask bit per owned key");
-  uint32_t above = 0u, inside = 0u;
+  uint32_t above = 0u, ge = 0u;
 #pragma unroll
   for (int j = 0; j < EMAX; ++j) {
-    if (j < mine) {
-      above |= (uint32_t)(key[j] > t_hi) << j;
-      inside |= (uint32_t)((key[j] >= t_lo) & (key[j] <= t_hi)) << j;
-    }
+    above |= (uint32_t)(key[j] > t_hi) << j;
+    ge |= (uint32_t)(key[j] >= t_lo) << j;
   }
+  const uint32_t owned = (mine >= 32) ? 0xFFFFFFFFu : ((1u << mine) - 1u);  // keys past mine are not the row's
+  above &= owned;
+  const uint32_t inside = ge & ~above & owned;
   const int before = block_excl_scan<NT>((__popc(above) << 16) | __popc(inside), sm.scan_a);  // list length <= 65535
   const int in_before = before & 0xFFFF;
   int pos = (before >> 16) + min(in_before, kk);
