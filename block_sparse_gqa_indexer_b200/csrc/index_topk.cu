@@ -47,11 +47,8 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&vals)[1 << LOGV], in
 // token-major; otherwise one query per token.  KEY8: block keys are one-byte
 // E4M3 codes (a lane reads 8 bytes = 8 dims of a key), decoded exactly to
 // fp32 before the same FMA chain as the bf16 keys.
-// (4-row bf16 tiles, the verify batches' shape, run 3 CTAs per SM at 80
-// registers: 64 x 4 rows at 32K-128K tokens in 0.106 ms per index call
-// against 0.111 ms at 97 registers and 2 CTAs per SM)
 template <int QT, int UNROLL, bool GROUPED, bool KEY8>
-__global__ void __launch_bounds__(256, (QT == 4 && !KEY8 && !GROUPED) ? 3 : 1) index_score_kernel(IndexScoreArgs a) {
+__device__ __forceinline__ void index_score_body(const IndexScoreArgs &a) {
   constexpr int LOGV = (QT == 1) ? 3 : (QT == 2) ? 4 : 5;
   constexpr int V = 1 << LOGV;  // 8 blocks x QT queries
   pdl_trigger();  // the select may launch now; it waits for these scores before reading them
@@ -181,6 +178,20 @@ __global__ void __launch_bounds__(256, (QT == 4 && !KEY8 && !GROUPED) ? 3 : 1) i
       }
     }
   }
+}
+
+template <int QT, int UNROLL, bool GROUPED, bool KEY8>
+__global__ void __launch_bounds__(256) index_score_kernel(IndexScoreArgs a) {
+  index_score_body<QT, UNROLL, GROUPED, KEY8>(a);
+}
+
+// 4-row bf16 tiles (the verify batches' shape) capped at 80 registers so that
+// 3 CTAs share an SM: 64 x 4 rows at 32K-128K tokens in 0.106 ms per index
+// call against 0.111 ms at 97 registers and 2 CTAs per SM.  (A minimum-blocks
+// bound on the shared template would also change the other tiles' register
+// allocation.)
+__global__ void __launch_bounds__(256, 3) index_score_kernel_rows4(IndexScoreArgs a) {
+  index_score_body<4, 1, false, false>(a);
 }
 
 // Per-KV-group rows (4 indexer queries per token) on the tensor cores: the
@@ -773,7 +784,7 @@ cudaError_t launch_index_score(const IndexScoreArgs &a, int max_q, int grid_page
   } else if (qt == 2) {
     index_score_kernel<2, 2, false, false><<<grid, 256, 0, st>>>(a);
   } else {
-    index_score_kernel<4, 1, false, false><<<grid, 256, 0, st>>>(a);
+    index_score_kernel_rows4<<<grid, 256, 0, st>>>(a);
   }
   return cudaGetLastError();
 }
