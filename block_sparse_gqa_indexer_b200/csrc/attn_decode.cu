@@ -378,7 +378,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     const int st = j % NST;
     uint8_t *buf = wring + st * SB;
     // warp-uniform outcome: every lane leaves together if any lane's wait expired
-    bool landed = mbar_wait_bounded(wbar + st, (j / NST) & 1, kWaitNs);
+    // (each poll may suspend the warp for up to 1 us: one-byte KV at the
+    // 64 x 131,072 headline shape 0.1044 -> 0.1024 ms; bf16 KV unchanged)
+    bool landed = mbar_wait_bounded_hint(wbar + st, (j / NST) & 1, kWaitNs, 1000u);
     if (stall_ns != 0 && j == 0) landed = landed && mbar_wait_bounded(stall_bar, 0, stall_ns);
     if (!__all_sync(0xffffffffu, landed)) {
       timed_out = true;

@@ -173,6 +173,32 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete may
+// be suspended for up to hint_ns (it resumes when the phase completes) instead
+// of returning at once, so a waiting warp does not take issue slots.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait that sleeps between polls (suspend hint of hint_ns per poll).
+__device__ __forceinline__ bool mbar_wait_bounded_hint(uint64_t *bar, uint32_t parity, uint64_t limit_ns,
+                                                       uint32_t hint_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // 3-D tiled TMA load (no multicast) into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, int c0, int c1, int c2,
                                             uint64_t *bar, uint64_t policy) {
