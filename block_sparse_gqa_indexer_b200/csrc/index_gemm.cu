@@ -15,8 +15,10 @@
 //   * one thread issues tcgen05.mma (bf16 x bf16 -> fp32) into two tensor-memory
 //     accumulators of 128 columns, so the epilogue of one tile overlaps the
 //     MMAs of the next;
-//   * four epilogue warps read their 32 tensor-memory lanes each and store
-//     the causally visible scores (b < t / 8 of each row).
+//   * four epilogue warps read their 32 tensor-memory lanes each (a thread
+//     holds one row) and store the causally visible scores (b < t / 8 of each
+//     row) through a shared-memory staging tile, 8 lanes writing one row's
+//     128 contiguous bytes at a time.
 //
 // Integer-valued inputs give exact fp32 scores in any summation order, so the
 // selection downstream is the same as with the CUDA-core path.

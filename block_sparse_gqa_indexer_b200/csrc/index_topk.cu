@@ -519,7 +519,7 @@ constexpr int kCandMax = 2048;  // threshold bins up to this size are refined ov
 
 struct HistSmem {
   uint32_t h1[kHistBins];       // row histogram of the top 12 key bits, when not given
-  uint32_t h2[1024];            // block-wide refinement of a large threshold bin
+  uint32_t h2[1024];            // 10-bit digits of the threshold bin's keys (refinement passes)
   uint32_t cand[kCandMax];      // keys of the threshold bin (any order)
   int scan_a[32];
   int ncand;
