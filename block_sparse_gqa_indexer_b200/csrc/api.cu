@@ -446,7 +446,9 @@ s5_status attn_common(int mode, const s5_kv_desc *kv, const s5_batch_desc *b, co
     if (launch_gqa_tile(t, tpk, tpv, device_slots() / kCtasPerSm, stream) != cudaSuccess) return S5_ERR_CUDA;
     a.row_skip = t.row_skip;
   }
-  return cuda_status(launch_gqa_decode(mode, a, tk, tv, b->total_q, stream));
+  // a grid of at most one CTA per SM takes the variant with the deeper ring
+  const bool deep = (long long)a.n_split * b->total_q * kKv <= device_slots() / kCtasPerSm;
+  return cuda_status(launch_gqa_decode(mode, a, tk, tv, b->total_q, deep, stream));
 }
 
 // Workspace of every call for this batch, with `groups` indexer queries and

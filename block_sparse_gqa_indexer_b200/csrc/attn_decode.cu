@@ -53,11 +53,29 @@ constexpr int kStageBytes8 = 4 * kBlockBytes8;
 static_assert(kStages8 * kStageBytes8 == kStages * kStageBytes, "both KV widths share one ring layout");
 constexpr int kMaxStages = kStages8;
 constexpr int kQStride = kD * 2 + 16;         // padded q row (bytes): conflict-free ldmatrix
-constexpr int kRingBytes = kWarps * kStages * kStageBytes;
 constexpr int kQBytes = kHpg * kQStride;
-constexpr int kListOff = kRingBytes + kQBytes;
-constexpr int kBarOff = kListOff + 2 * kMaxList * 4;
-constexpr int kAttnSmem = kBarOff + (kWarps * kMaxStages + 1) * 8 + 1024;  // + a stall barrier, alignment slack
+// Grids that fit one CTA per SM (the smallest batches) run a deep variant with
+// kDeep times the ring stages per warp: with one CTA on an SM the shared memory
+// is there, and a warp's few block pairs are in flight together instead of one
+// HBM round trip per pair.
+constexpr int kDeep = 2;
+template <bool DEEP>
+__host__ __device__ constexpr int ring_bytes() {
+  return kWarps * kStages * kStageBytes * (DEEP ? kDeep : 1);
+}
+template <bool DEEP>
+__host__ __device__ constexpr int list_off() {
+  return ring_bytes<DEEP>() + kQBytes;
+}
+template <bool DEEP>
+__host__ __device__ constexpr int bar_off() {
+  return list_off<DEEP>() + 2 * kMaxList * 4;
+}
+template <bool DEEP>  // + a stall barrier, alignment slack
+__host__ __device__ constexpr int attn_smem() {
+  return bar_off<DEEP>() + (kWarps * kMaxStages * (DEEP ? kDeep : 1) + 1) * 8 + 1024;
+}
+static_assert(attn_smem<true>() <= 227 * 1024, "deep variant: shared memory per CTA");
 constexpr uint64_t kWaitNs = 2000000000ull;                       // 2 s per wait
 constexpr float kLazyMax = 8.0f;  // log2 units: a softmax reference max moves only when exceeded by more
 constexpr int kMaxSplitMerge = 32;
@@ -170,20 +188,20 @@ __global__ void __launch_bounds__(kD / 4) s5_combine_kernel(const AttnArgs a) {
   if (threadIdx.x == 0 && a.lse != nullptr) a.lse[rh] = lse;
 }
 
-template <int MODE, bool KV8>
+template <int MODE, bool KV8, bool DEEP>
 __global__ void __launch_bounds__(kWarps * 32, 2)
     gqa_decode_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v) {
-  constexpr int NST = KV8 ? kStages8 : kStages;         // ring stages per warp
+  constexpr int NST = (KV8 ? kStages8 : kStages) * (DEEP ? kDeep : 1);  // ring stages per warp
   constexpr int BB = KV8 ? kBlockBytes8 : kBlockBytes;  // one block of one group (K or V)
   constexpr int SB = 4 * BB;                            // one stage: K A, K B, V A, V B
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *ring = smem;
-  uint8_t *q_s = smem + kRingBytes;
-  int32_t *blist = reinterpret_cast<int32_t *>(smem + kListOff);
+  uint8_t *q_s = smem + ring_bytes<DEEP>();
+  int32_t *blist = reinterpret_cast<int32_t *>(smem + list_off<DEEP>());
   int32_t *brow = blist + kMaxList;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + bar_off<DEEP>());
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -729,22 +747,25 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
 }
 
 cudaError_t launch_gqa_decode(int mode, const AttnArgs &a, const CUtensorMap &tk, const CUtensorMap &tv,
-                              int total_q, cudaStream_t st) {
+                              int total_q, bool deep, cudaStream_t st) {
   const long long n_cta = (long long)a.n_split * total_q * kKv;
   if (n_cta > 0x7fffffffLL) return cudaErrorInvalidValue;
   dim3 grid((unsigned)n_cta);
   cudaError_t e;
-  auto kernel = (mode == kModeSparse) ? (a.kv8 ? gqa_decode_kernel<kModeSparse, true>
-                                                : gqa_decode_kernel<kModeSparse, false>)
-                                      : gqa_decode_kernel<kModeSwa, false>;
-  e = ensure_dynamic_smem(reinterpret_cast<const void *>(kernel), kAttnSmem);
+  auto kernel = (mode == kModeSparse)
+                    ? (a.kv8 ? (deep ? gqa_decode_kernel<kModeSparse, true, true> : gqa_decode_kernel<kModeSparse, true, false>)
+                             : (deep ? gqa_decode_kernel<kModeSparse, false, true>
+                                     : gqa_decode_kernel<kModeSparse, false, false>))
+                    : (deep ? gqa_decode_kernel<kModeSwa, false, true> : gqa_decode_kernel<kModeSwa, false, false>);
+  const int smem = deep ? attn_smem<true>() : attn_smem<false>();
+  e = ensure_dynamic_smem(reinterpret_cast<const void *>(kernel), smem);
   if (e != cudaSuccess) return e;
   // programmatic stream serialization: launch and barrier setup overlap the
   // previous kernel; the kernel reads no global memory before pdl_wait()
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kWarps * 32);
-  cfg.dynamicSmemBytes = kAttnSmem;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

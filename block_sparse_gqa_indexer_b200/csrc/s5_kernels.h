@@ -156,7 +156,9 @@ cudaError_t launch_gather_keys(const GatherArgs &a, int batch, cudaStream_t st);
 cudaError_t launch_index_gemm(const GemmArgs &a, const CUtensorMap &tq, const CUtensorMap &tk, int batch, int max_q,
                               cudaStream_t st);
 cudaError_t launch_topk_select(const SelectArgs &a, int total_q, bool two_stage, cudaStream_t st);
+// deep: the variant with twice the ring stages per warp (one CTA per SM), for
+// grids that fit on the SMs one CTA each
 cudaError_t launch_gqa_decode(int mode, const AttnArgs &a, const CUtensorMap &tk, const CUtensorMap &tv,
-                              int total_q, cudaStream_t st);
+                              int total_q, bool deep, cudaStream_t st);
 
 }  // namespace s5
