@@ -178,12 +178,18 @@ def test_verify_rows_match_single_token_decode(lib):
     assert float((d.lse - lse1).abs().max()) <= LSE_ABS
 
 
+@pytest.mark.parametrize("wide", [False, True])
 @pytest.mark.parametrize("fp8", [False, True])
-def test_expired_wait_is_reported_and_the_next_call_succeeds(lib, fp8):
+def test_expired_wait_is_reported_and_the_next_call_succeeds(lib, fp8, wide):
     # the workspace's test hook makes every attention CTA's first block wait
     # also wait 200 us on a barrier nothing arrives on: the kernel records
-    # S5_ERR_TIMEOUT, drains its copies in flight and returns
-    w = S.Workload(ctx=[20000, 9000, 300], nq=[1, 1, 1], seed=76)
+    # S5_ERR_TIMEOUT, drains its copies in flight and returns.  Three rows
+    # launch fewer CTAs than there are SMs (the deeper-ring variant); forty
+    # rows launch more (the default variant).
+    if wide:
+        w = S.Workload(ctx=[5000 + 97 * i for i in range(40)], nq=[1] * 40, seed=77)
+    else:
+        w = S.Workload(ctx=[20000, 9000, 300], nq=[1, 1, 1], seed=76)
     d = DeviceInputs(w, lib)
     lib.s5_index_score_topk(d.key_pool, d.batch, d.qx, S.TOPK, d.sel, d.sel_count, d.ws)
     if fp8:
