@@ -221,6 +221,16 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   // global input (batch data, q, the selection) is read after this wait
   pdl_wait();
   if (a.row_skip != nullptr && ld_cg(a.row_skip + r) != 0) return;  // row computed by the tile kernel
+  // the query tile of the group (16 heads x 192) is loaded first: its address
+  // needs only the row and group, so it is in flight during the lookups below
+  constexpr int kQv = kHpg * (kD / 8) / (kWarps * 32);  // 16-byte pieces per thread
+  static_assert(kHpg * (kD / 8) % (kWarps * 32) == 0, "query tile split evenly over the CTA");
+  uint4 qv[kQv];
+  {
+    const uint4 *qg = reinterpret_cast<const uint4 *>(a.q) + ((size_t)r * kHeads + g * kHpg) * (kD / 8);
+#pragma unroll
+    for (int x = 0; x < kQv; ++x) qv[x] = ld_cg(qg + tid + x * kWarps * 32);
+  }
   // expired-wait test hook (workspace header, zero in normal use): a nonzero
   // count of nanoseconds makes each warp's first stage wait also wait that long
   // on stall_bar and then leave through the expired-wait path below
@@ -292,55 +302,49 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
       }
     }
   };
-  // resolve this warp's items to block ids and TMA rows (lane k: items k, k+32, ...);
-  // the first 32 are resolved before the first loads are issued
-  auto resolve = [&](int k) {
-    const int li = i_beg + w_beg + k;
-    int b;
-    bool ok = true;
-    if (MODE == kModeSparse) {
-      if (li < n_sel) {
-        b = ld_cg(a.sel + (size_t)srow * a.topk + li);
-        ok = (b >= 0) && (b < c);
-      } else {
-        b = c;
+  // resolve this warp's items to block ids and TMA rows (lane k: items k, k+32,
+  // ...) in two rounds of loads, every load of a round in flight together:
+  // the selected blocks, then their pages
+  {
+    constexpr int kRes = ((kMaxList + kWarps - 1) / kWarps + 31) / 32;  // items per lane at most
+    static_assert(kRes * 32 * kWarps >= kMaxList, "a warp owns at most ceil(kMaxList / kWarps) items");
+    int bv[kRes], ph[kRes];
+#pragma unroll
+    for (int u = 0; u < kRes; ++u) {
+      const int k = lane + 32 * u, li = i_beg + w_beg + k;
+      bv[u] = (MODE == kModeSparse) ? c : b_first + li;
+      if (MODE == kModeSparse && k < w_n && li < n_sel) bv[u] = ld_cg(a.sel + (size_t)srow * a.topk + li);
+    }
+#pragma unroll
+    for (int u = 0; u < kRes; ++u) {
+      const int k = lane + 32 * u, li = i_beg + w_beg + k;
+      const bool ok = k < w_n && (MODE != kModeSparse || li >= n_sel || (bv[u] >= 0 && bv[u] < c));
+      ph[u] = -1;
+      if (ok) ph[u] = ld_cg(pt + bv[u] / kBpp);
+      if (k < w_n && !ok) bv[u] = -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kRes; ++u) {
+      const int k = lane + 32 * u;
+      if (k < w_n) {
+        const bool ok = bv[u] >= 0 && ph[u] >= 0 && ph[u] < a.num_pages;
+        if (!ok) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
+        blist[w_beg + k] = ok ? bv[u] : -1;
+        brow[w_beg + k] = ok ? ((ph[u] * kKv + g) * kPage) + (bv[u] % kBpp) * kBlk : -1;
       }
-    } else {
-      b = b_first + li;
     }
-    int row = -1;
-    if (ok) {
-      const int ph = ld_cg(pt + b / kBpp);
-      if (ph >= 0 && ph < a.num_pages) row = ((ph * kKv + g) * kPage) + (b % kBpp) * kBlk;
-      else ok = false;
-    }
-    if (!ok) record_error(a.err, S5_ERR_DEVICE_BOUNDS, r);
-    blist[w_beg + k] = ok ? b : -1;
-    brow[w_beg + k] = row;
-  };
-  if (lane < w_n) resolve(lane);
+  }
   __syncwarp();
   if (lane == 0) {
     for (int j = 0; j < NST && j < n_pairs; ++j) issue(j);
   }
-  // the query tile of the group (16 heads x 192, padded rows) is read while
-  // the first blocks are in flight: every thread's loads issued together
-  {
-    constexpr int kQv = kHpg * (kD / 8) / (kWarps * 32);  // 16-byte pieces per thread
-    static_assert(kHpg * (kD / 8) % (kWarps * 32) == 0, "query tile split evenly over the CTA");
-    const uint4 *qg = reinterpret_cast<const uint4 *>(a.q) + ((size_t)r * kHeads + g * kHpg) * (kD / 8);
-    uint4 qv[kQv];
+  // the query tile into shared memory (one-byte KV: as f16, which its MMAs take)
 #pragma unroll
-    for (int x = 0; x < kQv; ++x) qv[x] = ld_cg(qg + tid + x * kWarps * 32);
-#pragma unroll
-    for (int x = 0; x < kQv; ++x) {
-      const int i = tid + x * kWarps * 32;
-      const int h = i / (kD / 8), cc = i % (kD / 8);
-      // one-byte KV: the f16 MMAs take Q as f16
-      *reinterpret_cast<uint4 *>(q_s + h * kQStride + cc * 16) = KV8 ? bf16x8_to_f16x8(qv[x]) : qv[x];
-    }
+  for (int x = 0; x < kQv; ++x) {
+    const int i = tid + x * kWarps * 32;
+    const int h = i / (kD / 8), cc = i % (kD / 8);
+    *reinterpret_cast<uint4 *>(q_s + h * kQStride + cc * 16) = KV8 ? bf16x8_to_f16x8(qv[x]) : qv[x];
   }
-  for (int k = lane + 32; k < w_n; k += 32) resolve(k);
   __syncthreads();  // the query tile is complete
 
   // Q fragments (A operand) for the 12 k-steps of 16 dims
