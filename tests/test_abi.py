@@ -251,3 +251,35 @@ def test_fp8_append_rejects_bad_scales_before_launch(s5):
                  None) == s5.S5_ERR_INVALID_ARG
     assert f(ctypes.byref(kv), None, ctypes.byref(_batch()), fake, fake, None, 1.0, 1.0, fake, 16,
              None) == s5.S5_ERR_WORKSPACE
+
+
+def test_noalloc_limits_checked_before_anything_is_enqueued(s5):
+    # every case returns from the host checks, before the entry point looks up
+    # its scratch array or enqueues anything
+    fake = ctypes.c_void_p(0x1000)
+    ix = s5.IndexDesc(0x1000, 8, 256)
+
+    def call(b, topk=512, index=ix, q=fake):
+        return s5._lib.s5_index_score_topk_noalloc(ctypes.byref(index), ctypes.byref(b), q, topk, fake, fake, None)
+
+    # the scoring grid: 4-row tiles of one sequence on grid.z (<= 65,535), one sequence per grid.y
+    # step; histories of 3 blocks (stride 4) let the 8 MiB scratch hold 262,141 rows
+    assert call(_batch(batch=1, total_q=262141, max_q=262141, max_pages=1, max_len=32)) == s5.S5_ERR_UNSUPPORTED
+    assert call(_batch(batch=65536, total_q=65536, max_q=1, max_pages=1, max_len=32)) == s5.S5_ERR_UNSUPPORTED
+    # scores beyond the scratch: 130 rows x 16,376 fp32 = 8.5 MB > 8 MiB
+    assert call(_batch(batch=2, total_q=130, max_q=65, max_pages=2048, max_len=131000)) == s5.S5_ERR_WORKSPACE
+    # more than 16,384 history blocks need the two-stage select: max_len 131,081 is the first such length
+    assert call(_batch(batch=1, total_q=1, max_q=1, max_pages=2049, max_len=131081)) == s5.S5_ERR_WORKSPACE
+    assert call(_batch(batch=1, total_q=1, max_q=1, max_pages=2188, max_len=140000)) == s5.S5_ERR_WORKSPACE
+    # argument checks shared with the workspace entry point
+    b = _batch()
+    assert call(b, topk=0) == s5.S5_ERR_INVALID_ARG
+    assert call(b, topk=513) == s5.S5_ERR_INVALID_ARG
+    assert call(b, index=s5.IndexDesc(0x1000, 8, 128)) == s5.S5_ERR_UNSUPPORTED
+    assert call(b, index=s5.IndexDesc(0x1008, 8, 256)) == s5.S5_ERR_INVALID_ARG
+    assert call(b, q=None) == s5.S5_ERR_INVALID_ARG
+    assert call(b, q=ctypes.c_void_p(0x1004)) == s5.S5_ERR_INVALID_ARG
+    assert call(_batch(max_len=4 * 64 + 1)) == s5.S5_ERR_INVALID_ARG  # pages cannot hold max_len
+    # an empty batch enqueues nothing
+    assert s5._lib.s5_index_score_topk_noalloc(ctypes.byref(ix), ctypes.byref(_batch(total_q=0)), None, 512, None,
+                                               None, None) == s5.S5_OK
